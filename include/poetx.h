@@ -1,0 +1,179 @@
+/*
+ * poetx.h — C ABI of the POET-X linear layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer is the spectrum-preserving linear map
+ *     y = (R W0 P)^T x            (row form, token-major X [T, m]:  Y = X R W0 P)
+ * with W0 [m, n] fixed, and R, P block-stochastic orthogonal matrices
+ *     R = Psi_R^T Diag(G_R^1 .. G_R^{m/b}) Psi_R,   P = Psi_P^T Diag(G_P^1 .. G_P^{n/b}) Psi_P
+ * whose b x b blocks come from the Cayley-Neumann parameterisation
+ *     G = I + 2(Q + Q^2 + Q^3) + Q^4  of a skew-symmetric Q stored as its packed strict upper triangle.
+ * Sources (web pages):
+ *   "Reparameterized LLM Training via Orthogonal Equivalence Transformation" (POET paper notes):
+ *       §整体框架 (W_RP = R W0 P, y = W_RP^T x), §1 SPO (block-stochastic form), §2 CNP (k = 3),
+ *       §3 Merge-then-Reinitialize.
+ *   "在单张 H100 上预训练 13B 模型：POET-X 如何把正交变换的内存开销砍到 1/3" (POET-X blog):
+ *       §第一斧 input-centric evaluation, §第二斧 index permutations and merging 2 of 4 into W,
+ *       §第三斧 batch-wise block-diagonal products, §第四斧 packed triangle and the Q/Q^2 form of CNP,
+ *       §第五斧 forward steps a = G_R^T x, b = W a, z = G_P^T b.
+ *
+ * Conventions shared by every call:
+ *  - All tensor pointers are DEVICE pointers to row-major, contiguous memory owned by the caller.
+ *    The library never allocates or frees device memory; calls that need scratch take a caller
+ *    workspace whose size the matching *_workspace_bytes query returns.
+ *  - A permutation is an int32 array pi of length k with Psi[i, pi[i]] = 1: X Psi^T = X[:, pi]
+ *    (column gather) and, for C Psi = Y, Y[:, pi[i]] = C[:, i] (column scatter).
+ *  - The merged weight is W0' = Psi_R W0 Psi_P^T, i.e. W0'[i, j] = W0[perm_r[i], perm_p[j]].
+ *  - q of one block holds Q[i, j] (i < j) in row-major order of the strict upper triangle;
+ *    Q[j, i] = -Q[i, j]; b(b-1)/2 floats per block.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream). Every call only enqueues
+ *    work on it and returns; nothing synchronises, except where a comment says so.
+ *  - Errors found on the host (bad arguments, shapes, alignment, workspace) return before any
+ *    launch and leave every output untouched. POETX_ERR_CUDA reports a failed launch or runtime
+ *    call; poetx_last_error_message() gives details (per host thread).
+ *  - Pointers must be 16-byte aligned (POETX_ERR_ALIGN). Row strides are the logical widths,
+ *    which for BF16 must be multiples of 8 elements (m, n, b, T-independent).
+ *  - Outputs are overwritten (never accumulated into).
+ */
+#ifndef POETX_H
+#define POETX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  POETX_OK = 0,
+  POETX_ERR_INVALID_ARG = 1, /* a required pointer is NULL, a size is negative, an enum is unknown */
+  POETX_ERR_SHAPE = 2,       /* b does not divide m or n, or a size is outside the supported range */
+  POETX_ERR_ALIGN = 3,       /* a pointer is not 16-byte aligned */
+  POETX_ERR_DTYPE = 4,       /* dtype not supported by this call */
+  POETX_ERR_BAD_INDEX = 5,   /* poetx_validate_permutation: the array is not a permutation */
+  POETX_ERR_CUDA = 6,        /* a CUDA runtime call or kernel launch failed */
+  POETX_ERR_UNSUPPORTED = 7, /* the current device is not sm_100 */
+  POETX_ERR_WORKSPACE = 8,   /* workspace is NULL or smaller than the query says */
+  POETX_ERR_TIMEOUT = 9      /* poetx_device_status: a kernel's bounded wait expired */
+} poetx_status;
+
+typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
+
+/* One POET-X linear. Every pointer is a device pointer owned by the caller. */
+typedef struct {
+  int64_t m;       /* in-features: rows of W0 */
+  int64_t n;       /* out-features: columns of W0 */
+  int64_t b;       /* block size; must divide m and n */
+  int32_t dtype;   /* poetx_dtype of w0m, activations, saved_b, gradients and g_*_lp */
+  int32_t flags;   /* reserved, must be 0 */
+  void* w0m;       /* [m, n] merged weight W0' (see poetx_merge_permutations) */
+  int32_t* perm_r; /* [m] permutation of R */
+  int32_t* perm_p; /* [n] permutation of P */
+  float* q_r;      /* [m/b, b(b-1)/2] packed skew parameters of R */
+  float* q_p;      /* [n/b, b(b-1)/2] packed skew parameters of P */
+  float* g_r;      /* [m/b, b, b] fp32 CNP blocks of R (written by poetx_cnp_build) */
+  float* g_p;      /* [n/b, b, b] fp32 CNP blocks of P */
+  void* g_r_lp;    /* [m/b, b, b] bf16 copy of g_r; required when dtype == POETX_BF16 */
+  void* g_p_lp;    /* [n/b, b, b] bf16 copy of g_p; required when dtype == POETX_BF16 */
+} poetx_layer;
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_cnp_build — packed skew parameters -> Cayley-Neumann blocks.
+ *   G = I + 2(Q + Q^2 + Q^2 Q) + Q^2 Q^2 per block ("POET-X" blog §第四斧 item 2; the truncated
+ *   Neumann series of "Reparameterized LLM Training ..." §2 CNP with k = 3).
+ *   q      [nblocks, b(b-1)/2] fp32, read only.
+ *   g      [nblocks, b, b] fp32 output, row-major blocks (may be NULL if g_lp is given).
+ *   g_lp   [nblocks, b, b] output in lp_dtype (POETX_BF16, round-to-nearest-even), may be NULL.
+ *   workspace >= poetx_cnp_workspace_bytes(nblocks, b) bytes of device scratch.
+ *   Accuracy: fp32 output within ~1e-6 absolute of the exact polynomial for |Q| entries <= 0.05.
+ *   Errors: INVALID_ARG (q NULL, both outputs NULL, nblocks < 0, b < 2), SHAPE (b > 1024),
+ *           WORKSPACE, ALIGN, DTYPE (lp_dtype not BF16 while g_lp != NULL).
+ * ------------------------------------------------------------------------------------------- */
+size_t poetx_cnp_workspace_bytes(int64_t nblocks, int64_t b);
+poetx_status poetx_cnp_build(const float* q, int64_t nblocks, int64_t b, float* g, void* g_lp,
+                             int32_t lp_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_linear_fwd — Y = X Psi_R^T Diag(G_R) W0' Diag(G_P) Psi_P, input-centric
+ *   ("POET-X" blog §第一斧 and §第五斧; permutations as index maps, §第二斧; per-block batched
+ *   products, §第三斧). R W0 P is never formed. Steps:
+ *     A = X[:, perm_r];  A'_j = A_j G_R^j;  B = A' W0';  C_j = B_j G_P^j;  Y[:, perm_p] = C.
+ *   x       [T, m] (layer dtype), read only.        y [T, n] output.
+ *   saved_b [T, n] output: B, kept for the backward pass (may be NULL when no backward follows).
+ *   Uses L->g_r/g_p (F32) or L->g_r_lp/g_p_lp (BF16) as built by poetx_cnp_build.
+ *   BF16 layers compute in bf16 x bf16 -> fp32 on tensor cores and round A', B, C, Y to bf16.
+ *   workspace >= poetx_fwd_workspace_bytes(L, T).
+ *   Errors: INVALID_ARG, SHAPE (T < 0, b does not divide m or n), ALIGN, WORKSPACE, CUDA.
+ * ------------------------------------------------------------------------------------------- */
+size_t poetx_fwd_workspace_bytes(const poetx_layer* L, int64_t T);
+poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, void* y,
+                              void* saved_b, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_linear_bwd — exact gradient of poetx_linear_fwd for upstream dY:
+ *     dC = dY[:, perm_p];  dB_j = dC_j (G_P^j)^T;  dG_P^j = B_j^T dC_j;  dA' = dB W0'^T;
+ *     dA_j = dA'_j (G_R^j)^T;  dG_R^j = A_j^T dA'_j (A = X[:, perm_r]);  dX[:, perm_r] = dA;
+ *     dq = skew-packed gradient of the CNP polynomial at q (chain rule through G(Q)).
+ *   x [T, m], dy [T, n], saved_b [T, n] (from the forward on the same x and layer state).
+ *   dx [T, m] output (may be NULL to skip it);  dq_r [m/b, b(b-1)/2], dq_p [n/b, b(b-1)/2]
+ *   fp32 outputs (either may be NULL to skip that side). Uses L->q_r/q_p and the G blocks.
+ *   workspace >= poetx_bwd_workspace_bytes(L, T).
+ *   Errors: as poetx_linear_fwd; saved_b and dy must not be NULL.
+ * ------------------------------------------------------------------------------------------- */
+size_t poetx_bwd_workspace_bytes(const poetx_layer* L, int64_t T);
+poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* dy,
+                              const void* saved_b, int64_t T, void* dx, float* dq_r, float* dq_p,
+                              void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_merge_permutations — W0' = Psi_R W0 Psi_P^T ("POET-X" blog §第二斧: the two permutations
+ *   next to the fixed W are folded into it before the inner loop).
+ *   w0 [m, n] input, w0m [m, n] output (must not overlap w0), dtype F32 or BF16. Bit-exact copy.
+ *   perm_r [m], perm_p [n] must be permutations (not checked; see poetx_validate_permutation).
+ * ------------------------------------------------------------------------------------------- */
+poetx_status poetx_merge_permutations(const void* w0, const int32_t* perm_r,
+                                      const int32_t* perm_p, int64_t m, int64_t n, int32_t dtype,
+                                      void* w0m, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_merge_reinit — merge-then-reinitialize ("Reparameterized LLM Training ..." §3):
+ *   W <- R W P using the current L->g_r, L->g_p (call poetx_cnp_build first), new permutations
+ *   drawn from `seed`, W0' <- the new merge of W, q <- 0. In place on L->w0m, L->perm_r,
+ *   L->perm_p, L->q_r, L->q_p. The G blocks are NOT reset: rebuild them with poetx_cnp_build
+ *   (q = 0 gives G = I exactly). The layer function is preserved up to rounding of W0'.
+ *   Permutation draw: key_l[i] = SplitMix64 output i of the stream started at
+ *   SplitMix64 output l of `seed` (l = 0 for R, 1 for P); pi_l sorts indices by (key, index).
+ *   workspace >= poetx_merge_reinit_workspace_bytes(L).
+ * ------------------------------------------------------------------------------------------- */
+size_t poetx_merge_reinit_workspace_bytes(const poetx_layer* L);
+poetx_status poetx_merge_reinit(poetx_layer* L, uint64_t seed, void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/* Draw the permutation that poetx_merge_reinit would use for (seed, lane) into perm [k]. */
+poetx_status poetx_resample_permutation(uint64_t seed, int32_t lane, int64_t k, int32_t* perm,
+                                        void* stream);
+
+/* Check on the device that perm [k] is a permutation of 0..k-1. SYNCHRONISES `stream`.
+ * workspace >= 4*k bytes. Returns POETX_OK or POETX_ERR_BAD_INDEX. */
+poetx_status poetx_validate_permutation(const int32_t* perm, int64_t k, void* workspace,
+                                        size_t ws_bytes, void* stream);
+
+/* Device error flag set by kernels whose bounded waits expired (POETX_ERR_TIMEOUT), then
+ * cleared. SYNCHRONISES `stream`. */
+poetx_status poetx_device_status(void* stream);
+
+/* Tracing: when enabled, every kernel the library launches is bracketed by CUDA events on its
+ * stream. poetx_trace_read() synchronises those events and writes one line per launch,
+ * "<kernel name> <milliseconds>\n", into buf (truncated to len), then clears the record.
+ * Returns the number of launches recorded. */
+poetx_status poetx_trace_enable(int32_t on);
+int64_t poetx_trace_read(char* buf, size_t len);
+
+const char* poetx_status_string(int32_t status);
+const char* poetx_last_error_message(void);
+int32_t poetx_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* POETX_H */

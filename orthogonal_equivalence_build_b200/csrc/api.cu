@@ -1,0 +1,487 @@
+// C ABI entry points: argument checks, workspace layout and launch order of the POET-X layer.
+//
+// Forward ("POET-X" blog §第一斧/§第五斧, permutations as index maps §第二斧, batched blocks §第三斧):
+//   A = X[:, perm_r];  A'_j = A_j G_R^j;  B = A' W0';  C_j = B_j G_P^j;  Y[:, perm_p] = C.
+// Backward (exact gradient of the forward):
+//   dC = dY[:, perm_p];  dB_j = dC_j G_P^jT;  dG_P^j = B_j^T dC_j;  dA' = dB W0'^T;
+//   dA_j = dA'_j G_R^jT;  dG_R^j = A_j^T dA'_j;  dX[:, perm_r] = dA;  dq = CNP chain rule.
+#include "internal.h"
+#include "gemm.h"
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+namespace poetx {
+
+// ------------------------------------------------------------------ error text
+static thread_local std::string g_last_error;
+
+void set_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+// ------------------------------------------------------------------ tracing
+namespace {
+struct TraceRec {
+  const char* name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_trace_mu;
+bool g_trace_on = false;
+std::vector<TraceRec> g_trace;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+}  // namespace
+
+int trace_begin(const char* name, cudaStream_t s) {
+  if (!g_trace_on) return -1;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  TraceRec r{name, pool_event(), pool_event()};
+  cudaEventRecord(r.start, s);
+  g_trace.push_back(r);
+  return (int)g_trace.size() - 1;
+}
+
+void trace_end(int slot, cudaStream_t s) {
+  if (slot < 0) return;
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  if (slot < (int)g_trace.size()) cudaEventRecord(g_trace[slot].stop, s);
+}
+
+// ------------------------------------------------------------------ device error word
+__device__ int g_device_error;
+
+int* device_error_word() {
+  static int* p = nullptr;
+  if (!p) cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_device_error);
+  return p;
+}
+
+}  // namespace poetx
+
+using namespace poetx;
+
+namespace {
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+int elem_size(int32_t dt) { return dt == POETX_BF16 ? 2 : 4; }
+
+poetx_status fail(poetx_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  set_error("%s", buf);
+  return st;
+}
+
+poetx_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(POETX_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define CHECK_CUDA(expr, where)                 \
+  do {                                          \
+    cudaError_t e_ = (expr);                    \
+    if (e_ != cudaSuccess) return cuda_fail(e_, where); \
+  } while (0)
+
+// The current device must be a compute-capability 10.x part (B200 = sm_100).
+poetx_status check_device() {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  static int cached_dev = -1, cached_major = -1;
+  if (dev != cached_dev) {
+    int major = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    cached_dev = dev;
+    cached_major = major;
+  }
+  if (cached_major != 10)
+    return fail(POETX_ERR_UNSUPPORTED, "device %d has compute capability %d.x; sm_100 required",
+                dev, cached_major);
+  return POETX_OK;
+}
+
+poetx_status check_layer(const poetx_layer* L, bool need_lp) {
+  if (!L) return fail(POETX_ERR_INVALID_ARG, "layer is NULL");
+  if (L->dtype != POETX_F32 && L->dtype != POETX_BF16)
+    return fail(POETX_ERR_DTYPE, "unknown layer dtype %d", L->dtype);
+  if (L->flags != 0) return fail(POETX_ERR_INVALID_ARG, "layer flags must be 0");
+  if (L->m <= 0 || L->n <= 0 || L->b < 2)
+    return fail(POETX_ERR_SHAPE, "bad layer shape m=%lld n=%lld b=%lld", (long long)L->m,
+                (long long)L->n, (long long)L->b);
+  if (L->m % L->b || L->n % L->b)
+    return fail(POETX_ERR_SHAPE, "b=%lld must divide m=%lld and n=%lld", (long long)L->b,
+                (long long)L->m, (long long)L->n);
+  if (L->b > 1024) return fail(POETX_ERR_SHAPE, "b=%lld exceeds 1024", (long long)L->b);
+  if (L->dtype == POETX_BF16 && (L->m % 8 || L->n % 8 || L->b % 8))
+    return fail(POETX_ERR_SHAPE, "bf16 layers need m, n, b multiples of 8");
+  if (!L->w0m || !L->perm_r || !L->perm_p || !L->g_r || !L->g_p)
+    return fail(POETX_ERR_INVALID_ARG, "layer has a NULL w0m/perm/g pointer");
+  if (need_lp && L->dtype == POETX_BF16 && (!L->g_r_lp || !L->g_p_lp))
+    return fail(POETX_ERR_INVALID_ARG, "bf16 layer needs g_r_lp and g_p_lp");
+  const void* ptrs[] = {L->w0m, L->perm_r, L->perm_p, L->g_r, L->g_p, L->g_r_lp, L->g_p_lp,
+                        L->q_r, L->q_p};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(POETX_ERR_ALIGN, "layer pointer %p not 16-byte aligned", p);
+  return POETX_OK;
+}
+
+poetx_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return POETX_OK;
+  if (!ws || have < need)
+    return fail(POETX_ERR_WORKSPACE, "workspace %zu bytes < %zu required", ws ? have : 0, need);
+  if (!aligned16(ws)) return fail(POETX_ERR_ALIGN, "workspace not 16-byte aligned");
+  return POETX_OK;
+}
+
+// ---- workspace layouts (each buffer 256-byte aligned)
+struct FwdWs {
+  void *A, *A1, *B, *C;
+};
+size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
+  Arena a(base, SIZE_MAX);
+  const size_t e = (size_t)elem_size(L->dtype);
+  FwdWs w;
+  w.A = a.take(T * L->m * e);
+  w.A1 = a.take(T * L->m * e);
+  w.C = a.take(T * L->n * e);
+  w.B = a.take(T * L->n * e);  // used only when the caller does not keep B
+  if (o) *o = w;
+  return a.used;
+}
+
+struct BwdWs {
+  void *dC, *dB, *dA1, *A, *dA;
+  float *dG_r, *dG_p;
+  void* chain;
+  void* partials;
+};
+size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
+  Arena a(base, SIZE_MAX);
+  const size_t e = (size_t)elem_size(L->dtype);
+  BwdWs w;
+  w.dC = a.take(T * L->n * e);
+  w.dB = a.take(T * L->n * e);
+  w.dA1 = a.take(T * L->m * e);
+  w.A = a.take(T * L->m * e);
+  w.dA = a.take(T * L->m * e);
+  w.dG_r = static_cast<float*>(a.take((size_t)(L->m * L->b) * sizeof(float)));
+  w.dG_p = static_cast<float*>(a.take((size_t)(L->n * L->b) * sizeof(float)));
+  const size_t chain = std::max(dq_ws_bytes(L->m / L->b, L->b), dq_ws_bytes(L->n / L->b, L->b));
+  w.chain = a.take(chain);
+  const DT t = L->dtype == POETX_BF16 ? DT::BF16 : DT::F32;
+  w.partials = a.take(std::max(block_grad_ws_bytes(t, L->m, L->b, T),
+                               block_grad_ws_bytes(t, L->n, L->b, T)));
+  if (o) *o = w;
+  return a.used;
+}
+
+struct MergeWs {
+  void *N1, *M;
+  int32_t *pr_new, *pp_new, *inv, *rho_r, *rho_p;
+};
+size_t merge_layout(const poetx_layer* L, void* base, MergeWs* o) {
+  Arena a(base, SIZE_MAX);
+  const size_t e = (size_t)elem_size(L->dtype);
+  MergeWs w;
+  w.N1 = a.take(L->m * L->n * e);
+  w.M = a.take(L->m * L->n * e);
+  w.pr_new = static_cast<int32_t*>(a.take(L->m * 4));
+  w.pp_new = static_cast<int32_t*>(a.take(L->n * 4));
+  w.inv = static_cast<int32_t*>(a.take(std::max(L->m, L->n) * 4));
+  w.rho_r = static_cast<int32_t*>(a.take(L->m * 4));
+  w.rho_p = static_cast<int32_t*>(a.take(L->n * 4));
+  if (o) *o = w;
+  return a.used;
+}
+
+DT dt_of(int32_t d) { return d == POETX_BF16 ? DT::BF16 : DT::F32; }
+
+}  // namespace
+
+extern "C" {
+
+int32_t poetx_abi_version(void) { return 1; }
+
+const char* poetx_status_string(int32_t st) {
+  switch (st) {
+    case POETX_OK: return "ok";
+    case POETX_ERR_INVALID_ARG: return "invalid argument";
+    case POETX_ERR_SHAPE: return "unsupported shape";
+    case POETX_ERR_ALIGN: return "misaligned pointer";
+    case POETX_ERR_DTYPE: return "unsupported dtype";
+    case POETX_ERR_BAD_INDEX: return "not a permutation";
+    case POETX_ERR_CUDA: return "CUDA error";
+    case POETX_ERR_UNSUPPORTED: return "unsupported device";
+    case POETX_ERR_WORKSPACE: return "workspace too small";
+    case POETX_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+const char* poetx_last_error_message(void) { return g_last_error.c_str(); }
+
+poetx_status poetx_trace_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  g_trace_on = on != 0;
+  return POETX_OK;
+}
+
+int64_t poetx_trace_read(char* buf, size_t len) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  size_t off = 0;
+  if (buf && len) buf[0] = 0;
+  for (auto& r : g_trace) {
+    float ms = -1.f;
+    if (cudaEventSynchronize(r.stop) == cudaSuccess) cudaEventElapsedTime(&ms, r.start, r.stop);
+    if (buf && off + 1 < len) {
+      int w = snprintf(buf + off, len - off, "%s %.6f\n", r.name, ms);
+      if (w > 0) off = std::min(len - 1, off + (size_t)w);
+    }
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  const int64_t count = (int64_t)g_trace.size();
+  g_trace.clear();
+  return count;
+}
+
+poetx_status poetx_device_status(void* stream) {
+  poetx_status st = check_device();
+  if (st != POETX_OK) return st;
+  int* w = device_error_word();
+  if (!w) return fail(POETX_ERR_CUDA, "device error word unavailable");
+  int host = 0;
+  CHECK_CUDA(cudaMemcpyAsync(&host, w, sizeof(int), cudaMemcpyDeviceToHost, as_stream(stream)),
+             "read error word");
+  CHECK_CUDA(cudaStreamSynchronize(as_stream(stream)), "sync");
+  if (host != 0) {
+    int zero = 0;
+    CHECK_CUDA(cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice), "clear error word");
+    return fail(POETX_ERR_TIMEOUT, "device error code %d", host);
+  }
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------ CNP
+size_t poetx_cnp_workspace_bytes(int64_t nblocks, int64_t b) {
+  if (nblocks <= 0 || b < 2) return 0;
+  return cnp_ws_bytes(nblocks, b);
+}
+
+poetx_status poetx_cnp_build(const float* q, int64_t nblocks, int64_t b, float* g, void* g_lp,
+                             int32_t lp_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  if (nblocks < 0 || b < 2) return fail(POETX_ERR_INVALID_ARG, "nblocks < 0 or b < 2");
+  if (b > 1024) return fail(POETX_ERR_SHAPE, "b=%lld exceeds 1024", (long long)b);
+  if (nblocks == 0) return POETX_OK;
+  if (!q) return fail(POETX_ERR_INVALID_ARG, "q is NULL");
+  if (!g && !g_lp) return fail(POETX_ERR_INVALID_ARG, "both outputs are NULL");
+  if (g_lp && lp_dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "g_lp must be BF16");
+  if (!aligned16(q) || (g && !aligned16(g)) || (g_lp && !aligned16(g_lp)))
+    return fail(POETX_ERR_ALIGN, "cnp pointers must be 16-byte aligned");
+  poetx_status st = check_ws(workspace, ws_bytes, poetx_cnp_workspace_bytes(nblocks, b));
+  if (st != POETX_OK) return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  CHECK_CUDA(gemm_cnp_build(q, nblocks, b, g, static_cast<__nv_bfloat16*>(g_lp), workspace,
+                            as_stream(stream)),
+             "cnp_build");
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------ forward
+size_t poetx_fwd_workspace_bytes(const poetx_layer* L, int64_t T) {
+  if (!L || T < 0 || L->m <= 0 || L->n <= 0) return 0;
+  return fwd_layout(L, T, nullptr, nullptr);
+}
+
+poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, void* y,
+                              void* saved_b, void* workspace, size_t ws_bytes, void* stream) {
+  poetx_status st = check_layer(L, true);
+  if (st != POETX_OK) return st;
+  if (T < 0) return fail(POETX_ERR_SHAPE, "T < 0");
+  if (T == 0) return POETX_OK;
+  if (!x || !y) return fail(POETX_ERR_INVALID_ARG, "x or y is NULL");
+  if (!aligned16(x) || !aligned16(y) || (saved_b && !aligned16(saved_b)))
+    return fail(POETX_ERR_ALIGN, "x, y, saved_b must be 16-byte aligned");
+  if ((st = check_ws(workspace, ws_bytes, poetx_fwd_workspace_bytes(L, T))) != POETX_OK) return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  FwdWs w;
+  fwd_layout(L, T, workspace, &w);
+  void* B = saved_b ? saved_b : w.B;
+  const int e = elem_size(L->dtype);
+  const DT t = dt_of(L->dtype);
+  const int64_t m = L->m, n = L->n, b = L->b;
+  const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
+  const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
+  CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s), "fwd gather");
+  CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.A1, T, m, b, false, s), "fwd R blocks");
+  CHECK_CUDA(gemm_dense(t, w.A1, L->w0m, B, T, n, m, false, s), "fwd W0' GEMM");
+  CHECK_CUDA(gemm_blockwise(t, B, Gp, w.C, T, n, b, false, s), "fwd P blocks");
+  CHECK_CUDA(scatter_cols(w.C, y, T, n, L->perm_p, e, s), "fwd scatter");
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------ backward
+size_t poetx_bwd_workspace_bytes(const poetx_layer* L, int64_t T) {
+  if (!L || T < 0 || L->m <= 0 || L->n <= 0 || L->b < 2) return 0;
+  return bwd_layout(L, T, nullptr, nullptr);
+}
+
+poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* dy,
+                              const void* saved_b, int64_t T, void* dx, float* dq_r, float* dq_p,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  poetx_status st = check_layer(L, true);
+  if (st != POETX_OK) return st;
+  if (T < 0) return fail(POETX_ERR_SHAPE, "T < 0");
+  if ((dq_r && !L->q_r) || (dq_p && !L->q_p))
+    return fail(POETX_ERR_INVALID_ARG, "dq requested but the layer has no q");
+  if (!x || !dy || !saved_b) return fail(POETX_ERR_INVALID_ARG, "x, dy or saved_b is NULL");
+  if (!aligned16(x) || !aligned16(dy) || !aligned16(saved_b) || (dx && !aligned16(dx)) ||
+      (dq_r && !aligned16(dq_r)) || (dq_p && !aligned16(dq_p)))
+    return fail(POETX_ERR_ALIGN, "backward pointers must be 16-byte aligned");
+  if ((st = check_ws(workspace, ws_bytes, poetx_bwd_workspace_bytes(L, T))) != POETX_OK) return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  BwdWs w;
+  bwd_layout(L, T, workspace, &w);
+  const int e = elem_size(L->dtype);
+  const DT t = dt_of(L->dtype);
+  const int64_t m = L->m, n = L->n, b = L->b;
+  const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
+  const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
+  CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s), "bwd gather dY");
+  CHECK_CUDA(gemm_blockwise(t, w.dC, Gp, w.dB, T, n, b, true, s), "bwd P blocks");
+  if (dq_p)
+    CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, w.dG_p, T, n, b, w.partials, s), "bwd dG_P");
+  CHECK_CUDA(gemm_dense(t, w.dB, L->w0m, w.dA1, T, m, n, true, s), "bwd W0'^T GEMM");
+  if (dx) {
+    CHECK_CUDA(gemm_blockwise(t, w.dA1, Gr, w.dA, T, m, b, true, s), "bwd R blocks");
+    CHECK_CUDA(scatter_cols(w.dA, dx, T, m, L->perm_r, e, s), "bwd scatter dX");
+  }
+  if (dq_r) {
+    CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s), "bwd gather X");
+    CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, w.dG_r, T, m, b, w.partials, s), "bwd dG_R");
+  }
+  if (dq_r) CHECK_CUDA(gemm_dq_from_dg(L->q_r, w.dG_r, m / b, b, dq_r, w.chain, s), "dq_r");
+  if (dq_p) CHECK_CUDA(gemm_dq_from_dg(L->q_p, w.dG_p, n / b, b, dq_p, w.chain, s), "dq_p");
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------ permutations
+poetx_status poetx_merge_permutations(const void* w0, const int32_t* perm_r,
+                                      const int32_t* perm_p, int64_t m, int64_t n, int32_t dtype,
+                                      void* w0m, void* stream) {
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (m < 0 || n < 0) return fail(POETX_ERR_SHAPE, "negative size");
+  if (m == 0 || n == 0) return POETX_OK;
+  if (!w0 || !perm_r || !perm_p || !w0m) return fail(POETX_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(w0) || !aligned16(w0m) || !aligned16(perm_r) || !aligned16(perm_p))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  const size_t bytes = (size_t)(m * n * elem_size(dtype));
+  const char* a = static_cast<const char*>(w0);
+  const char* c = static_cast<const char*>(w0m);
+  if (a < c + bytes && c < a + bytes) return fail(POETX_ERR_INVALID_ARG, "w0m overlaps w0");
+  poetx_status st = check_device();
+  if (st != POETX_OK) return st;
+  CHECK_CUDA(gather_cols(w0, w0m, m, n, perm_r, perm_p, elem_size(dtype), as_stream(stream)),
+             "merge_permutations");
+  return POETX_OK;
+}
+
+poetx_status poetx_resample_permutation(uint64_t seed, int32_t lane, int64_t k, int32_t* perm,
+                                        void* stream) {
+  if (k < 0 || k > (int64_t)INT32_MAX) return fail(POETX_ERR_SHAPE, "bad length");
+  if (k == 0) return POETX_OK;
+  if (!perm) return fail(POETX_ERR_INVALID_ARG, "perm is NULL");
+  poetx_status st = check_device();
+  if (st != POETX_OK) return st;
+  CHECK_CUDA(resample_permutation(seed, lane, k, perm, as_stream(stream)), "resample");
+  return POETX_OK;
+}
+
+poetx_status poetx_validate_permutation(const int32_t* perm, int64_t k, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  if (k < 0) return fail(POETX_ERR_SHAPE, "negative length");
+  if (k == 0) return POETX_OK;
+  if (!perm) return fail(POETX_ERR_INVALID_ARG, "perm is NULL");
+  poetx_status st = check_ws(workspace, ws_bytes, (size_t)(k + 1) * 4);
+  if (st != POETX_OK) return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  int32_t* cnt = static_cast<int32_t*>(workspace);
+  CHECK_CUDA(count_permutation(perm, k, cnt, s), "validate");
+  int32_t flag = 0;
+  CHECK_CUDA(cudaMemcpyAsync(&flag, cnt + k, 4, cudaMemcpyDeviceToHost, s), "validate read");
+  CHECK_CUDA(cudaStreamSynchronize(s), "validate sync");
+  return flag ? fail(POETX_ERR_BAD_INDEX, "array is not a permutation of 0..%lld",
+                     (long long)(k - 1))
+              : POETX_OK;
+}
+
+// ------------------------------------------------------------------ merge-then-reinitialize
+size_t poetx_merge_reinit_workspace_bytes(const poetx_layer* L) {
+  if (!L || L->m <= 0 || L->n <= 0) return 0;
+  return merge_layout(L, nullptr, nullptr);
+}
+
+poetx_status poetx_merge_reinit(poetx_layer* L, uint64_t seed, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  poetx_status st = check_layer(L, true);
+  if (st != POETX_OK) return st;
+  if (!L->q_r || !L->q_p) return fail(POETX_ERR_INVALID_ARG, "layer has no q");
+  if ((st = check_ws(workspace, ws_bytes, poetx_merge_reinit_workspace_bytes(L))) != POETX_OK)
+    return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  cudaStream_t s = as_stream(stream);
+  MergeWs w;
+  merge_layout(L, workspace, &w);
+  const int e = elem_size(L->dtype);
+  const DT t = dt_of(L->dtype);
+  const int64_t m = L->m, n = L->n, b = L->b;
+  const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
+  const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
+  // M = Diag(G_R) W0' Diag(G_P), block by block
+  CHECK_CUDA(gemm_blockwise(t, L->w0m, Gp, w.N1, m, n, b, false, s), "merge W0' G_P");
+  CHECK_CUDA(gemm_blockwise_left(t, Gr, w.N1, w.M, m, n, b, s), "merge G_R (.)");
+  // new permutations, composed index maps rho = perm_old^{-1} o perm_new
+  CHECK_CUDA(resample_permutation(seed, 0, m, w.pr_new, s), "resample R");
+  CHECK_CUDA(resample_permutation(seed, 1, n, w.pp_new, s), "resample P");
+  CHECK_CUDA(compose_inverse(L->perm_r, w.pr_new, w.inv, w.rho_r, m, s), "compose R");
+  CHECK_CUDA(compose_inverse(L->perm_p, w.pp_new, w.inv, w.rho_p, n, s), "compose P");
+  // W0'_new[i, j] = M[rho_r[i], rho_p[j]]
+  CHECK_CUDA(gather_cols(w.M, L->w0m, m, n, w.rho_r, w.rho_p, e, s), "merge regather");
+  CHECK_CUDA(cudaMemcpyAsync(L->perm_r, w.pr_new, m * 4, cudaMemcpyDeviceToDevice, s), "perm_r");
+  CHECK_CUDA(cudaMemcpyAsync(L->perm_p, w.pp_new, n * 4, cudaMemcpyDeviceToDevice, s), "perm_p");
+  CHECK_CUDA(fill_zero_f32(L->q_r, m / b * (b * (b - 1) / 2), s), "zero q_r");
+  CHECK_CUDA(fill_zero_f32(L->q_p, n / b * (b * (b - 1) / 2), s), "zero q_p");
+  return POETX_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,160 @@
+// Routing of the layer's contractions: bf16 operands go to the tcgen05 kernel (umma_gemm.cu)
+// whenever its tiling fits the shape; fp32 operands (and bf16 shapes the tensor-core tiling does
+// not cover, e.g. b < 64) go to the SIMT kernel.
+#include "gemm.h"
+
+#include <algorithm>
+
+#include "umma_gemm.h"
+
+namespace poetx {
+namespace {
+
+int sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+__global__ void sum_partials_kernel(const float* __restrict__ part, float* __restrict__ out,
+                                    int64_t count, int splits) {
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < count;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    float v = 0.f;
+    for (int s = 0; s < splits; ++s) v += part[(int64_t)s * count + e];
+    out[e] = v;
+  }
+}
+
+}  // namespace
+
+int grad_splits(int64_t nb, int64_t b, int64_t rows) {
+  // enough (group, tile, split) work units for two waves, each split >= 1024 token rows
+  const int64_t tiles = nb * ((b + 127) / 128) * std::max<int64_t>(1, b / 256);
+  int64_t s = (2 * 148 + tiles - 1) / std::max<int64_t>(tiles, 1);
+  s = std::min<int64_t>(s, std::max<int64_t>(1, rows / 1024));
+  return (int)std::max<int64_t>(1, std::min<int64_t>(s, 16));
+}
+
+cudaError_t gemm_blockwise(DT t, const void* A, const void* G, void* C, int64_t rows,
+                           int64_t width, int64_t b, bool transpose_g, cudaStream_t s) {
+  if (t == DT::BF16) {
+    umma::Gemm g;
+    g.M = rows; g.N = b; g.K = b; g.groups = width / b;
+    g.A = A; g.a_rows = rows; g.a_cols = width; g.a_ld = width; g.a_mn = false;
+    g.a_gm = 0; g.a_gk = b;
+    g.B = G; g.b_rows = width; g.b_cols = b; g.b_ld = b;
+    if (transpose_g) { g.b_mn = false; g.b_gn = b; g.b_gk = 0; }   // B(k, j) = G[j][k]
+    else { g.b_mn = true; g.b_gn = 0; g.b_gk = b; }                // B(k, j) = G[k][j]
+    g.C = C; g.ldc = width; g.c_gs = b;
+    g.name = transpose_g ? "umma_blockwise_T" : "umma_blockwise";
+    if (umma::supported(g)) return umma::gemm(g, s);
+  }
+  SimtGemm g{};
+  g.M = rows; g.N = b; g.K = b; g.batch = width / b;
+  g.A = A; g.a_t = t; g.a_rs = width; g.a_cs = 1; g.a_bs = b;
+  g.B = G; g.b_t = t; g.b_bs = b * b;
+  g.b_rs = transpose_g ? 1 : b; g.b_cs = transpose_g ? b : 1;
+  g.C = C; g.c_t = t; g.c_rs = width; g.c_bs = b;
+  g.alpha = 1.f;
+  return simt_gemm(g, s);
+}
+
+cudaError_t gemm_blockwise_left(DT t, const void* G, const void* N, void* C, int64_t m,
+                                int64_t n, int64_t b, cudaStream_t s) {
+  if (t == DT::BF16) {
+    umma::Gemm g;
+    g.M = b; g.N = n; g.K = b; g.groups = m / b;
+    g.A = G; g.a_rows = m; g.a_cols = b; g.a_ld = b; g.a_mn = false; g.a_gm = b; g.a_gk = 0;
+    g.B = N; g.b_rows = m; g.b_cols = n; g.b_ld = n; g.b_mn = true; g.b_gn = 0; g.b_gk = b;
+    g.C = C; g.ldc = n; g.c_gs = b * n;
+    g.name = "umma_blockwise_left";
+    if (b % 128 == 0 && umma::supported(g)) return umma::gemm(g, s);
+  }
+  SimtGemm g{};
+  g.M = b; g.N = n; g.K = b; g.batch = m / b;
+  g.A = G; g.a_t = t; g.a_rs = b; g.a_cs = 1; g.a_bs = b * b;
+  g.B = N; g.b_t = t; g.b_rs = n; g.b_cs = 1; g.b_bs = b * n;
+  g.C = C; g.c_t = t; g.c_rs = n; g.c_bs = b * n;
+  g.alpha = 1.f;
+  return simt_gemm(g, s);
+}
+
+cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, int64_t N,
+                       int64_t K, bool w_trans, cudaStream_t s) {
+  if (t == DT::BF16) {
+    umma::Gemm g;
+    g.M = M; g.N = N; g.K = K;
+    g.A = A; g.a_rows = M; g.a_cols = K; g.a_ld = K; g.a_mn = false;
+    g.B = W;
+    if (w_trans) { g.b_rows = N; g.b_cols = K; g.b_ld = K; g.b_mn = false; }
+    else { g.b_rows = K; g.b_cols = N; g.b_ld = N; g.b_mn = true; }
+    g.C = C; g.ldc = N;
+    g.name = w_trans ? "umma_dense_W0T" : "umma_dense_W0";
+    if (umma::supported(g)) return umma::gemm(g, s);
+  }
+  SimtGemm g{};
+  g.M = M; g.N = N; g.K = K; g.batch = 1;
+  g.A = A; g.a_t = t; g.a_rs = K; g.a_cs = 1;
+  g.B = W; g.b_t = t;
+  g.b_rs = w_trans ? 1 : N; g.b_cs = w_trans ? K : 1;
+  g.C = C; g.c_t = t; g.c_rs = N;
+  g.alpha = 1.f;
+  return simt_gemm(g, s);
+}
+
+size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows) {
+  if (t != DT::BF16) return 0;
+  const int sp = grad_splits(width / b, b, rows);
+  return sp > 1 ? (size_t)sp * (size_t)(width * b) * sizeof(float) : 0;
+}
+
+cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
+                            int64_t width, int64_t b, void* partials, cudaStream_t s) {
+  if (rows == 0) return cudaMemsetAsync(dG, 0, (size_t)(width * b) * sizeof(float), s);
+  if (t == DT::BF16) {
+    const int sp = grad_splits(width / b, b, rows);
+    umma::Gemm g;
+    g.M = b; g.N = b; g.K = rows; g.groups = width / b; g.splits = sp;
+    g.A = A; g.a_rows = rows; g.a_cols = width; g.a_ld = width; g.a_mn = true;
+    g.a_gm = b; g.a_gk = 0;
+    g.B = B; g.b_rows = rows; g.b_cols = width; g.b_ld = width; g.b_mn = true;
+    g.b_gn = b; g.b_gk = 0;
+    g.out_f32 = true; g.ldc = b; g.c_gs = b * b; g.c_split = width * b;
+    g.C = sp > 1 ? partials : dG;
+    g.name = "umma_block_grad";
+    if (b % 128 == 0 && umma::supported(g) && (sp == 1 || partials)) {
+      cudaError_t e = umma::gemm(g, s);
+      if (e != cudaSuccess || sp == 1) return e;
+      const int64_t count = width * b;
+      TraceScope tr("sum_split_partials", s);
+      sum_partials_kernel<<<(int)std::min<int64_t>((count + 255) / 256, sms() * 8), 256, 0, s>>>(
+          static_cast<const float*>(partials), dG, count, sp);
+      return cudaGetLastError();
+    }
+  }
+  SimtGemm g{};
+  g.M = b; g.N = b; g.K = rows; g.batch = width / b;
+  g.A = A; g.a_t = t; g.a_rs = 1; g.a_cs = width; g.a_bs = b;
+  g.B = B; g.b_t = t; g.b_rs = width; g.b_cs = 1; g.b_bs = b;
+  g.C = dG; g.c_t = DT::F32; g.c_rs = b; g.c_bs = b * b;
+  g.alpha = 1.f;
+  return simt_gemm(g, s);
+}
+
+cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
+                           void* ws, cudaStream_t s) {
+  return cnp_build(q, nb, b, g, g_lp, ws, s);
+}
+
+cudaError_t gemm_dq_from_dg(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
+                            void* ws, cudaStream_t s) {
+  return dq_from_dg(q, dG, nb, b, dq, ws, s);
+}
+
+}  // namespace poetx

@@ -1,0 +1,31 @@
+// Contractions of the POET-X layer, routed to the tensor-core (tcgen05) kernel for bf16 operands
+// and to the SIMT kernel for fp32 operands.
+#pragma once
+#include "internal.h"
+
+namespace poetx {
+
+// C_j = A_j G_j (or A_j G_j^T), j = 0..width/b-1: A, C [rows, width] row-major, G [width/b, b, b].
+// The batch-wise block-diagonal product ("POET-X" blog §第三斧).
+cudaError_t gemm_blockwise(DT t, const void* A, const void* G, void* C, int64_t rows,
+                           int64_t width, int64_t b, bool transpose_g, cudaStream_t s);
+// C[rb + i, :] = sum_k G_r[i, k] N[rb + k, :] for row block r (C = Diag(G) N), N, C [m, n].
+cudaError_t gemm_blockwise_left(DT t, const void* G, const void* N, void* C, int64_t m,
+                                int64_t n, int64_t b, cudaStream_t s);
+// C [M, N] = A [M, K] W, with W [K, N] (w_trans = false) or W^T for W [N, K] (w_trans = true).
+cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, int64_t N,
+                       int64_t K, bool w_trans, cudaStream_t s);
+// dG_j = A_j^T B_j (contraction over the rows): A, B [rows, width], dG [width/b, b, b] fp32.
+// bf16 operands split the contraction over `grad_splits` ranges of rows; their fp32 partial
+// sums go to `partials` (block_grad_ws_bytes bytes) and are then added in a fixed order.
+int grad_splits(int64_t nb, int64_t b, int64_t rows);
+size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows);
+cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
+                            int64_t width, int64_t b, void* partials, cudaStream_t s);
+// CNP blocks and the dq chain (see cnp.cu for the algebra).
+cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
+                           void* ws, cudaStream_t s);
+cudaError_t gemm_dq_from_dg(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
+                            void* ws, cudaStream_t s);
+
+}  // namespace poetx

@@ -1,0 +1,278 @@
+// Index-array permutations ("POET-X" blog §第二斧: a permutation is an index array, applied as a
+// reorder of rows/columns instead of a product with an explicit permutation matrix).
+//
+// Column gathers/scatters move whole token rows: a CTA stages one row in shared memory with
+// coalesced 16-byte loads, then reads (gather) or writes (scatter) the shared copy through the
+// index array, and streams the result out with coalesced stores. Every value is copied
+// bit-for-bit.
+#include "internal.h"
+
+#include <algorithm>
+
+namespace poetx {
+namespace {
+
+constexpr int kPermThreads = 512;
+
+template <typename T>
+__device__ __forceinline__ void load_row_to_smem(const T* __restrict__ src, T* sm, int64_t cols) {
+  // 16-byte vector path when the row is 16-byte aligned and a multiple of 16 bytes long
+  const int64_t bytes = cols * (int64_t)sizeof(T);
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (bytes & 15) == 0) {
+    const int4* s4 = reinterpret_cast<const int4*>(src);
+    int4* d4 = reinterpret_cast<int4*>(sm);
+    for (int64_t i = threadIdx.x; i < bytes / 16; i += blockDim.x) d4[i] = __ldg(s4 + i);
+  } else {
+    for (int64_t i = threadIdx.x; i < cols; i += blockDim.x) sm[i] = src[i];
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store_row_from_smem(T* __restrict__ dst, const T* sm, int64_t cols) {
+  const int64_t bytes = cols * (int64_t)sizeof(T);
+  if ((reinterpret_cast<uintptr_t>(dst) & 15) == 0 && (bytes & 15) == 0) {
+    const int4* s4 = reinterpret_cast<const int4*>(sm);
+    int4* d4 = reinterpret_cast<int4*>(dst);
+    for (int64_t i = threadIdx.x; i < bytes / 16; i += blockDim.x) d4[i] = s4[i];
+  } else {
+    for (int64_t i = threadIdx.x; i < cols; i += blockDim.x) dst[i] = sm[i];
+  }
+}
+
+// out[r, c] = in[rmap(r), cmap[c]]: stage the source row, gather from shared memory.
+template <typename T>
+__global__ void __launch_bounds__(kPermThreads)
+gather_cols_kernel(const T* __restrict__ in, T* __restrict__ out, int64_t rows, int64_t cols,
+                   const int32_t* __restrict__ row_map, const int32_t* __restrict__ col_map) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T* src = reinterpret_cast<T*>(smem_raw);
+  T* dst = src + pad8(cols);
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    const int64_t rs = row_map ? (int64_t)row_map[r] : r;
+    load_row_to_smem(in + rs * cols, src, cols);
+    __syncthreads();
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) dst[c] = src[col_map[c]];
+    __syncthreads();
+    store_row_from_smem(out + r * cols, dst, cols);
+    __syncthreads();
+  }
+}
+
+// out[r, cmap[c]] = in[r, c]: stage the source row, scatter into a shared output row.
+template <typename T>
+__global__ void __launch_bounds__(kPermThreads)
+scatter_cols_kernel(const T* __restrict__ in, T* __restrict__ out, int64_t rows, int64_t cols,
+                    const int32_t* __restrict__ col_map) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T* src = reinterpret_cast<T*>(smem_raw);
+  T* dst = src + pad8(cols);
+  for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
+    load_row_to_smem(in + r * cols, src, cols);
+    __syncthreads();
+    for (int64_t c = threadIdx.x; c < cols; c += blockDim.x) dst[col_map[c]] = src[c];
+    __syncthreads();
+    store_row_from_smem(out + r * cols, dst, cols);
+    __syncthreads();
+  }
+}
+
+// Rows too long for shared memory: direct global gather/scatter (still bit-exact).
+template <typename T>
+__global__ void gather_cols_global(const T* __restrict__ in, T* __restrict__ out, int64_t rows,
+                                   int64_t cols, const int32_t* __restrict__ row_map,
+                                   const int32_t* __restrict__ col_map) {
+  const int64_t total = rows * cols;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    const int64_t rs = row_map ? (int64_t)row_map[r] : r;
+    out[e] = in[rs * cols + col_map[c]];
+  }
+}
+
+template <typename T>
+__global__ void scatter_cols_global(const T* __restrict__ in, T* __restrict__ out, int64_t rows,
+                                    int64_t cols, const int32_t* __restrict__ col_map) {
+  const int64_t total = rows * cols;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    out[r * cols + col_map[c]] = in[e];
+  }
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+constexpr size_t kMaxRowSmem = 200 * 1024;
+
+template <typename T>
+cudaError_t launch_gather(const void* in, void* out, int64_t rows, int64_t cols,
+                          const int32_t* row_map, const int32_t* col_map, cudaStream_t s) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const size_t smem = 2 * (size_t)pad8(cols) * sizeof(T);
+  if (smem <= kMaxRowSmem) {
+    cudaFuncSetAttribute(gather_cols_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    const int per_sm = std::max(1, (int)(220 * 1024 / std::max<size_t>(smem, 1)));
+    const int64_t grid = std::min<int64_t>(rows, (int64_t)num_sms() * std::min(per_sm, 4));
+    TraceScope t(sizeof(T) == 2 ? "perm_gather_cols_bf16" : "perm_gather_cols_f32", s);
+    gather_cols_kernel<T><<<(unsigned)grid, kPermThreads, smem, s>>>(
+        static_cast<const T*>(in), static_cast<T*>(out), rows, cols, row_map, col_map);
+  } else {
+    TraceScope t("perm_gather_cols_global", s);
+    gather_cols_global<T><<<num_sms() * 8, 256, 0, s>>>(static_cast<const T*>(in),
+                                                        static_cast<T*>(out), rows, cols,
+                                                        row_map, col_map);
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_scatter(const void* in, void* out, int64_t rows, int64_t cols,
+                           const int32_t* col_map, cudaStream_t s) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const size_t smem = 2 * (size_t)pad8(cols) * sizeof(T);
+  if (smem <= kMaxRowSmem) {
+    cudaFuncSetAttribute(scatter_cols_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    const int per_sm = std::max(1, (int)(220 * 1024 / std::max<size_t>(smem, 1)));
+    const int64_t grid = std::min<int64_t>(rows, (int64_t)num_sms() * std::min(per_sm, 4));
+    TraceScope t(sizeof(T) == 2 ? "perm_scatter_cols_bf16" : "perm_scatter_cols_f32", s);
+    scatter_cols_kernel<T><<<(unsigned)grid, kPermThreads, smem, s>>>(
+        static_cast<const T*>(in), static_cast<T*>(out), rows, cols, col_map);
+  } else {
+    TraceScope t("perm_scatter_cols_global", s);
+    scatter_cols_global<T><<<num_sms() * 8, 256, 0, s>>>(static_cast<const T*>(in),
+                                                         static_cast<T*>(out), rows, cols,
+                                                         col_map);
+  }
+  return cudaGetLastError();
+}
+
+__global__ void invert_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                              int64_t k) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < k;
+       i += (int64_t)gridDim.x * blockDim.x)
+    inv[perm[i]] = (int32_t)i;
+}
+
+__global__ void compose_kernel(const int32_t* __restrict__ inv, const int32_t* __restrict__ pn,
+                               int32_t* __restrict__ rho, int64_t k) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < k;
+       i += (int64_t)gridDim.x * blockDim.x)
+    rho[i] = inv[pn[i]];
+}
+
+// ---- counter-based SplitMix64 (Steele, Lea & Flood 2014): the i-th output of the stream that
+// starts at `state` is mix(state + (i + 1) * gamma).
+__host__ __device__ __forceinline__ uint64_t sm64_mix(uint64_t z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+__host__ __device__ __forceinline__ uint64_t sm64_output(uint64_t state, uint64_t i) {
+  return sm64_mix(state + (i + 1) * 0x9E3779B97F4A7C15ull);
+}
+
+constexpr int kRankThreads = 256;
+constexpr int kRankTile = 2048;
+
+// perm[rank(i)] = i with rank(i) = #{j : (key_j, j) < (key_i, i)}: the stable argsort of the
+// keys, computed by counting (k is at most a few tens of thousands; this runs once per merge).
+__global__ void __launch_bounds__(kRankThreads)
+rank_permutation_kernel(uint64_t stream_state, int64_t k, int32_t* __restrict__ perm) {
+  __shared__ uint64_t tile[kRankTile];
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  const uint64_t ki = (i < k) ? sm64_output(stream_state, (uint64_t)i) : 0ull;
+  int64_t rank = 0;
+  for (int64_t j0 = 0; j0 < k; j0 += kRankTile) {
+    const int64_t nj = min((int64_t)kRankTile, k - j0);
+    __syncthreads();
+    for (int t = threadIdx.x; t < nj; t += blockDim.x) tile[t] = sm64_output(stream_state, j0 + t);
+    __syncthreads();
+    if (i < k) {
+      for (int t = 0; t < nj; ++t) {
+        const uint64_t kj = tile[t];
+        rank += (kj < ki) || (kj == ki && (j0 + t) < i);
+      }
+    }
+  }
+  if (i < k) perm[rank] = (int32_t)i;
+}
+
+__global__ void count_kernel(const int32_t* __restrict__ perm, int64_t k,
+                             int32_t* __restrict__ counts) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < k;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t v = perm[i];
+    if (v < 0 || (int64_t)v >= k) atomicExch(counts + k, 1);
+    else atomicAdd(counts + v, 1);
+  }
+}
+
+__global__ void check_counts_kernel(int32_t* __restrict__ counts, int64_t k) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < k;
+       i += (int64_t)gridDim.x * blockDim.x)
+    if (counts[i] != 1) atomicExch(counts + k, 1);
+}
+
+}  // namespace
+
+cudaError_t gather_cols(const void* in, void* out, int64_t rows, int64_t cols,
+                        const int32_t* row_map, const int32_t* col_map, int elem_bytes,
+                        cudaStream_t s) {
+  if (elem_bytes == 2) return launch_gather<__nv_bfloat16>(in, out, rows, cols, row_map, col_map, s);
+  return launch_gather<float>(in, out, rows, cols, row_map, col_map, s);
+}
+
+cudaError_t scatter_cols(const void* in, void* out, int64_t rows, int64_t cols,
+                         const int32_t* col_map, int elem_bytes, cudaStream_t s) {
+  if (elem_bytes == 2) return launch_scatter<__nv_bfloat16>(in, out, rows, cols, col_map, s);
+  return launch_scatter<float>(in, out, rows, cols, col_map, s);
+}
+
+cudaError_t compose_inverse(const int32_t* perm_old, const int32_t* perm_new, int32_t* inv_tmp,
+                            int32_t* rho, int64_t k, cudaStream_t s) {
+  if (k == 0) return cudaSuccess;
+  const int grid = (int)std::min<int64_t>((k + 255) / 256, 4096);
+  {
+    TraceScope t("perm_invert", s);
+    invert_kernel<<<grid, 256, 0, s>>>(perm_old, inv_tmp, k);
+  }
+  TraceScope t("perm_compose", s);
+  compose_kernel<<<grid, 256, 0, s>>>(inv_tmp, perm_new, rho, k);
+  return cudaGetLastError();
+}
+
+cudaError_t resample_permutation(uint64_t seed, int lane, int64_t k, int32_t* perm,
+                                 cudaStream_t s) {
+  if (k == 0) return cudaSuccess;
+  const uint64_t stream_state = sm64_output(seed, (uint64_t)lane);
+  TraceScope t("perm_resample_rank", s);
+  rank_permutation_kernel<<<(unsigned)((k + kRankThreads - 1) / kRankThreads), kRankThreads, 0,
+                            s>>>(stream_state, k, perm);
+  return cudaGetLastError();
+}
+
+cudaError_t count_permutation(const int32_t* perm, int64_t k, int32_t* counts_and_flag,
+                              cudaStream_t s) {
+  cudaError_t e = cudaMemsetAsync(counts_and_flag, 0, (size_t)(k + 1) * sizeof(int32_t), s);
+  if (e != cudaSuccess) return e;
+  if (k == 0) return cudaSuccess;
+  const int grid = (int)std::min<int64_t>((k + 255) / 256, 4096);
+  TraceScope t("perm_validate", s);
+  count_kernel<<<grid, 256, 0, s>>>(perm, k, counts_and_flag);
+  check_counts_kernel<<<grid, 256, 0, s>>>(counts_and_flag, k);
+  return cudaGetLastError();
+}
+
+}  // namespace poetx

@@ -1,0 +1,503 @@
+// bf16 x bf16 -> fp32 GEMM on the 5th-generation tensor cores (tcgen05 / TMEM / TMA), sm_100a.
+//
+// One kernel serves every bf16 contraction of the layer: the W0' products (dense), the
+// batch-wise block-diagonal products A_j G_j ("POET-X" blog §第三斧: each b x b block is one
+// batch element) and the per-block gradients dG_j = A_j^T B_j (contraction over tokens, split-K).
+//
+// Structure (persistent, warp-specialised, 192 threads, one CTA per SM):
+//   warp 0      TMA producer: streams 128 x 64 A and BN x 64 B tiles into a STAGES-deep ring of
+//               128-byte-swizzled shared-memory stages (mbarrier complete_tx).
+//   warp 1      owns the TMEM allocation (2 x BN fp32 columns: two accumulators) and one lane
+//               issues tcgen05.mma (M = 128, N = BN, K = 16 per instruction); tcgen05.commit
+//               frees a stage when its MMAs retire and publishes a finished accumulator.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator (warp w reads TMEM lanes 32*(w%4)..+31),
+//               convert, store; then hand the accumulator back, so tile i's epilogue overlaps
+//               tile i+1's main loop.
+// Operands may be K-major (K contiguous) or MN-major (M/N contiguous); the shared-memory matrix
+// descriptors follow the canonical SW128 layouts (K-major: 8-row groups 1024 B apart; MN-major:
+// 64-element chunks LBO apart, 8-row K groups 1024 B apart).
+// Every mbarrier wait is bounded (a few seconds of %globaltimer); on expiry the kernel records
+// a code in the device error word, lets the other roles leave their loops, waits (bounded) for
+// its own copies and MMAs in flight, frees TMEM and returns.
+#include "umma_gemm.h"
+
+#include <cuda.h>
+
+#include <algorithm>
+#include <mutex>
+
+namespace poetx {
+namespace umma {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int kThreads = 192;
+constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s
+constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per drain wait
+
+enum : int { kErrProducer = 0x101, kErrMma = 0x102, kErrEpilogue = 0x103 };
+
+struct Params {
+  int M, N, K, groups, splits;
+  int tiles_m, tiles_n, kblocks_per_split, total_tiles;
+  int a_gm, a_gk, b_gn, b_gk;   // per-group coordinate offsets (elements)
+  void* C;
+  long long ldc, c_gs, c_split;
+  int* err;
+};
+
+// ------------------------------------------------------------------ PTX wrappers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+struct Ctl {
+  volatile int* abort;
+  int* err;
+};
+
+// Wait for `parity` on `bar`; false if the CTA is aborting or the wait expired.
+__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl c, int code,
+                                          uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 31) == 0) {
+      if (*c.abort) return false;
+      if (global_ns() - t0 > limit_ns) {
+        *c.abort = 1;
+        if (code) atomicCAS(c.err, 0, code);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, SW128, sm_100 format (version 1 at bit 46, layout 2 at 61).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+// Instruction descriptor, kind::f16: fp32 accumulate, bf16 A and B, M = 128, N = BN.
+template <int BN, bool A_MN, bool B_MN>
+__device__ __forceinline__ constexpr uint32_t instr_desc() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) |
+         ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+struct TileCoord {
+  int g, mb, nb, split;
+};
+
+__device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile) {
+  constexpr int GROUP_M = 16;
+  const int per_group = p.tiles_m * p.tiles_n;
+  const int per_split = per_group * p.groups;
+  TileCoord t;
+  t.split = tile / per_split;
+  const int r = tile - t.split * per_split;
+  t.g = r / per_group;
+  const int local = r - t.g * per_group;
+  const int band = local / (GROUP_M * p.tiles_n);
+  const int first_m = band * GROUP_M;
+  const int gm = min(GROUP_M, p.tiles_m - first_m);
+  const int within = local - band * GROUP_M * p.tiles_n;
+  t.mb = first_m + within % gm;
+  t.nb = within / gm;
+  return t;
+}
+
+template <int BN, bool A_MN, bool B_MN, bool OUT_F32, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
+                 const Params p) {
+  constexpr int A_BYTES = BM * BK * 2;
+  constexpr int B_BYTES = BN * BK * 2;
+  constexpr uint32_t TMEM_COLS = 2 * BN;  // power of two: 128, 256 or 512
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + STAGES * B_BYTES);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const Ctl ctl{abort_flag, p.err};
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(tfull + a), 1);
+      mbar_init(smem_u32(tempty + a), 4);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x) {
+        const TileCoord tc = decode_tile(p, tile);
+        const int kb0 = tc.split * p.kblocks_per_split;
+        const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
+        const int am = tc.g * p.a_gm + tc.mb * BM, ak = tc.g * p.a_gk;
+        const int bn = tc.g * p.b_gn + tc.nb * BN, bk = tc.g * p.b_gk;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_bounded(smem_u32(empty + s), ph ^ 1u, ctl, kErrProducer, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(full + s);
+          mbar_expect_tx(fb, A_BYTES + B_BYTES);
+          const int k = kb * BK;
+          if constexpr (A_MN) {
+#pragma unroll
+            for (int h = 0; h < BM / 64; ++h)
+              tma_load_2d(smem_u32(sa + s * A_BYTES + h * 64 * BK * 2), &tma_a, fb, am + 64 * h,
+                          ak + k);
+          } else {
+            tma_load_2d(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k, am);
+          }
+          if constexpr (B_MN) {
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h)
+              tma_load_2d(smem_u32(sb + s * B_BYTES + h * 64 * BK * 2), &tma_b, fb, bn + 64 * h,
+                          bk + k);
+          } else {
+            tma_load_2d(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k, bn);
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies already issued land before the CTA leaves
+        for (int j = max(0, it - STAGES); j < it; ++j)
+          wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
+                       kDrainLimitNs);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc<BN, A_MN, B_MN>();
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < p.total_tiles; tile += gridDim.x, ++tcount) {
+        const TileCoord tc = decode_tile(p, tile);
+        const int kb0 = tc.split * p.kblocks_per_split;
+        const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
+        const int acc = tcount & 1;
+        const uint32_t use = (uint32_t)(tcount >> 1);
+        if (!wait_bounded(smem_u32(tempty + acc), (use & 1u) ^ 1u, ctl, kErrMma, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_bounded(smem_u32(full + s), ph, ctl, kErrMma, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sa + s * A_BYTES), b0 = smem_u32(sb + s * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc(a0 + kk * 2048, 64 * BK * 2, 1024)
+                                     : smem_desc(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc(b0 + kk * 2048, 64 * BK * 2, 1024)
+                                     : smem_desc(b0 + kk * 32, 16, 1024);
+            umma_bf16(d, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(smem_u32(empty + s));
+        }
+        if (!ok) break;
+        umma_commit(smem_u32(tfull + acc));
+      }
+      // every MMA this thread issued has retired once `drain` completes
+      umma_commit(smem_u32(drain));
+      wait_bounded(smem_u32(drain), 0, ctl, ok ? kErrMma : 0, ok ? kWaitLimitNs : kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tcount) {
+      const TileCoord tc = decode_tile(p, tile);
+      const int acc = tcount & 1;
+      const uint32_t use = (uint32_t)(tcount >> 1);
+      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
+      tc_fence_after();
+      const int grow = tc.mb * BM + row;
+      const bool live = grow < p.M;
+      const long long base = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
+                             (long long)grow * p.ldc + (long long)tc.nb * BN;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + c), r);
+        if (live) {
+          if constexpr (OUT_F32) {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.C) + base + c);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + base + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+                  pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                  pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                  pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][cols] (cols contiguous, row stride ld elements), box {64, box_rows}.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+              int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+template <int BN>
+constexpr int stages_for() {
+  return BN == 256 ? 4 : (BN == 128 ? 6 : 8);
+}
+
+template <int BN, bool A_MN, bool B_MN, bool OUT_F32>
+cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
+  constexpr int STAGES = stages_for<BN>();
+  constexpr size_t smem = (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : BM)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : BN)) return cudaErrorInvalidValue;
+  Params p;
+  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = (int)g.groups;
+  p.tiles_m = (int)((g.M + BM - 1) / BM);
+  p.tiles_n = (int)(g.N / BN);
+  const int kblocks = (int)((g.K + BK - 1) / BK);
+  const int splits = (int)std::max<int64_t>(1, std::min<int64_t>(g.splits, kblocks));
+  p.kblocks_per_split = (kblocks + splits - 1) / splits;
+  p.splits = (kblocks + p.kblocks_per_split - 1) / p.kblocks_per_split;
+  p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
+  p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
+  p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
+  p.err = device_error_word();
+  auto kern = umma_gemm_kernel<BN, A_MN, B_MN, OUT_F32, STAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = std::min(p.total_tiles, sm_count());
+  TraceScope t(name, s);
+  kern<<<grid, kThreads, smem, s>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+template <int BN>
+cudaError_t dispatch_majors(const Gemm& g, cudaStream_t s) {
+#define POETX_UM(AM, BMJ, F)                                                                   \
+  if (g.a_mn == AM && g.b_mn == BMJ && g.out_f32 == F)                                         \
+    return launch_t<BN, AM, BMJ, F>(g, s, g.name ? g.name : "umma_gemm");
+  POETX_UM(false, false, false)
+  POETX_UM(false, true, false)
+  POETX_UM(true, true, true)
+  POETX_UM(false, false, true)
+  POETX_UM(false, true, true)
+#undef POETX_UM
+  return cudaErrorNotSupported;
+}
+
+}  // namespace
+
+bool supported(const Gemm& g) {
+  if (!encode_fn()) return false;
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.groups <= 0) return false;
+  if (g.K % BK != 0 && g.groups > 1 && g.a_gk + g.b_gk != 0) return false;
+  if (g.N % 64 != 0) return false;
+  if (g.a_cols % 8 || g.b_cols % 8 || g.a_ld % 8 || g.b_ld % 8) return false;
+  if ((reinterpret_cast<uintptr_t>(g.A) | reinterpret_cast<uintptr_t>(g.B) |
+       reinterpret_cast<uintptr_t>(g.C)) & 15)
+    return false;
+  if (g.ldc % (g.out_f32 ? 4 : 8)) return false;
+  if (g.a_cols < 64 || g.b_cols < 64) return false;
+  // coordinates must fit in int32 and offsets must keep 64-element alignment
+  const int64_t lim = (int64_t)1 << 31;
+  if (g.a_rows >= lim || g.a_cols >= lim || g.b_rows >= lim || g.b_cols >= lim) return false;
+  if ((g.a_gm | g.a_gk | g.b_gn | g.b_gk) % 64) return false;
+  return true;
+}
+
+cudaError_t gemm(const Gemm& g, cudaStream_t s) {
+  if (g.N % 256 == 0) return dispatch_majors<256>(g, s);
+  if (g.N % 128 == 0) return dispatch_majors<128>(g, s);
+  return dispatch_majors<64>(g, s);
+}
+
+}  // namespace umma
+}  // namespace poetx

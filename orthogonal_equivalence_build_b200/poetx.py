@@ -1,0 +1,258 @@
+"""Thin Python binding of libpoetx (include/poetx.h), one function per C entry point.
+
+Argument marshalling only: tensors become device pointers, the current torch
+CUDA stream is passed as the stream, workspaces are caller-owned torch
+buffers sized by the library's own queries.  Every step of the layer runs in
+the library's CUDA kernels; there is no other code path.  If the shared
+library is missing the import fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "lib", "libpoetx.so")
+
+F32, BF16 = 0, 1
+_STATUS = {0: "OK", 1: "INVALID_ARG", 2: "SHAPE", 3: "ALIGN", 4: "DTYPE", 5: "BAD_INDEX",
+           6: "CUDA", 7: "UNSUPPORTED", 8: "WORKSPACE", 9: "TIMEOUT"}
+
+
+class PoetxError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"poetx status {status} ({_STATUS.get(status, '?')}): {message}")
+        self.status = status
+
+
+class Layer(ctypes.Structure):
+    """Mirror of poetx_layer."""
+    _fields_ = [("m", ctypes.c_int64), ("n", ctypes.c_int64), ("b", ctypes.c_int64),
+                ("dtype", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("w0m", ctypes.c_void_p), ("perm_r", ctypes.c_void_p),
+                ("perm_p", ctypes.c_void_p), ("q_r", ctypes.c_void_p), ("q_p", ctypes.c_void_p),
+                ("g_r", ctypes.c_void_p), ("g_p", ctypes.c_void_p),
+                ("g_r_lp", ctypes.c_void_p), ("g_p_lp", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m orthogonal_equivalence_build_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    V, I32, I64, U64, SZ = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64,
+                            ctypes.c_size_t)
+    LP = ctypes.POINTER(Layer)
+    sig = {
+        "poetx_cnp_workspace_bytes": (SZ, [I64, I64]),
+        "poetx_cnp_build": (I32, [V, I64, I64, V, V, I32, V, SZ, V]),
+        "poetx_fwd_workspace_bytes": (SZ, [LP, I64]),
+        "poetx_linear_fwd": (I32, [LP, V, I64, V, V, V, SZ, V]),
+        "poetx_bwd_workspace_bytes": (SZ, [LP, I64]),
+        "poetx_linear_bwd": (I32, [LP, V, V, V, I64, V, V, V, V, SZ, V]),
+        "poetx_merge_permutations": (I32, [V, V, V, I64, I64, I32, V, V]),
+        "poetx_merge_reinit_workspace_bytes": (SZ, [LP]),
+        "poetx_merge_reinit": (I32, [LP, U64, V, SZ, V]),
+        "poetx_resample_permutation": (I32, [U64, I32, I64, V, V]),
+        "poetx_validate_permutation": (I32, [V, I64, V, SZ, V]),
+        "poetx_device_status": (I32, [V]),
+        "poetx_trace_enable": (I32, [I32]),
+        "poetx_trace_read": (I64, [ctypes.c_char_p, SZ]),
+        "poetx_status_string": (ctypes.c_char_p, [I32]),
+        "poetx_last_error_message": (ctypes.c_char_p, []),
+        "poetx_abi_version": (I32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = _load()
+EXPORTED = (
+    "poetx_cnp_workspace_bytes", "poetx_cnp_build", "poetx_fwd_workspace_bytes",
+    "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
+    "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
+    "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
+    "poetx_trace_enable", "poetx_trace_read", "poetx_status_string",
+    "poetx_last_error_message", "poetx_abi_version")
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise PoetxError(status, lib.poetx_last_error_message().decode(errors="replace"))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to poetx must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if nbytes == 0:
+        return workspace
+    if workspace is not None and workspace.numel() * workspace.element_size() >= nbytes:
+        return workspace
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def dtype_code(t: torch.dtype) -> int:
+    if t == torch.bfloat16:
+        return BF16
+    if t == torch.float32:
+        return F32
+    raise ValueError(f"unsupported dtype {t}")
+
+
+# ----------------------------------------------------------------------------- layer state
+class PoetxLinear:
+    """Device state of one POET-X linear (caller-owned torch tensors) plus its C descriptor.
+
+    w0m [m, n] (dtype), perm_r [m], perm_p [n] (int32), q_r [m/b, b(b-1)/2], q_p (fp32),
+    g_r [m/b, b, b], g_p (fp32) and, for bf16 layers, g_r_lp / g_p_lp (bf16).
+    """
+
+    def __init__(self, w0m: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,
+                 q_r: torch.Tensor, q_p: torch.Tensor, b: int):
+        m, n = w0m.shape
+        dev = w0m.device
+        self.b = int(b)
+        self.w0m, self.perm_r, self.perm_p = w0m, perm_r, perm_p
+        self.q_r, self.q_p = q_r, q_p
+        self.g_r = torch.empty(m // b, b, b, dtype=torch.float32, device=dev)
+        self.g_p = torch.empty(n // b, b, b, dtype=torch.float32, device=dev)
+        lp = w0m.dtype == torch.bfloat16
+        self.g_r_lp = torch.empty(m // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
+        self.g_p_lp = torch.empty(n // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
+        self.desc = Layer(m=m, n=n, b=self.b, dtype=dtype_code(w0m.dtype), flags=0,
+                          w0m=_ptr(w0m), perm_r=_ptr(perm_r), perm_p=_ptr(perm_p),
+                          q_r=_ptr(q_r), q_p=_ptr(q_p), g_r=_ptr(self.g_r), g_p=_ptr(self.g_p),
+                          g_r_lp=_ptr(self.g_r_lp), g_p_lp=_ptr(self.g_p_lp))
+
+    @property
+    def m(self) -> int:
+        return int(self.desc.m)
+
+    @property
+    def n(self) -> int:
+        return int(self.desc.n)
+
+    @property
+    def dtype(self) -> torch.dtype:
+        return self.w0m.dtype
+
+
+# ----------------------------------------------------------------------------- entry points
+def cnp_workspace_bytes(nblocks: int, b: int) -> int:
+    return int(lib.poetx_cnp_workspace_bytes(nblocks, b))
+
+
+def cnp_build(q: torch.Tensor, b: int, g: Optional[torch.Tensor] = None,
+              g_lp: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> None:
+    nb = q.shape[0]
+    ws = _workspace(cnp_workspace_bytes(nb, b), q.device, workspace)
+    _check(lib.poetx_cnp_build(_ptr(q), nb, b, _ptr(g), _ptr(g_lp), BF16, _ptr(ws),
+                               0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def layer_cnp_build(layer: PoetxLinear, workspace: Optional[torch.Tensor] = None,
+                    stream=None) -> None:
+    cnp_build(layer.q_r, layer.b, layer.g_r, layer.g_r_lp, workspace, stream)
+    cnp_build(layer.q_p, layer.b, layer.g_p, layer.g_p_lp, workspace, stream)
+
+
+def fwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:
+    return int(lib.poetx_fwd_workspace_bytes(ctypes.byref(layer.desc), T))
+
+
+def linear_fwd(layer: PoetxLinear, x: torch.Tensor, y: torch.Tensor,
+               saved_b: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    T = x.shape[0]
+    ws = _workspace(fwd_workspace_bytes(layer, T), x.device, workspace)
+    _check(lib.poetx_linear_fwd(ctypes.byref(layer.desc), _ptr(x), T, _ptr(y), _ptr(saved_b),
+                                _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def bwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:
+    return int(lib.poetx_bwd_workspace_bytes(ctypes.byref(layer.desc), T))
+
+
+def linear_bwd(layer: PoetxLinear, x: torch.Tensor, dy: torch.Tensor, saved_b: torch.Tensor,
+               dx: Optional[torch.Tensor], dq_r: Optional[torch.Tensor],
+               dq_p: Optional[torch.Tensor], workspace: Optional[torch.Tensor] = None,
+               stream=None) -> None:
+    T = x.shape[0]
+    ws = _workspace(bwd_workspace_bytes(layer, T), x.device, workspace)
+    _check(lib.poetx_linear_bwd(ctypes.byref(layer.desc), _ptr(x), _ptr(dy), _ptr(saved_b), T,
+                                _ptr(dx), _ptr(dq_r), _ptr(dq_p), _ptr(ws),
+                                0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def merge_permutations(w0: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,
+                       w0m: torch.Tensor, stream=None) -> None:
+    m, n = w0.shape
+    _check(lib.poetx_merge_permutations(_ptr(w0), _ptr(perm_r), _ptr(perm_p), m, n,
+                                        dtype_code(w0.dtype), _ptr(w0m), _stream(stream)))
+
+
+def merge_reinit_workspace_bytes(layer: PoetxLinear) -> int:
+    return int(lib.poetx_merge_reinit_workspace_bytes(ctypes.byref(layer.desc)))
+
+
+def merge_reinit(layer: PoetxLinear, seed: int, workspace: Optional[torch.Tensor] = None,
+                 stream=None) -> None:
+    ws = _workspace(merge_reinit_workspace_bytes(layer), layer.w0m.device, workspace)
+    _check(lib.poetx_merge_reinit(ctypes.byref(layer.desc), seed & ((1 << 64) - 1), _ptr(ws),
+                                  0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def resample_permutation(seed: int, lane: int, perm: torch.Tensor, stream=None) -> None:
+    _check(lib.poetx_resample_permutation(seed & ((1 << 64) - 1), lane, perm.numel(), _ptr(perm),
+                                          _stream(stream)))
+
+
+def validate_permutation(perm: torch.Tensor, stream=None) -> bool:
+    k = perm.numel()
+    ws = torch.empty(4 * (k + 1), dtype=torch.uint8, device=perm.device)
+    st = lib.poetx_validate_permutation(_ptr(perm), k, _ptr(ws), ws.numel(), _stream(stream))
+    if st == 5:
+        return False
+    _check(st)
+    return True
+
+
+def device_status(stream=None) -> None:
+    _check(lib.poetx_device_status(_stream(stream)))
+
+
+def trace_enable(on: bool = True) -> None:
+    _check(lib.poetx_trace_enable(1 if on else 0))
+
+
+def trace_read(maxlen: int = 1 << 20):
+    buf = ctypes.create_string_buffer(maxlen)
+    lib.poetx_trace_read(buf, maxlen)
+    out = []
+    for line in buf.value.decode().splitlines():
+        name, ms = line.rsplit(" ", 1)
+        out.append((name, float(ms)))
+    return out
+
+
+def abi_version() -> int:
+    return int(lib.poetx_abi_version())

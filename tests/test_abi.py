@@ -1,0 +1,113 @@
+"""The C ABI loads, exports every entry point include/poetx.h declares, and rejects bad
+arguments on the host before touching a GPU.  CPU only: no call here launches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from orthogonal_equivalence_build_b200 import poetx
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "poetx.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(poetx_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_symbols_are_exported():
+    syms = declared_symbols()
+    assert len(syms) >= 17
+    for s in syms:
+        assert hasattr(poetx.lib, s), s
+    assert set(syms) == set(poetx.EXPORTED)
+
+
+def test_abi_version_and_strings():
+    assert poetx.abi_version() == 1
+    assert poetx.lib.poetx_status_string(0) == b"ok"
+    assert poetx.lib.poetx_status_string(8) == b"workspace too small"
+
+
+def _layer(**kw):
+    base = dict(m=512, n=1024, b=64, dtype=poetx.BF16, flags=0, w0m=0x10000, perm_r=0x20000,
+                perm_p=0x30000, q_r=0x40000, q_p=0x50000, g_r=0x60000, g_p=0x70000,
+                g_r_lp=0x80000, g_p_lp=0x90000)
+    base.update(kw)
+    return poetx.Layer(**base)
+
+
+def _fwd(L, x=0x100000, T=128, y=0x200000, ws=None, wsb=0):
+    return poetx.lib.poetx_linear_fwd(ctypes.byref(L), x, T, y, None, ws, wsb, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(b=48), 2),                           # b does not divide m
+    (dict(b=1), 2),                             # b < 2
+    (dict(m=0), 2),
+    (dict(dtype=7), 4),
+    (dict(flags=1), 1),
+    (dict(w0m=None), 1),
+    (dict(g_r_lp=None), 1),                     # bf16 layer needs the bf16 copies
+    (dict(perm_r=0x20004), 3),                  # misaligned
+    (dict(b=2048, m=4096, n=4096), 2),          # b too large
+])
+def test_layer_validation(kw, status):
+    assert _fwd(_layer(**kw)) == status
+
+
+def test_forward_argument_checks():
+    L = _layer()
+    assert _fwd(L, x=None) == 1
+    assert _fwd(L, T=-1) == 2
+    assert _fwd(L, T=0) == 0                    # nothing to do, no launch
+    assert _fwd(L, y=0x200008) == 3
+    need = poetx.lib.poetx_fwd_workspace_bytes(ctypes.byref(L), 128)
+    assert need > 0
+    assert _fwd(L, ws=0x400000, wsb=need - 1) == 8
+    assert _fwd(L, ws=None, wsb=need) == 8
+
+
+def test_backward_argument_checks():
+    L = _layer()
+    bwd = poetx.lib.poetx_linear_bwd
+    assert bwd(ctypes.byref(L), 0x100000, None, 0x300000, 128, None, None, None, None, 0, None) == 1
+    L2 = _layer(q_r=None)
+    assert bwd(ctypes.byref(L2), 0x100000, 0x200000, 0x300000, 128, None, 0x500000, None,
+               None, 0, None) == 1
+    need = poetx.lib.poetx_bwd_workspace_bytes(ctypes.byref(L), 128)
+    assert bwd(ctypes.byref(L), 0x100000, 0x200000, 0x300000, 128, None, None, None,
+               0x400000, need - 1, None) == 8
+
+
+def test_cnp_argument_checks():
+    f = poetx.lib.poetx_cnp_build
+    assert f(None, 2, 64, 0x1000, None, 1, None, 0, None) == 1
+    assert f(0x1000, 2, 64, None, None, 1, None, 0, None) == 1
+    assert f(0x1000, 2, 2048, 0x2000, None, 1, None, 0, None) == 2
+    assert f(0x1000, 2, 64, 0x2000, 0x3000, 0, None, 0, None) == 4
+    assert f(0x1000, 2, 64, 0x2004, None, 1, 0x8000, 1 << 30, None) == 3
+    assert f(0x1000, 2, 64, 0x2000, None, 1, None, 0, None) == 8
+    assert f(0x1000, 0, 64, 0x2000, None, 1, None, 0, None) == 0
+
+
+def test_merge_argument_checks():
+    f = poetx.lib.poetx_merge_permutations
+    assert f(0x1000, 0x2000, 0x3000, 64, 64, 5, 0x9000, None) == 4
+    assert f(None, 0x2000, 0x3000, 64, 64, 1, 0x9000, None) == 1
+    # output overlapping the input
+    assert f(0x10000, 0x2000, 0x3000, 64, 64, 1, 0x10000 + 64, None) == 1
+    L = _layer(q_p=None)
+    need = poetx.lib.poetx_merge_reinit_workspace_bytes(ctypes.byref(_layer()))
+    assert need >= 2 * 512 * 1024 * 2
+    assert poetx.lib.poetx_merge_reinit(ctypes.byref(L), 1, 0x100000, need, None) == 1
+    assert poetx.lib.poetx_merge_reinit(ctypes.byref(_layer()), 1, 0x100000, need - 1, None) == 8
+
+
+def test_workspace_queries_scale_with_tokens():
+    L = _layer()
+    f = poetx.lib.poetx_fwd_workspace_bytes
+    assert f(ctypes.byref(L), 256) > f(ctypes.byref(L), 128) > 0
+    assert poetx.lib.poetx_fwd_workspace_bytes(None, 128) == 0

@@ -1,0 +1,184 @@
+"""GPU parity: the CUDA path through the C ABI against the float64 oracle on the same seeded
+inputs.  Bit-exact for permutations and index work; max|gpu - oracle| / max|oracle| within
+1e-5 for the fp32 CNP build and fp32 layer, within 1e-2 for the bf16 layer (y, dx, dq)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import poetx_workloads as W
+from tests.gpu_util import TOL_BF16, TOL_F32, LayerCase, poetx, rel_err
+
+pytestmark = [pytest.mark.gpu,
+              pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA GPU")]
+
+
+# ------------------------------------------------------------------ CNP
+@pytest.mark.parametrize("b,sigma,nb", [(4, 0.2, 3), (16, 0.05, 2), (64, 0.01, 8), (96, 0.01, 2),
+                                        (256, 0.005, 3), (512, 0.005, 2)])
+def test_cnp_build_matches_oracle(b, sigma, nb):
+    rng = np.random.default_rng(b)
+    q = (rng.standard_normal((nb, b * (b - 1) // 2)) * sigma).astype(np.float32)
+    qd = torch.from_numpy(q).cuda()
+    g = torch.empty(nb, b, b, device="cuda")
+    g_lp = torch.empty(nb, b, b, device="cuda", dtype=torch.bfloat16)
+    poetx.cnp_build(qd, b, g, g_lp)
+    torch.cuda.synchronize()
+    assert rel_err(g, O.cnp(q, b)) <= TOL_F32
+    # the bf16 copy is the round-to-nearest-even of the fp32 blocks
+    assert torch.equal(g_lp, g.to(torch.bfloat16))
+
+
+def test_cnp_q_zero_is_exact_identity():
+    b, nb = 128, 3
+    q = torch.zeros(nb, b * (b - 1) // 2, device="cuda")
+    g = torch.empty(nb, b, b, device="cuda")
+    g_lp = torch.empty(nb, b, b, device="cuda", dtype=torch.bfloat16)
+    poetx.cnp_build(q, b, g, g_lp)
+    eye = torch.eye(b, device="cuda").expand(nb, b, b)
+    assert torch.equal(g, eye) and torch.equal(g_lp, eye.to(torch.bfloat16))
+
+
+# ------------------------------------------------------------------ permutations
+@pytest.mark.parametrize("dt", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("m,n", [(512, 512), (256, 1536), (1000, 24)])
+def test_merge_permutations_bit_exact(dt, m, n):
+    rng = np.random.default_rng(m + n)
+    w0 = rng.standard_normal((m, n)).astype(np.float32)
+    pr, pp = rng.permutation(m).astype(np.int32), rng.permutation(n).astype(np.int32)
+    w0d = torch.from_numpy(w0).to(dt).cuda()
+    out = torch.empty_like(w0d)
+    poetx.merge_permutations(w0d, torch.from_numpy(pr).cuda(), torch.from_numpy(pp).cuda(), out)
+    ref = O.merge_permutations(w0d.cpu().float().numpy(), pr, pp)
+    assert np.array_equal(out.cpu().float().numpy(), ref)
+
+
+@pytest.mark.parametrize("seed,lane,k", [(0, 0, 1), (1, 0, 7), (1, 1, 7), (1234, 0, 512),
+                                         (2 ** 64 - 1, 1, 2048), (42, 0, 14336)])
+def test_resampled_permutation_matches_oracle(seed, lane, k):
+    perm = torch.empty(k, dtype=torch.int32, device="cuda")
+    poetx.resample_permutation(seed, lane, perm)
+    assert np.array_equal(perm.cpu().numpy(), O.resample_permutation(seed, lane, k))
+
+
+def test_validate_permutation():
+    p = torch.randperm(1000, dtype=torch.int32, device="cuda")
+    assert poetx.validate_permutation(p)
+    bad = p.clone(); bad[3] = bad[4]
+    assert not poetx.validate_permutation(bad)
+    bad = p.clone(); bad[0] = 1000
+    assert not poetx.validate_permutation(bad)
+
+
+# ------------------------------------------------------------------ bit-exact layer cases
+@pytest.mark.parametrize("key,m,b,T", [("tiny_fp32", 512, 64, 200),
+                                       ("llama1p3b_attn", 512, 128, 333),
+                                       ("llama1p3b_attn", 1024, 256, 130)])
+def test_identity_layer_is_bit_exact(key, m, b, T):
+    """q = 0 and W0 = I: G = I exactly and every product is by 1.0 or 0.0, so Y == X and
+    dX == dY bit for bit; this pins the gathers, scatters and operand layouts."""
+    c = LayerCase(key, m=m, n=m, b=b, tokens=T, q_zero=True, w0=np.eye(m, dtype=np.float32))
+    y, bsave = c.forward()
+    dx, dq_r, dq_p = c.backward(bsave)
+    torch.cuda.synchronize()
+    assert torch.equal(y, c.x)
+    assert torch.equal(dx, c.dy)
+
+
+@pytest.mark.parametrize("key,m,b,T", [("tiny_fp32", 256, 64, 77), ("llama1p3b_attn", 512, 128, 260)])
+def test_permutation_weight_is_bit_exact(key, m, b, T):
+    rng = np.random.default_rng(5)
+    s = rng.permutation(m)
+    w0 = np.zeros((m, m), dtype=np.float32)
+    w0[np.arange(m), s] = 1.0
+    c = LayerCase(key, m=m, n=m, b=b, tokens=T, q_zero=True, w0=w0)
+    y, _ = c.forward()
+    ref = torch.empty_like(c.x)
+    ref[:, torch.from_numpy(s).cuda()] = c.x
+    assert torch.equal(y, ref)
+
+
+# ------------------------------------------------------------------ layer parity
+def _check_layer(c: LayerCase, tol: float, rows=None):
+    h = c.host()
+    y, bsave = c.forward()
+    dx, dq_r, dq_p = c.backward(bsave)
+    torch.cuda.synchronize()
+    G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
+    ref = O.linear_bwd(h["X"], h["dY"], h["W0m"], h["perm_r"], h["perm_p"], G_r, G_p,
+                       h["q_r"], h["q_p"], c.b)
+    errs = {"y": rel_err(y, ref["Y"]), "dx": rel_err(dx, ref["dX"]),
+            "dq_r": rel_err(dq_r, ref["dq_r"]), "dq_p": rel_err(dq_p, ref["dq_p"])}
+    for k, e in errs.items():
+        assert e <= tol, (k, errs)
+    return errs
+
+
+def test_fp32_layer_full_tiny_workload():
+    """The tiny fp32 workload at its full size: 512x512, b = 64, 256 tokens."""
+    _check_layer(LayerCase("tiny_fp32"), TOL_F32)
+
+
+@pytest.mark.parametrize("m,n,b,T", [(512, 768, 64, 100), (1024, 512, 128, 257)])
+def test_fp32_layer_shapes(m, n, b, T):
+    _check_layer(LayerCase("tiny_fp32", m=m, n=n, b=b, tokens=T), TOL_F32)
+
+
+@pytest.mark.parametrize("key,m,n,b,T", [
+    ("llama1p3b_attn", 1024, 1024, 256, 333),
+    ("llama8b_up_proj", 1024, 3584, 512, 300),
+    ("llama8b_decoder", 512, 1536, 256, 129),
+    ("llama1p3b_attn", 512, 512, 128, 1),
+])
+def test_bf16_layer_parity(key, m, n, b, T):
+    _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), TOL_BF16)
+
+
+# ------------------------------------------------------------------ merge-then-reinitialize
+@pytest.mark.parametrize("key,m,n,b,tol", [("tiny_fp32", None, None, None, TOL_F32),
+                                           ("llama1p3b_attn", 512, 768, 128, TOL_BF16)])
+def test_merge_reinit_matches_oracle(key, m, n, b, tol):
+    c = LayerCase(key, m=m, n=n, b=b, tokens=64, q_scale=4.0)
+    h = c.host()
+    y0, _ = c.forward()
+    seed = 0xC0FFEE
+    poetx.merge_reinit(c.layer, seed)
+    torch.cuda.synchronize()
+    ref = O.merge_reinit(h["W0m"], h["perm_r"], h["perm_p"], h["q_r"], h["q_p"], c.b, seed)
+    assert np.array_equal(c.perm_r.cpu().numpy(), ref["perm_r"])
+    assert np.array_equal(c.perm_p.cpu().numpy(), ref["perm_p"])
+    assert torch.count_nonzero(c.q_r) == 0 and torch.count_nonzero(c.q_p) == 0
+    assert rel_err(c.layer.w0m, ref["W0m"]) <= tol
+    # the layer function survives the merge (q = 0 now, so G = I)
+    poetx.layer_cnp_build(c.layer)
+    y1, _ = c.forward()
+    torch.cuda.synchronize()
+    assert rel_err(y1, y0.double().cpu().numpy()) <= (tol if tol > TOL_F32 else 1e-5)
+
+
+# ------------------------------------------------------------------ full-size sampled checks
+@pytest.mark.parametrize("key", ["llama1p3b_attn", "llama8b_up_proj"])
+def test_full_size_sampled(key):
+    """Full workload sizes: sampled token rows of Y and dX against the oracle row by row, and
+    dq against the oracle restricted to the sampled rows (dY is zero elsewhere)."""
+    c = LayerCase(key)
+    h = c.host()
+    rows = np.sort(np.random.default_rng(0).choice(c.T, 12, replace=False))
+    G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
+    y, bsave = c.forward()
+    dx, _, _ = c.backward(bsave)
+    torch.cuda.synchronize()
+    Xs, dYs = h["X"][rows], h["dY"][rows]
+    y_ref = O.linear_fwd_rows(Xs, h["W0m"], h["perm_r"], h["perm_p"], G_r, G_p)
+    dx_ref = O.linear_dx_rows(dYs, h["W0m"], h["perm_r"], h["perm_p"], G_r, G_p)
+    assert rel_err(y[rows], y_ref) <= TOL_BF16
+    assert rel_err(dx[rows], dx_ref) <= TOL_BF16
+    dy_sparse = torch.zeros_like(c.dy)
+    idx = torch.from_numpy(rows).cuda()
+    dy_sparse[idx] = c.dy[idx]
+    _, dq_r, dq_p = c.backward(bsave, dy=dy_sparse)
+    torch.cuda.synchronize()
+    ref = O.linear_bwd(Xs, dYs, h["W0m"], h["perm_r"], h["perm_p"], G_r, G_p, h["q_r"],
+                       h["q_p"], c.b)
+    assert rel_err(dq_r, ref["dq_r"]) <= TOL_BF16
+    assert rel_err(dq_p, ref["dq_p"]) <= TOL_BF16
