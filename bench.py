@@ -1,0 +1,411 @@
+"""Benchmark of the POET-X linear layer step (CNP rebuild + forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY] [--tokens T]
+                    [--impl ours|reference]
+
+One step is the whole hot path over one batch: poetx_cnp_build for R and P, poetx_linear_fwd,
+poetx_linear_bwd (dx, dq_r, dq_p).  Inputs are synthetic (seeded, poetx_workloads) and resident
+in HBM before the timed region.  For N > 1 (torchrun, one rank per GPU) every rank runs the step
+on its own tokens (weak scaling) and the packed dq gradients are summed over ranks with NCCL,
+as data-parallel training does.  Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle on the host cores instead (a bounded sample of the
+same workload per step); under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import poetx_workloads as W  # noqa: E402
+
+METRIC = "POET-X linear fwd+bwd tokens/s at Llama-8B shapes; % of 1-B200 roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ----------------------------------------------------------------------------- helpers
+def env_rank():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def layer_flops(T, m, n, b, cnp=True):
+    """Algorithmic FLOPs of one step: fwd 2T(mb+mn+nb), bwd dx 2T(mn+mb+nb), dG 2T(mb+nb),
+    CNP 2 products per block (S = QQ and S(2I+2Q+S)), dq 4 products per block."""
+    f = 2 * T * (m * b + m * n + n * b) * 2 + 2 * T * (m * b + n * b)
+    nblk = m // b + n // b
+    if cnp:
+        f += nblk * (2 * 2 * b ** 3 + 4 * 2 * b ** 3)
+    return f
+
+
+def layer_bytes(T, m, n, b, e=2):
+    """Algorithmic HBM bytes of one step: boundary tensors plus the saved B.
+    fwd reads X, W0', G and writes Y, B; bwd reads dY, X, B, W0', G and writes dX;
+    q, G, dq in fp32."""
+    gblk = (m // b + n // b) * b * b
+    qn = (m // b + n // b) * b * (b - 1) // 2
+    fwd = e * (T * m + m * n + T * n + T * n) + e * gblk
+    bwd = e * (T * n + T * m + T * n + m * n + T * m) + e * gblk
+    cnp = 4 * qn + 4 * gblk + 2 * gblk
+    dq = 4 * qn * 2
+    return fwd + bwd + cnp + dq
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], 0.0, set()
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = max(smax, float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names[1:], parts[5:9]):
+                if v.lower() in ("active", "1"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle arm
+def oracle_step_sample(wl, T_sample: int):
+    """One float64 oracle step (CNP of R and P, forward, backward with dq) of the workload's
+    first linear on T_sample tokens.  Returns (seconds, tokens)."""
+    import oracle as O
+    p = W.layer_params(wl)
+    a = W.layer_acts(wl, tokens=T_sample)
+    W0m = O.merge_permutations(p["W0"], p["perm_r"], p["perm_p"])
+    t0 = time.perf_counter()
+    G_r, G_p = O.cnp(p["q_r"], wl.b), O.cnp(p["q_p"], wl.b)
+    O.linear_bwd(a["X"], a["dY"], W0m, p["perm_r"], p["perm_p"], G_r, G_p, p["q_r"], p["q_p"],
+                 wl.b)
+    return time.perf_counter() - t0, T_sample
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads") for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, T_sample):
+    dt, tok = oracle_step_sample(wl, T_sample)
+    return {"value": tok / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"one float64 oracle step (CNP + fwd + bwd with dq) of the {wl.key} layer "
+                      f"on {T_sample} of its {wl.tokens} tokens: {dt:.2f} s",
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank, _, world = env_rank()
+    if rank != 0:
+        return 0
+    wl = W.WORKLOADS[args.workload]
+    lin = wl.linears[0]
+    T_sample = args.ref_tokens
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, _ = oracle_step_sample(wl, T_sample)
+        if i >= args.warmup:
+            times.append(dt)
+    sec = statistics.mean(times)
+    value = T_sample / sec
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.key, "m": lin.m, "n": lin.n, "b": wl.b,
+                   "tokens_per_step": T_sample, "parallelism": "none (host cores)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle",
+                         "sample": f"float64 oracle step on {T_sample} of {wl.tokens} tokens"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from orthogonal_equivalence_build_b200 import poetx
+
+    rank, local, world = env_rank()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    wl = W.WORKLOADS[args.workload]
+    lin = wl.linears[0]
+    m, n, b = lin.m, lin.n, wl.b
+    T = args.tokens or wl.tokens
+    dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    esz = 2 if dt == torch.bfloat16 else 4
+
+    # ---- inputs: same layer on every rank, each rank its own tokens
+    p = W.layer_params(wl)
+    a = W.layer_acts(wl, tokens=T, seed=W.WORKLOAD_SEED[wl.key] * 1000 + rank)
+    w0 = torch.from_numpy(p["W0"]).to(dt).to(dev)
+    pr = torch.from_numpy(p["perm_r"]).to(dev)
+    pp = torch.from_numpy(p["perm_p"]).to(dev)
+    q_r = torch.from_numpy(p["q_r"]).to(dev)
+    q_p = torch.from_numpy(p["q_p"]).to(dev)
+    x_host = torch.from_numpy(a["X"]).to(dt).pin_memory()
+    dy_host = torch.from_numpy(a["dY"]).to(dt).pin_memory()
+    del a
+    x = x_host.to(dev)
+    dy = dy_host.to(dev)
+    w0m = torch.empty_like(w0)
+    poetx.merge_permutations(w0, pr, pp, w0m)
+    del w0
+    layer = poetx.PoetxLinear(w0m, pr, pp, q_r, q_p, b)
+    y = torch.empty(T, n, dtype=dt, device=dev)
+    bsave = torch.empty(T, n, dtype=dt, device=dev)
+    dx = torch.empty(T, m, dtype=dt, device=dev)
+    dq_r = torch.empty_like(q_r)
+    dq_p = torch.empty_like(q_p)
+    ws = torch.empty(max(poetx.fwd_workspace_bytes(layer, T), poetx.bwd_workspace_bytes(layer, T),
+                         poetx.cnp_workspace_bytes(max(m, n) // b, b)),
+                     dtype=torch.uint8, device=dev)
+    flat_dq = torch.empty(dq_r.numel() + dq_p.numel(), device=dev) if world > 1 else None
+    stream = torch.cuda.current_stream(dev)
+    flush = None
+    if (x.numel() + dy.numel()) * esz <= L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(xin, dyin):
+        poetx.layer_cnp_build(layer, ws)
+        poetx.linear_fwd(layer, xin, y, bsave, ws)
+        poetx.linear_bwd(layer, xin, dyin, bsave, dx, dq_r, dq_p, ws)
+        if world > 1:
+            flat_dq[:dq_r.numel()].copy_(dq_r.view(-1))
+            flat_dq[dq_r.numel():].copy_(dq_p.view(-1))
+            dist.all_reduce(flat_dq)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step(x, dy)
+    torch.cuda.synchronize()
+    poetx.device_status()
+
+    # ---- timed region (device time, per-step CUDA events, kernel trace on)
+    sampler = ClockSampler(local) if rank == 0 or True else None
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    poetx.trace_read()
+    poetx.trace_enable(True)
+    sampler.start()
+    for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
+        ev[i][0].record(stream)
+        step(x, dy)
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    poetx.trace_enable(False)
+    trace = poetx.trace_read()
+    step_ms = [s.elapsed_time(e) for s, e in ev]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = T * world * args.steps / (total_ms / 1e3)
+
+    # ---- dominant kernel: the two W0' GEMMs
+    w0_launches = [ms for name, ms in trace if name in ("umma_dense_W0", "umma_dense_W0T")]
+    launches = len(trace)
+    peaks, peak_src = measured_peaks()
+    roofline = None
+    if w0_launches:
+        avg_ms = statistics.mean(w0_launches)
+        flops = 2.0 * T * m * n
+        achieved = flops / (avg_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "kernel": "umma_dense_W0 / umma_dense_W0T (B = A' W0', dA' = dB W0'^T)",
+                    "peak_source": f"{peak_src} bf16_tflops_sustained",
+                    "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
+                    "avg_launch_ms": avg_ms, "launches": len(w0_launches)}
+        tr = os.path.join(ROOT, "profiles", "traffic.txt")
+        if os.path.exists(tr):
+            for ln in open(tr):
+                parts = ln.split()
+                if len(parts) >= 3 and parts[0] == "umma_dense" and parts[1] == str(T):
+                    roofline["traffic"] = float(parts[2])
+    F = layer_flops(T, m, n, b)
+    Bb = layer_bytes(T, m, n, b, esz)
+    t_roof = max(F / (peaks["bf16_tflops"] * 1e12), Bb / (peaks["hbm_gbs"] * 1e9))
+    per_kernel = {}
+    for name, ms in trace:
+        per_kernel[name] = per_kernel.get(name, 0.0) + ms
+
+    # ---- end to end through the API: pinned host inputs in, dq out, every step
+    dq_host = torch.empty(dq_r.numel() + dq_p.numel(), dtype=torch.float32).pin_memory()
+    x_dev2 = torch.empty_like(x)
+    dy_dev2 = torch.empty_like(dy)
+    e2e_steps = max(2, min(args.steps, 5))
+    for _ in range(1):
+        x_dev2.copy_(x_host, non_blocking=True)
+        dy_dev2.copy_(dy_host, non_blocking=True)
+        step(x_dev2, dy_dev2)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        x_dev2.copy_(x_host, non_blocking=True)
+        dy_dev2.copy_(dy_host, non_blocking=True)
+        step(x_dev2, dy_dev2)
+        dq_host[:dq_r.numel()].copy_(dq_r.view(-1), non_blocking=True)
+        dq_host[dq_r.numel():].copy_(dq_p.view(-1), non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": (x.numel() + dy.numel()) * esz,
+           "d2h_bytes_per_step": dq_host.numel() * 4}
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(wl, args.ref_tokens)
+            cpu.pop("seconds", None)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": {"workload": wl.key, "m": m, "n": n, "b": b, "tokens_per_gpu": T,
+                       "global_batch_tokens": T * world, "parallelism": f"dp{world}",
+                       "step": "cnp_build(R,P) + linear_fwd + linear_bwd(dx, dq)"
+                               + (" + NCCL all-reduce of dq" if world > 1 else ""),
+                       "l2": ("inputs larger than L2: X + dY = "
+                              f"{(x.numel() + dy.numel()) * esz / 2**20:.0f} MiB per step")
+                       if flush is None else "L2 flushed (2x126 MiB write) between steps"},
+            "tflops": F * world / (ms_per_step / 1e3) / 1e12,
+            "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_per_step,
+                              "flops": F, "bytes": Bb, "peaks": peak_src},
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clocks,
+            "kernel_ms_per_step": {k: v / args.steps for k, v in sorted(per_kernel.items(),
+                                                                        key=lambda kv: -kv[1])},
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama8b_up_proj", choices=list(W.WORKLOADS))
+    ap.add_argument("--tokens", type=int, default=0, help="override tokens per GPU")
+    ap.add_argument("--ref-tokens", type=int, default=256,
+                    help="tokens in the oracle's bounded sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3 and args.impl == "ours" and not os.environ.get("POETX_BENCH_ALLOW_SHORT"):
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

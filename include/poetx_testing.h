@@ -1,0 +1,35 @@
+/*
+ * poetx_testing.h — kernel-level test hook of libpoetx (not needed by users of the layer).
+ *
+ * poetx_testing_gemm_bf16 runs the library's bf16 tensor-core contraction (tcgen05.mma with TMEM
+ * accumulators, operands staged by TMA) on one plain product, so unit tests can compare the
+ * kernel against a reference matmul for each operand layout:
+ *     C[i, j] = sum_k A(i, k) B(k, j),  0 <= i < M, 0 <= j < N, 0 <= k < K
+ *   A: bf16 device tensor [a_rows][a_cols] row-major.  a_mn = 0: A(i, k) = A[i][k] (K-major,
+ *      a_rows >= M rows, a_cols = K);  a_mn = 1: A(i, k) = A[k][i] (M-major, a_rows = K).
+ *   B: bf16 device tensor [b_rows][b_cols].  b_mn = 0: B(k, j) = B[j][k] (K-major, b_cols = K);
+ *      b_mn = 1: B(k, j) = B[k][j] (N-major, b_rows = K).
+ *   C: [M][ldc] row-major, fp32 (c_f32 = 1) or bf16 (c_f32 = 0, round-to-nearest-even).
+ *   splits > 1 splits K into that many ranges of whole 64-wide K blocks and writes fp32
+ *   partial products to C + s * M * ldc (c_f32 must be 1); the caller adds them. A count that
+ *   would leave a range empty (e.g. 5 ranges over 16 blocks) is rejected with INVALID_ARG.
+ * Returns POETX_ERR_UNSUPPORTED when the tensor-core tiling does not cover the shape
+ * (N % 64 != 0, K-major extents < 64, misaligned pointers or strides); it never falls back.
+ * Asynchronous on `stream`.
+ */
+#ifndef POETX_TESTING_H
+#define POETX_TESTING_H
+#include "poetx.h"
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, int64_t a_cols, int32_t a_mn,
+                                     const void* B, int64_t b_rows, int64_t b_cols, int32_t b_mn,
+                                     int64_t M, int64_t N, int64_t K, void* C, int32_t c_f32,
+                                     int64_t ldc, int32_t splits, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -193,9 +193,10 @@ size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   w.dA = a.take(T * L->m * e);
   w.dG_r = static_cast<float*>(a.take((size_t)(L->m * L->b) * sizeof(float)));
   w.dG_p = static_cast<float*>(a.take((size_t)(L->n * L->b) * sizeof(float)));
-  const size_t chain = std::max(dq_ws_bytes(L->m / L->b, L->b), dq_ws_bytes(L->n / L->b, L->b));
-  w.chain = a.take(chain);
   const DT t = L->dtype == POETX_BF16 ? DT::BF16 : DT::F32;
+  const size_t chain =
+      std::max(gemm_dq_ws_bytes(t, L->m / L->b, L->b), gemm_dq_ws_bytes(t, L->n / L->b, L->b));
+  w.chain = a.take(chain);
   w.partials = a.take(std::max(block_grad_ws_bytes(t, L->m, L->b, T),
                                block_grad_ws_bytes(t, L->n, L->b, T)));
   if (o) *o = w;
@@ -292,7 +293,7 @@ poetx_status poetx_device_status(void* stream) {
 // ------------------------------------------------------------------ CNP
 size_t poetx_cnp_workspace_bytes(int64_t nblocks, int64_t b) {
   if (nblocks <= 0 || b < 2) return 0;
-  return cnp_ws_bytes(nblocks, b);
+  return gemm_cnp_ws_bytes(nblocks, b);
 }
 
 poetx_status poetx_cnp_build(const float* q, int64_t nblocks, int64_t b, float* g, void* g_lp,
@@ -389,8 +390,8 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
     CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s), "bwd gather X");
     CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, w.dG_r, T, m, b, w.partials, s), "bwd dG_R");
   }
-  if (dq_r) CHECK_CUDA(gemm_dq_from_dg(L->q_r, w.dG_r, m / b, b, dq_r, w.chain, s), "dq_r");
-  if (dq_p) CHECK_CUDA(gemm_dq_from_dg(L->q_p, w.dG_p, n / b, b, dq_p, w.chain, s), "dq_p");
+  if (dq_r) CHECK_CUDA(gemm_dq_from_dg(t, L->q_r, w.dG_r, m / b, b, dq_r, w.chain, s), "dq_r");
+  if (dq_p) CHECK_CUDA(gemm_dq_from_dg(t, L->q_p, w.dG_p, n / b, b, dq_p, w.chain, s), "dq_p");
   return POETX_OK;
 }
 

@@ -110,7 +110,7 @@ cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, i
 
 size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows) {
   if (t != DT::BF16) return 0;
-  const int sp = grad_splits(width / b, b, rows);
+  const int sp = umma::effective_splits(rows, grad_splits(width / b, b, rows));
   return sp > 1 ? (size_t)sp * (size_t)(width * b) * sizeof(float) : 0;
 }
 
@@ -118,7 +118,7 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
                             int64_t width, int64_t b, void* partials, cudaStream_t s) {
   if (rows == 0) return cudaMemsetAsync(dG, 0, (size_t)(width * b) * sizeof(float), s);
   if (t == DT::BF16) {
-    const int sp = grad_splits(width / b, b, rows);
+    const int sp = umma::effective_splits(rows, grad_splits(width / b, b, rows));
     umma::Gemm g;
     g.M = b; g.N = b; g.K = rows; g.groups = width / b; g.splits = sp;
     g.A = A; g.a_rows = rows; g.a_cols = width; g.a_ld = width; g.a_mn = true;
@@ -147,13 +147,23 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
   return simt_gemm(g, s);
 }
 
+size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b) {
+  return tc_blocks_supported(b) ? cnp_tc_ws_bytes(nb, b) : cnp_ws_bytes(nb, b);
+}
+
 cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                            void* ws, cudaStream_t s) {
+  if (tc_blocks_supported(b)) return cnp_build_tc(q, nb, b, g, g_lp, ws, s);
   return cnp_build(q, nb, b, g, g_lp, ws, s);
 }
 
-cudaError_t gemm_dq_from_dg(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
-                            void* ws, cudaStream_t s) {
+size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b) {
+  return (t == DT::BF16 && tc_blocks_supported(b)) ? dq_tc_ws_bytes(nb, b) : dq_ws_bytes(nb, b);
+}
+
+cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG, int64_t nb, int64_t b,
+                            float* dq, void* ws, cudaStream_t s) {
+  if (t == DT::BF16 && tc_blocks_supported(b)) return dq_from_dg_tc(q, dG, nb, b, dq, ws, s);
   return dq_from_dg(q, dG, nb, b, dq, ws, s);
 }
 

@@ -22,10 +22,21 @@ int grad_splits(int64_t nb, int64_t b, int64_t rows);
 size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows);
 cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
                             int64_t width, int64_t b, void* partials, cudaStream_t s);
-// CNP blocks and the dq chain (see cnp.cu for the algebra).
+// CNP blocks and the dq chain: tensor cores (cnp_tc.cu) when b is a multiple of 128, SIMT fp32
+// (cnp.cu) otherwise; the dq chain of fp32 layers always runs in fp32 SIMT.
+bool tc_blocks_supported(int64_t b);
+size_t cnp_tc_ws_bytes(int64_t nb, int64_t b);
+size_t dq_tc_ws_bytes(int64_t nb, int64_t b);
+cudaError_t cnp_build_tc(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
+                         void* ws, cudaStream_t s);
+cudaError_t dq_from_dg_tc(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
+                          void* ws, cudaStream_t s);
+
+size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b);
 cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                            void* ws, cudaStream_t s);
-cudaError_t gemm_dq_from_dg(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
-                            void* ws, cudaStream_t s);
+size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b);
+cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG, int64_t nb, int64_t b,
+                            float* dq, void* ws, cudaStream_t s);
 
 }  // namespace poetx

@@ -443,9 +443,8 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   p.tiles_m = (int)((g.M + BM - 1) / BM);
   p.tiles_n = (int)(g.N / BN);
   const int kblocks = (int)((g.K + BK - 1) / BK);
-  const int splits = (int)std::max<int64_t>(1, std::min<int64_t>(g.splits, kblocks));
-  p.kblocks_per_split = (kblocks + splits - 1) / splits;
-  p.splits = (kblocks + p.kblocks_per_split - 1) / p.kblocks_per_split;
+  p.splits = effective_splits(g.K, g.splits);
+  p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
   p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
   p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
@@ -474,6 +473,13 @@ cudaError_t dispatch_majors(const Gemm& g, cudaStream_t s) {
 }
 
 }  // namespace
+
+int effective_splits(int64_t K, int64_t splits) {
+  const int64_t kblocks = (K + BK - 1) / BK;
+  const int64_t s = std::max<int64_t>(1, std::min<int64_t>(splits, kblocks));
+  const int64_t per = (kblocks + s - 1) / s;
+  return (int)((kblocks + per - 1) / per);
+}
 
 bool supported(const Gemm& g) {
   if (!encode_fn()) return false;

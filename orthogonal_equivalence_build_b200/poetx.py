@@ -64,6 +64,8 @@ def _load() -> ctypes.CDLL:
         "poetx_status_string": (ctypes.c_char_p, [I32]),
         "poetx_last_error_message": (ctypes.c_char_p, []),
         "poetx_abi_version": (I32, []),
+        "poetx_testing_gemm_bf16": (I32, [V, I64, I64, I32, V, I64, I64, I32, I64, I64, I64, V,
+                                          I32, I64, I32, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -79,7 +81,7 @@ EXPORTED = (
     "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
     "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
     "poetx_trace_enable", "poetx_trace_read", "poetx_status_string",
-    "poetx_last_error_message", "poetx_abi_version")
+    "poetx_last_error_message", "poetx_abi_version", "poetx_testing_gemm_bf16")
 
 
 def _check(status: int) -> None:
@@ -252,6 +254,15 @@ def trace_read(maxlen: int = 1 << 20):
         name, ms = line.rsplit(" ", 1)
         out.append((name, float(ms)))
     return out
+
+
+def testing_gemm_bf16(a: torch.Tensor, a_mn: bool, b: torch.Tensor, b_mn: bool, M: int, N: int,
+                      K: int, c: torch.Tensor, splits: int = 1, stream=None) -> None:
+    """Kernel-level hook (include/poetx_testing.h): C = A B on the tcgen05 kernel."""
+    _check(lib.poetx_testing_gemm_bf16(_ptr(a), a.shape[0], a.shape[1], int(a_mn), _ptr(b),
+                                       b.shape[0], b.shape[1], int(b_mn), M, N, K, _ptr(c),
+                                       int(c.dtype == torch.float32), c.shape[-1], splits,
+                                       _stream(stream)))
 
 
 def abi_version() -> int:

@@ -1,6 +1,7 @@
 """The C ABI loads, exports every entry point include/poetx.h declares, and rejects bad
 arguments on the host before touching a GPU.  CPU only: no call here launches a kernel."""
 import ctypes
+import glob
 import os
 import re
 
@@ -8,13 +9,15 @@ import pytest
 
 from orthogonal_equivalence_build_b200 import poetx
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "poetx.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include")
 
 
 def declared_symbols():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(poetx_[a-z_0-9]+)\s*\(", text)))
+    syms = set()
+    for h in glob.glob(os.path.join(INCLUDE, "*.h")):
+        text = re.sub(r"/\*.*?\*/", "", open(h).read(), flags=re.S)
+        syms |= set(re.findall(r"\b(poetx_[a-z_0-9]+)\s*\(", text))
+    return sorted(syms)
 
 
 def test_header_symbols_are_exported():
