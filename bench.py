@@ -18,7 +18,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -72,69 +71,83 @@ def layer_bytes(T, m, n, b, e=2):
 
 
 class ClockSampler:
-    """nvidia-smi clocks/throttle reasons sampled every 200 ms during the timed region."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons sampled every 20 ms through NVML (read-only queries)
+    while the timed region runs."""
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device: int):
+        self.dev = torch_device
+        self.samples = []
+        self.reasons = set()
+        self.smax = 0.0
+        self._stop = threading.Event()
+        self.t = None
+        self.nv = None
+
+    def _handle(self):
+        import pynvml as nv
+        import torch
+        nv.nvmlInit()
+        try:
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            return nv, nv.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            return nv, nv.nvmlDeviceGetHandleByIndex(self.dev)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            self.nv, self.h = self._handle()
+            self.smax = float(self.nv.nvmlDeviceGetMaxClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        except Exception:
+            self.nv = None
+            return
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, attr in self.REASONS:
+                    bit = getattr(nv, attr, 0)
+                    if bit and mask & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            self._stop.wait(0.02)
 
     def stop(self):
-        if not self.proc:
+        if self.t is None:
             return None
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
+        self._stop.set()
         self.t.join(timeout=2)
-        sm, smax, reasons = [], 0.0, set()
-        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
-                 "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax = max(smax, float(parts[2]))
-            except ValueError:
-                continue
-            for nm, v in zip(names[1:], parts[5:9]):
-                if v.lower() in ("active", "1"):
-                    reasons.add(nm)
-        if not sm:
+        if not self.samples:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.smax,
+                "reasons": sorted(self.reasons), "samples": len(self.samples),
+                "source": "NVML, 20 ms period, timed region only"}
 
 
 # ----------------------------------------------------------------------------- oracle arm
+_SAMPLE_CACHE = {}
+
+
 def oracle_step_sample(wl, T_sample: int):
     """One float64 oracle step (CNP of R and P, forward, backward with dq) of the workload's
     first linear on T_sample tokens.  Returns (seconds, tokens)."""
     import oracle as O
-    p = W.layer_params(wl)
-    a = W.layer_acts(wl, tokens=T_sample)
-    W0m = O.merge_permutations(p["W0"], p["perm_r"], p["perm_p"])
+    key = (wl.key, T_sample)
+    if key not in _SAMPLE_CACHE:
+        p = W.layer_params(wl)
+        a = W.layer_acts(wl, tokens=T_sample)
+        _SAMPLE_CACHE[key] = (p, a, O.merge_permutations(p["W0"], p["perm_r"], p["perm_p"]))
+    p, a, W0m = _SAMPLE_CACHE[key]
     t0 = time.perf_counter()
     G_r, G_p = O.cnp(p["q_r"], wl.b), O.cnp(p["q_p"], wl.b)
     O.linear_bwd(a["X"], a["dY"], W0m, p["perm_r"], p["perm_p"], G_r, G_p, p["q_r"], p["q_p"],
@@ -265,7 +278,7 @@ def run_ours(args):
     poetx.device_status()
 
     # ---- timed region (device time, per-step CUDA events, kernel trace on)
-    sampler = ClockSampler(local) if rank == 0 or True else None
+    sampler = ClockSampler(local)
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     barrier()
