@@ -94,6 +94,31 @@ poetx_status poetx_cnp_build(const float* q, int64_t nblocks, int64_t b, float* 
                              int32_t lp_dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * poetx_cnp_build_noalloc — poetx_cnp_build for callers that cannot allocate device memory.
+ *   The pages have no counterpart to this call; it exists for library users only. Some callers
+ *   may not allocate device memory when they build the blocks (a host program that hands out all
+ *   device memory at start-up and forbids later allocation, or code that must not risk the
+ *   device-wide synchronisation of cudaMalloc/cudaFree). This variant takes no workspace: its
+ *   scratch is a fixed POETX_CNP_NOALLOC_SCRATCH_BYTES buffer inside the library's own device
+ *   memory, which every GPU that loads the library holds until the process exits. It allocates
+ *   nothing and calls no allocating routine.
+ *   Arguments, outputs and accuracy are those of poetx_cnp_build; any nblocks is accepted (the
+ *   blocks are processed in chunks that fit the buffer).
+ *   Limit: b must need at most POETX_CNP_NOALLOC_SCRATCH_BYTES of scratch for ONE block
+ *   (20*b*b bytes when b is a multiple of 128, else 12*b*b): b <= 896 for multiples of 128,
+ *   b <= 1024 otherwise; larger b returns POETX_ERR_SHAPE with a message.
+ *   The first call on each device looks up the buffer's device address (cudaGetSymbolAddress)
+ *   with that device current; make that first call before any stream capture.
+ *   All calls on a device share the one buffer and it keeps the last call's contents (nothing in
+ *   it needs to start at zero: every byte read is written earlier in the same call). Calls whose
+ *   work overlaps on the GPU (e.g. on two streams without ordering) race on the buffer: order
+ *   them on one stream or with events.
+ * ------------------------------------------------------------------------------------------- */
+#define POETX_CNP_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+poetx_status poetx_cnp_build_noalloc(const float* q, int64_t nblocks, int64_t b, float* g,
+                                     void* g_lp, int32_t lp_dtype, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * poetx_linear_fwd — Y = X Psi_R^T Diag(G_R) W0' Diag(G_P) Psi_P, input-centric
  *   ("POET-X" blog §第一斧 and §第五斧; permutations as index maps, §第二斧; per-block batched
  *   products, §第三斧). R W0 P is never formed. Steps:

@@ -49,6 +49,7 @@ def _load() -> ctypes.CDLL:
     sig = {
         "poetx_cnp_workspace_bytes": (SZ, [I64, I64]),
         "poetx_cnp_build": (I32, [V, I64, I64, V, V, I32, V, SZ, V]),
+        "poetx_cnp_build_noalloc": (I32, [V, I64, I64, V, V, I32, V]),
         "poetx_fwd_workspace_bytes": (SZ, [LP, I64]),
         "poetx_linear_fwd": (I32, [LP, V, I64, V, V, V, SZ, V]),
         "poetx_bwd_workspace_bytes": (SZ, [LP, I64]),
@@ -76,7 +77,8 @@ def _load() -> ctypes.CDLL:
 
 lib = _load()
 EXPORTED = (
-    "poetx_cnp_workspace_bytes", "poetx_cnp_build", "poetx_fwd_workspace_bytes",
+    "poetx_cnp_workspace_bytes", "poetx_cnp_build", "poetx_cnp_build_noalloc",
+    "poetx_fwd_workspace_bytes",
     "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
     "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
     "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
@@ -169,6 +171,13 @@ def cnp_build(q: torch.Tensor, b: int, g: Optional[torch.Tensor] = None,
     ws = _workspace(cnp_workspace_bytes(nb, b), q.device, workspace)
     _check(lib.poetx_cnp_build(_ptr(q), nb, b, _ptr(g), _ptr(g_lp), BF16, _ptr(ws),
                                0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def cnp_build_noalloc(q: torch.Tensor, b: int, g: Optional[torch.Tensor] = None,
+                      g_lp: Optional[torch.Tensor] = None, stream=None) -> None:
+    """poetx_cnp_build without a workspace (fixed library-owned scratch; see include/poetx.h)."""
+    _check(lib.poetx_cnp_build_noalloc(_ptr(q), q.shape[0], b, _ptr(g), _ptr(g_lp), BF16,
+                                       _stream(stream)))
 
 
 def layer_cnp_build(layer: PoetxLinear, workspace: Optional[torch.Tensor] = None,
