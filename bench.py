@@ -70,6 +70,26 @@ def layer_bytes(T, m, n, b, e=2):
     return fwd + bwd + cnp + dq
 
 
+def sum_over_ranks_(flat, group=None):
+    """Data-parallel reduction of the packed dq gradients: dq is linear in dG, and dG is a sum
+    over tokens, so the dq of the whole batch is the sum of the ranks' dq."""
+    import torch.distributed as dist
+    if dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=group)
+    return flat
+
+
+def max_over_ranks(value: float, device=None, group=None) -> float:
+    """The job's time is the slowest rank's."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_initialized() and dist.get_world_size(group) > 1):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
 class ClockSampler:
     """SM clock and clock-event reasons sampled every 20 ms through NVML (read-only queries)
     while the timed region runs."""
@@ -266,7 +286,7 @@ def run_ours(args):
         if world > 1:
             flat_dq[:dq_r.numel()].copy_(dq_r.view(-1))
             flat_dq[dq_r.numel():].copy_(dq_p.view(-1))
-            dist.all_reduce(flat_dq)
+            sum_over_ranks_(flat_dq)
 
     def barrier():
         if world > 1:
@@ -298,11 +318,7 @@ def run_ours(args):
     poetx.trace_enable(False)
     trace = poetx.trace_read()
     step_ms = [s.elapsed_time(e) for s, e in ev]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     value = T * world * args.steps / (total_ms / 1e3)
 
@@ -356,11 +372,7 @@ def run_ours(args):
         dq_host[dq_r.numel():].copy_(dq_p.view(-1), non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e = {"value": T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
            "h2d_bytes_per_step": (x.numel() + dy.numel()) * esz,
            "d2h_bytes_per_step": dq_host.numel() * 4}

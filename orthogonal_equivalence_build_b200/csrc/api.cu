@@ -163,6 +163,7 @@ poetx_status check_ws(void* ws, size_t have, size_t need) {
 // ---- workspace layouts (each buffer 256-byte aligned)
 struct FwdWs {
   void *A, *A1, *B, *C;
+  int32_t* inv;
 };
 size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
   Arena a(base, SIZE_MAX);
@@ -172,6 +173,7 @@ size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
   w.A1 = a.take(T * L->m * e);
   w.C = a.take(T * L->n * e);
   w.B = a.take(T * L->n * e);  // used only when the caller does not keep B
+  w.inv = static_cast<int32_t*>(a.take(L->n * 4));
   if (o) *o = w;
   return a.used;
 }
@@ -181,6 +183,7 @@ struct BwdWs {
   float *dG_r, *dG_p;
   void* chain;
   void* partials;
+  int32_t* inv;
 };
 size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   Arena a(base, SIZE_MAX);
@@ -199,6 +202,7 @@ size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   w.chain = a.take(chain);
   w.partials = a.take(std::max(block_grad_ws_bytes(t, L->m, L->b, T),
                                block_grad_ws_bytes(t, L->n, L->b, T)));
+  w.inv = static_cast<int32_t*>(a.take(L->m * 4));
   if (o) *o = w;
   return a.used;
 }
@@ -341,11 +345,11 @@ poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, vo
   const int64_t m = L->m, n = L->n, b = L->b;
   const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
-  CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s), "fwd gather");
+  CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_fwd_gather_X"), "fwd gather");
   CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.A1, T, m, b, false, s), "fwd R blocks");
   CHECK_CUDA(gemm_dense(t, w.A1, L->w0m, B, T, n, m, false, s), "fwd W0' GEMM");
   CHECK_CUDA(gemm_blockwise(t, B, Gp, w.C, T, n, b, false, s), "fwd P blocks");
-  CHECK_CUDA(scatter_cols(w.C, y, T, n, L->perm_p, e, s), "fwd scatter");
+  CHECK_CUDA(scatter_cols(w.C, y, T, n, L->perm_p, e, w.inv, s, "perm_fwd_scatter_Y"), "fwd scatter");
   return POETX_OK;
 }
 
@@ -377,21 +381,31 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   const int64_t m = L->m, n = L->n, b = L->b;
   const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
-  CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s), "bwd gather dY");
+  CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s, "perm_bwd_gather_dY"), "bwd gather dY");
   CHECK_CUDA(gemm_blockwise(t, w.dC, Gp, w.dB, T, n, b, true, s), "bwd P blocks");
-  if (dq_p)
-    CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, w.dG_p, T, n, b, w.partials, s), "bwd dG_P");
+  const float* parts = static_cast<const float*>(w.partials);
+  if (dq_p) {
+    // dG_P, then its dq chain right away: the split-K partials buffer is shared with the R side
+    int sp = 1;
+    CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, w.dG_p, T, n, b, w.partials, &sp, s), "bwd dG_P");
+    CHECK_CUDA(gemm_dq_from_dg(t, L->q_p, sp > 1 ? parts : w.dG_p, sp, w.dG_p, n / b, b, dq_p,
+                               w.chain, s),
+               "dq_p");
+  }
   CHECK_CUDA(gemm_dense(t, w.dB, L->w0m, w.dA1, T, m, n, true, s), "bwd W0'^T GEMM");
   if (dx) {
     CHECK_CUDA(gemm_blockwise(t, w.dA1, Gr, w.dA, T, m, b, true, s), "bwd R blocks");
-    CHECK_CUDA(scatter_cols(w.dA, dx, T, m, L->perm_r, e, s), "bwd scatter dX");
+    CHECK_CUDA(scatter_cols(w.dA, dx, T, m, L->perm_r, e, w.inv, s, "perm_bwd_scatter_dX"),
+               "bwd scatter dX");
   }
   if (dq_r) {
-    CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s), "bwd gather X");
-    CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, w.dG_r, T, m, b, w.partials, s), "bwd dG_R");
+    int sp = 1;
+    CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_gather_X"), "bwd gather X");
+    CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, w.dG_r, T, m, b, w.partials, &sp, s), "bwd dG_R");
+    CHECK_CUDA(gemm_dq_from_dg(t, L->q_r, sp > 1 ? parts : w.dG_r, sp, w.dG_r, m / b, b, dq_r,
+                               w.chain, s),
+               "dq_r");
   }
-  if (dq_r) CHECK_CUDA(gemm_dq_from_dg(t, L->q_r, w.dG_r, m / b, b, dq_r, w.chain, s), "dq_r");
-  if (dq_p) CHECK_CUDA(gemm_dq_from_dg(t, L->q_p, w.dG_p, n / b, b, dq_p, w.chain, s), "dq_p");
   return POETX_OK;
 }
 

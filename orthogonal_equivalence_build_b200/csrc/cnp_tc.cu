@@ -21,130 +21,277 @@
 namespace poetx {
 namespace {
 
-__device__ __forceinline__ int64_t triu_index(int64_t i, int64_t j, int64_t b) {
-  return i * b - i * (i + 1) / 2 + (j - i - 1);
+// ---------------------------------------------------------------- 32 x 32 mirrored tile pairs
+// Every elementwise pass works on a pair of tiles (I, J), (J, I) with I <= J of one b x b block:
+// loads and stores stay coalesced along rows, transposes go through shared memory, and the
+// packed q of the pair is read once (its upper tile is contiguous along each row).
+constexpr int TS = 32;
+constexpr int kTileThreads = 256;  // 32 x 8: thread (tx, ty) owns rows ty, ty+8, ty+16, ty+24
+
+struct Tile {
+  float v[TS][TS + 1];
+};
+
+struct PairCtx {
+  int g, I, J;      // block, tile row, tile column (I <= J)
+  int tx, ty;
+  bool diag;
+  int64_t bb;       // b * b
+};
+
+__device__ __forceinline__ bool pair_ctx(int b, PairCtx& c) {
+  const int nt = b / TS;
+  c.I = blockIdx.x / nt;
+  c.J = blockIdx.x - c.I * nt;
+  if (c.I > c.J) return false;
+  c.g = blockIdx.y;
+  c.tx = threadIdx.x & 31;
+  c.ty = threadIdx.x >> 5;
+  c.diag = c.I == c.J;
+  c.bb = (int64_t)b * b;
+  return true;
 }
-__device__ __forceinline__ float skew_entry(const float* __restrict__ qb, int64_t i, int64_t j,
-                                            int64_t b) {
-  if (i < j) return qb[triu_index(i, j, b)];
-  if (i > j) return -qb[triu_index(j, i, b)];
-  return 0.f;
+
+// up <- Q tile (I, J), I <= J, from the packed strict upper triangle of block g.
+__device__ __forceinline__ void load_q_tile(Tile& up, const float* __restrict__ q, int b,
+                                            const PairCtx& c) {
+  const float* qb = q + (int64_t)c.g * (b * (b - 1) / 2);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    const int i = c.I * TS + r, j = c.J * TS + c.tx;
+    up.v[r][c.tx] = (i < j) ? qb[i * b - i * (i + 1) / 2 + (j - i - 1)] : 0.f;
+  }
+  __syncthreads();
+  if (c.diag) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const int r = c.ty + 8 * k;
+      if (r > c.tx) up.v[r][c.tx] = -up.v[c.tx][r];
+    }
+    __syncthreads();
+  }
 }
+// Q tile (J, I) entry (r, col) is -up.v[col][r].
+
 __device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
   hi = __float2bfloat16_rn(x);
   lo = __float2bfloat16_rn(x - __bfloat162float(hi));
 }
 
-int grid_for(int64_t n) {
-  return (int)std::max<int64_t>(1, std::min<int64_t>((n + 255) / 256, 148 * 16));
+// Concatenated split operands of one block product X Y:
+//   Acat [nb*b][3b]: row (g, i) = [Xhi(i, :) | Xhi(i, :) | Xlo(i, :)]
+//   Bcat [nb*3b][b]: rows (g, k') = Yhi (k' < b), Ylo (b <= k' < 2b), Yhi (2b <= k')
+__device__ __forceinline__ void put_split(__nv_bfloat16* __restrict__ Acat,
+                                          __nv_bfloat16* __restrict__ Bcat, int b, int g, int i,
+                                          int j, float x, float y) {
+  __nv_bfloat16 xh, xl, yh, yl;
+  split_bf16(x, xh, xl);
+  split_bf16(y, yh, yl);
+  __nv_bfloat16* arow = Acat + ((int64_t)g * b + i) * (3 * b);
+  arow[j] = xh;
+  arow[b + j] = xh;
+  arow[2 * b + j] = xl;
+  __nv_bfloat16* bblk = Bcat + (int64_t)g * 3 * b * b;
+  const int64_t e = (int64_t)i * b + j, bb = (int64_t)b * b;
+  bblk[e] = yh;
+  bblk[bb + e] = yl;
+  bblk[2 * bb + e] = yh;
 }
 
-// Concatenated split operands of one product X Y per block:
-//   Acat [nb*b][3b] row (g, i) = [Xhi(i, :) | Xhi(i, :) | Xlo(i, :)]
-//   Bcat [nb*3b][b] rows (g, k') = Yhi (k' < b), Ylo (b <= k' < 2b), Yhi (2b <= k')
-// X and Y are given elementwise: mode 0: X = Y = Q(q);  mode 1: X = S, Y = 2I + 2Q(q) + S.
-__global__ void split_operands_kernel(const float* __restrict__ q, const float* __restrict__ S,
-                                      int64_t nb, int64_t b, int mode,
-                                      __nv_bfloat16* __restrict__ Acat,
-                                      __nv_bfloat16* __restrict__ Bcat) {
-  const int64_t bb = b * b, total = nb * bb, qs = b * (b - 1) / 2;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t g = e / bb, r = e - g * bb, i = r / b, j = r - i * b;
-    const float qv = skew_entry(q + g * qs, i, j, b);
-    float x, y;
-    if (mode == 0) {
-      x = qv;
-      y = qv;
-    } else {
+// CNP pass 1: X = Y = Q.
+__global__ void __launch_bounds__(kTileThreads)
+split_q_kernel(const float* __restrict__ q, int b, __nv_bfloat16* __restrict__ Acat,
+               __nv_bfloat16* __restrict__ Bcat) {
+  __shared__ Tile up;
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  load_q_tile(up, q, b, c);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    const float v = up.v[r][c.tx];
+    put_split(Acat, Bcat, b, c.g, c.I * TS + r, c.J * TS + c.tx, v, v);
+    if (!c.diag) {
+      const float w = -up.v[c.tx][r];
+      put_split(Acat, Bcat, b, c.g, c.J * TS + r, c.I * TS + c.tx, w, w);
+    }
+  }
+}
+
+// CNP pass 2: X = S, Y = 2I + 2Q + S.
+__global__ void __launch_bounds__(kTileThreads)
+split_sh_kernel(const float* __restrict__ q, const float* __restrict__ S, int b,
+                __nv_bfloat16* __restrict__ Acat, __nv_bfloat16* __restrict__ Bcat) {
+  __shared__ Tile up;
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  load_q_tile(up, q, b, c);
+  const float* Sg = S + (int64_t)c.g * c.bb;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    {
+      const int i = c.I * TS + r, j = c.J * TS + c.tx;
+      const float s = Sg[(int64_t)i * b + j];
+      put_split(Acat, Bcat, b, c.g, i, j, s, ((i == j) ? 2.f : 0.f) + 2.f * up.v[r][c.tx] + s);
+    }
+    if (!c.diag) {
+      const int i = c.J * TS + r, j = c.I * TS + c.tx;
+      const float s = Sg[(int64_t)i * b + j];
+      put_split(Acat, Bcat, b, c.g, i, j, s, -2.f * up.v[c.tx][r] + s);
+    }
+  }
+}
+
+// CNP finish: G = I + 2Q + P (fp32 and its bf16 copy).
+__global__ void __launch_bounds__(kTileThreads)
+cnp_finish_kernel(const float* __restrict__ q, const float* __restrict__ P, int b,
+                  float* __restrict__ g, __nv_bfloat16* __restrict__ g_lp) {
+  __shared__ Tile up;
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  load_q_tile(up, q, b, c);
+  const int64_t base = (int64_t)c.g * c.bb;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    {
+      const int i = c.I * TS + r, j = c.J * TS + c.tx;
+      const int64_t e = base + (int64_t)i * b + j;
+      const float v = ((i == j) ? 1.f : 0.f) + 2.f * up.v[r][c.tx] + P[e];
+      if (g) g[e] = v;
+      if (g_lp) g_lp[e] = __float2bfloat16_rn(v);
+    }
+    if (!c.diag) {
+      const int i = c.J * TS + r, j = c.I * TS + c.tx;
+      const int64_t e = base + (int64_t)i * b + j;
+      const float v = -2.f * up.v[c.tx][r] + P[e];
+      if (g) g[e] = v;
+      if (g_lp) g_lp[e] = __float2bfloat16_rn(v);
+    }
+  }
+}
+
+// dq pass 1: Qh = bf16(Q); dG = sum of the split partials (fixed order), dGh = bf16(dG).
+__global__ void __launch_bounds__(kTileThreads)
+dq_prep_kernel(const float* __restrict__ q, const float* __restrict__ parts, int splits,
+               int64_t split_stride, int b, float* __restrict__ dG,
+               __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ dGh) {
+  __shared__ Tile up;
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  load_q_tile(up, q, b, c);
+  const int64_t base = (int64_t)c.g * c.bb;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (h == 1 && c.diag) break;
+      const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
+      const int64_t e = base + (int64_t)i * b + j;
+      float v = 0.f;
+      for (int sp = 0; sp < splits; ++sp) v += parts[sp * split_stride + e];
+      if (splits > 1) dG[e] = v;
+      dGh[e] = __float2bfloat16_rn(v);
+      Qh[e] = __float2bfloat16_rn(h ? -up.v[c.tx][r] : up.v[r][c.tx]);
+    }
+  }
+}
+
+// dq pass 2: Sh = bf16(S), SmQ = bf16(S - 2Q).
+__global__ void __launch_bounds__(kTileThreads)
+dq_prep2_kernel(const float* __restrict__ q, const float* __restrict__ S, int b,
+                __nv_bfloat16* __restrict__ Sh, __nv_bfloat16* __restrict__ SmQ) {
+  __shared__ Tile up;
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  load_q_tile(up, q, b, c);
+  const int64_t base = (int64_t)c.g * c.bb;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      if (h == 1 && c.diag) break;
+      const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
+      const int64_t e = base + (int64_t)i * b + j;
       const float s = S[e];
-      x = s;
-      y = ((i == j) ? 2.f : 0.f) + 2.f * qv + s;
-    }
-    __nv_bfloat16 xh, xl, yh, yl;
-    split_bf16(x, xh, xl);
-    split_bf16(y, yh, yl);
-    __nv_bfloat16* arow = Acat + (g * b + i) * 3 * b;
-    arow[j] = xh;
-    arow[b + j] = xh;
-    arow[2 * b + j] = xl;
-    __nv_bfloat16* bblk = Bcat + g * 3 * bb;
-    bblk[i * b + j] = yh;
-    bblk[bb + i * b + j] = yl;
-    bblk[2 * bb + i * b + j] = yh;
-  }
-}
-
-// G = I + 2Q + P, and its bf16 copy.
-__global__ void cnp_finish_kernel(const float* __restrict__ q, const float* __restrict__ P,
-                                  int64_t nb, int64_t b, float* __restrict__ g,
-                                  __nv_bfloat16* __restrict__ g_lp) {
-  const int64_t bb = b * b, total = nb * bb, qs = b * (b - 1) / 2;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t blk = e / bb, r = e - blk * bb, i = r / b, j = r - i * b;
-    const float v = ((i == j) ? 1.f : 0.f) + 2.f * skew_entry(q + blk * qs, i, j, b) + P[e];
-    if (g) g[e] = v;
-    if (g_lp) g_lp[e] = __float2bfloat16_rn(v);
-  }
-}
-
-// bf16 Q and dG for the gradient chain.
-__global__ void dq_prep_kernel(const float* __restrict__ q, const float* __restrict__ dG,
-                               int64_t nb, int64_t b, __nv_bfloat16* __restrict__ Qh,
-                               __nv_bfloat16* __restrict__ dGh) {
-  const int64_t bb = b * b, total = nb * bb, qs = b * (b - 1) / 2;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t blk = e / bb, r = e - blk * bb, i = r / b, j = r - i * b;
-    Qh[e] = __float2bfloat16_rn(skew_entry(q + blk * qs, i, j, b));
-    dGh[e] = __float2bfloat16_rn(dG[e]);
-  }
-}
-
-// Sh = bf16(S), SmQ = bf16(S - 2Q)
-__global__ void dq_prep2_kernel(const float* __restrict__ q, const float* __restrict__ S,
-                                int64_t nb, int64_t b, __nv_bfloat16* __restrict__ Sh,
-                                __nv_bfloat16* __restrict__ SmQ) {
-  const int64_t bb = b * b, total = nb * bb, qs = b * (b - 1) / 2;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t blk = e / bb, r = e - blk * bb, i = r / b, j = r - i * b;
-    const float s = S[e];
-    Sh[e] = __float2bfloat16_rn(s);
-    SmQ[e] = __float2bfloat16_rn(s - 2.f * skew_entry(q + blk * qs, i, j, b));
-  }
-}
-
-// Sbar = 2dG + T1 + Hb;  Zh = bf16(Sbar + Sbar^T);  V = 2dG + 2Hb (written over S)
-__global__ void dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
-                              const float* __restrict__ Hb, int64_t nb, int64_t b,
-                              __nv_bfloat16* __restrict__ Zh, float* __restrict__ V) {
-  const int64_t bb = b * b, total = nb * bb;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t blk = e / bb, r = e - blk * bb, i = r / b, j = r - i * b;
-    const int64_t et = blk * bb + j * b + i;
-    const float sb = 2.f * dG[e] + T1[e] + Hb[e];
-    const float sbt = 2.f * dG[et] + T1[et] + Hb[et];
-    Zh[e] = __float2bfloat16_rn(sb + sbt);
-    V[e] = 2.f * dG[e] + 2.f * Hb[e];
-  }
-}
-
-// dq_ij = (V_ij - ZQ_ij) - (V_ji - ZQ_ji), i < j
-__global__ void dq_pack_kernel(const float* __restrict__ V, const float* __restrict__ ZQ,
-                               int64_t nb, int64_t b, float* __restrict__ dq) {
-  const int64_t bb = b * b, total = nb * bb, qs = b * (b - 1) / 2;
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-       e += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t blk = e / bb, r = e - blk * bb, i = r / b, j = r - i * b;
-    if (i < j) {
-      const int64_t et = blk * bb + j * b + i;
-      dq[blk * qs + triu_index(i, j, b)] = (V[e] - ZQ[e]) - (V[et] - ZQ[et]);
+      const float qv = h ? -up.v[c.tx][r] : up.v[r][c.tx];
+      Sh[e] = __float2bfloat16_rn(s);
+      SmQ[e] = __float2bfloat16_rn(s - 2.f * qv);
     }
   }
 }
+
+// dq pass 3: Sbar = 2dG + T1 + Hb; Zh = bf16(Sbar + Sbar^T); V = 2dG + 2Hb (written over S).
+__global__ void __launch_bounds__(kTileThreads)
+dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
+              const float* __restrict__ Hb, int b, __nv_bfloat16* __restrict__ Zh,
+              float* __restrict__ V) {
+  __shared__ Tile sa, sb;  // Sbar tiles (I, J) and (J, I)
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  const int64_t base = (int64_t)c.g * c.bb;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
+      const int64_t e = base + (int64_t)i * b + j;
+      const float d = dG[e], hb = Hb[e];
+      (h ? sb : sa).v[r][c.tx] = 2.f * d + T1[e] + hb;
+      if (h == 0 || !c.diag) V[e] = 2.f * d + 2.f * hb;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    {
+      const int i = c.I * TS + r, j = c.J * TS + c.tx;
+      Zh[base + (int64_t)i * b + j] = __float2bfloat16_rn(sa.v[r][c.tx] + sb.v[c.tx][r]);
+    }
+    if (!c.diag) {
+      const int i = c.J * TS + r, j = c.I * TS + c.tx;
+      Zh[base + (int64_t)i * b + j] = __float2bfloat16_rn(sb.v[r][c.tx] + sa.v[c.tx][r]);
+    }
+  }
+}
+
+// dq pass 4: U = V - ZQ; dq_ij = U_ij - U_ji (i < j), written packed.
+__global__ void __launch_bounds__(kTileThreads)
+dq_pack_kernel(const float* __restrict__ V, const float* __restrict__ ZQ, int b,
+               float* __restrict__ dq) {
+  __shared__ Tile ua, ub;  // U tiles (I, J) and (J, I)
+  PairCtx c;
+  if (!pair_ctx(b, c)) return;
+  const int64_t base = (int64_t)c.g * c.bb;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    {
+      const int64_t e = base + (int64_t)(c.I * TS + r) * b + c.J * TS + c.tx;
+      ua.v[r][c.tx] = V[e] - ZQ[e];
+    }
+    {
+      const int64_t e = base + (int64_t)(c.J * TS + r) * b + c.I * TS + c.tx;
+      ub.v[r][c.tx] = V[e] - ZQ[e];
+    }
+  }
+  __syncthreads();
+  float* dqb = dq + (int64_t)c.g * (b * (b - 1) / 2);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int r = c.ty + 8 * k;
+    const int i = c.I * TS + r, j = c.J * TS + c.tx;
+    if (i < j) dqb[i * b - i * (i + 1) / 2 + (j - i - 1)] = ua.v[r][c.tx] - ub.v[c.tx][r];
+  }
+}
+
+dim3 pair_grid(int64_t nb, int64_t b) { return dim3((unsigned)((b / TS) * (b / TS)), (unsigned)nb); }
 
 // C_g = X_g Y_g for nb blocks of b x b (fp32 out), X K-major [nb*b][kx] (kx = K), Y MN-major
 // [nb*K][b]. K = b (single pass) or 3b (split operands).
@@ -184,21 +331,22 @@ cudaError_t cnp_build_tc(const float* q, int64_t nb, int64_t b, float* g, __nv_b
   auto* Bcat = static_cast<__nv_bfloat16*>(a.take((size_t)(nb * b * 3 * b) * 2));
   auto* S = static_cast<float*>(a.take((size_t)(nb * b * b) * 4));
   auto* P = static_cast<float*>(a.take((size_t)(nb * b * b) * 4));
-  const int grid = grid_for(nb * b * b);
+  const dim3 grid = pair_grid(nb, b);
+  const int bi = (int)b;
   {
     TraceScope t("cnp_split_Q", s);
-    split_operands_kernel<<<grid, 256, 0, s>>>(q, nullptr, nb, b, 0, Acat, Bcat);
+    split_q_kernel<<<grid, kTileThreads, 0, s>>>(q, bi, Acat, Bcat);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Acat, Bcat, S, nb, b, 3 * b, "umma_cnp_QQ", s));
   {
     TraceScope t("cnp_split_SH", s);
-    split_operands_kernel<<<grid, 256, 0, s>>>(q, S, nb, b, 1, Acat, Bcat);
+    split_sh_kernel<<<grid, kTileThreads, 0, s>>>(q, S, bi, Acat, Bcat);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Acat, Bcat, P, nb, b, 3 * b, "umma_cnp_SH", s));
   TraceScope t("cnp_finish", s);
-  cnp_finish_kernel<<<grid, 256, 0, s>>>(q, P, nb, b, g, g_lp);
+  cnp_finish_kernel<<<grid, kTileThreads, 0, s>>>(q, P, bi, g, g_lp);
   return cudaGetLastError();
 }
 
@@ -208,8 +356,8 @@ size_t dq_tc_ws_bytes(int64_t nb, int64_t b) {
   return 5 * h + 3 * f;
 }
 
-cudaError_t dq_from_dg_tc(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
-                          void* ws, cudaStream_t s) {
+cudaError_t dq_from_dg_tc(const float* q, const float* dG_parts, int splits, float* dG,
+                          int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s) {
   if (nb == 0) return cudaSuccess;
   Arena a(ws, dq_tc_ws_bytes(nb, b));
   const size_t hb = (size_t)(nb * b * b) * 2, fb = (size_t)(nb * b * b) * 4;
@@ -221,28 +369,32 @@ cudaError_t dq_from_dg_tc(const float* q, const float* dG, int64_t nb, int64_t b
   auto* S = static_cast<float*>(a.take(fb));
   auto* Hb = static_cast<float*>(a.take(fb));
   auto* T1 = static_cast<float*>(a.take(fb));
-  const int grid = grid_for(nb * b * b);
+  const dim3 grid = pair_grid(nb, b);
+  const int bi = (int)b;
+  // with one split the gradient is read in place; with several it is summed into dG
+  const float* dGsum = splits > 1 ? dG : dG_parts;
   {
     TraceScope t("dq_prep", s);
-    dq_prep_kernel<<<grid, 256, 0, s>>>(q, dG, nb, b, Qh, dGh);
+    dq_prep_kernel<<<grid, kTileThreads, 0, s>>>(q, dG_parts, splits, nb * b * b, bi, dG, Qh,
+                                                 dGh);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Qh, Qh, S, nb, b, b, "umma_dq_QQ", s));
   {
     TraceScope t("dq_prep2", s);
-    dq_prep2_kernel<<<grid, 256, 0, s>>>(q, S, nb, b, Sh, SmQ);
+    dq_prep2_kernel<<<grid, kTileThreads, 0, s>>>(q, S, bi, Sh, SmQ);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Sh, dGh, Hb, nb, b, b, "umma_dq_SdG", s));
   POETX_TRY(block_product(dGh, SmQ, T1, nb, b, b, "umma_dq_dGH", s));
   {
     TraceScope t("dq_mid", s);
-    dq_mid_kernel<<<grid, 256, 0, s>>>(dG, T1, Hb, nb, b, Zh, S);
+    dq_mid_kernel<<<grid, kTileThreads, 0, s>>>(dGsum, T1, Hb, bi, Zh, S);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Zh, Qh, T1, nb, b, b, "umma_dq_ZQ", s));
   TraceScope t("dq_pack", s);
-  dq_pack_kernel<<<grid, 256, 0, s>>>(S, T1, nb, b, dq);
+  dq_pack_kernel<<<grid, kTileThreads, 0, s>>>(S, T1, bi, dq);
   return cudaGetLastError();
 }
 

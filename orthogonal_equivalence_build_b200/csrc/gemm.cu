@@ -34,11 +34,23 @@ __global__ void sum_partials_kernel(const float* __restrict__ part, float* __res
 }  // namespace
 
 int grad_splits(int64_t nb, int64_t b, int64_t rows) {
-  // enough (group, tile, split) work units for two waves, each split >= 1024 token rows
+  // Split the contraction over tokens so the (group, tile, split) work units fill whole waves of
+  // the persistent grid (all units cost the same); each split keeps >= 512 token rows.
   const int64_t tiles = nb * ((b + 127) / 128) * std::max<int64_t>(1, b / 256);
-  int64_t s = (2 * 148 + tiles - 1) / std::max<int64_t>(tiles, 1);
-  s = std::min<int64_t>(s, std::max<int64_t>(1, rows / 1024));
-  return (int)std::max<int64_t>(1, std::min<int64_t>(s, 16));
+  const int64_t waves_unit = sms();
+  const int64_t max_s = std::max<int64_t>(1, std::min<int64_t>(16, rows / 512));
+  int best = 1;
+  double best_eff = 0.0;
+  for (int64_t s = 1; s <= max_s; ++s) {
+    const int64_t units = tiles * s;
+    const int64_t waves = (units + waves_unit - 1) / waves_unit;
+    // efficiency of the last wave, discounted slightly per extra split (partial-sum traffic)
+    const double eff = (double)units / (double)(waves * waves_unit) - 0.05 * (double)(s - 1);
+    if (units < waves_unit) continue;  // below one wave: more splits always help
+    if (eff > best_eff + 1e-9) { best_eff = eff; best = (int)s; }
+  }
+  if (best_eff == 0.0) best = (int)std::min<int64_t>(max_s, (waves_unit + tiles - 1) / tiles);
+  return std::max(1, best);
 }
 
 cudaError_t gemm_blockwise(DT t, const void* A, const void* G, void* C, int64_t rows,
@@ -115,7 +127,9 @@ size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows) {
 }
 
 cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
-                            int64_t width, int64_t b, void* partials, cudaStream_t s) {
+                            int64_t width, int64_t b, void* partials, int* splits_used,
+                            cudaStream_t s) {
+  *splits_used = 1;
   if (rows == 0) return cudaMemsetAsync(dG, 0, (size_t)(width * b) * sizeof(float), s);
   if (t == DT::BF16) {
     const int sp = umma::effective_splits(rows, grad_splits(width / b, b, rows));
@@ -129,13 +143,8 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
     g.C = sp > 1 ? partials : dG;
     g.name = "umma_block_grad";
     if (b % 128 == 0 && umma::supported(g) && (sp == 1 || partials)) {
-      cudaError_t e = umma::gemm(g, s);
-      if (e != cudaSuccess || sp == 1) return e;
-      const int64_t count = width * b;
-      TraceScope tr("sum_split_partials", s);
-      sum_partials_kernel<<<(int)std::min<int64_t>((count + 255) / 256, sms() * 8), 256, 0, s>>>(
-          static_cast<const float*>(partials), dG, count, sp);
-      return cudaGetLastError();
+      *splits_used = sp;
+      return umma::gemm(g, s);
     }
   }
   SimtGemm g{};
@@ -161,10 +170,20 @@ size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b) {
   return (t == DT::BF16 && tc_blocks_supported(b)) ? dq_tc_ws_bytes(nb, b) : dq_ws_bytes(nb, b);
 }
 
-cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG, int64_t nb, int64_t b,
-                            float* dq, void* ws, cudaStream_t s) {
-  if (t == DT::BF16 && tc_blocks_supported(b)) return dq_from_dg_tc(q, dG, nb, b, dq, ws, s);
-  return dq_from_dg(q, dG, nb, b, dq, ws, s);
+cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG_parts, int splits, float* dG,
+                            int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s) {
+  if (t == DT::BF16 && tc_blocks_supported(b))
+    return dq_from_dg_tc(q, dG_parts, splits, dG, nb, b, dq, ws, s);
+  if (splits > 1) {
+    const int64_t count = nb * b * b;
+    TraceScope tr("sum_split_partials", s);
+    sum_partials_kernel<<<(int)std::min<int64_t>((count + 255) / 256, sms() * 8), 256, 0, s>>>(
+        dG_parts, dG, count, splits);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    dG_parts = dG;
+  }
+  return dq_from_dg(q, dG_parts, nb, b, dq, ws, s);
 }
 
 }  // namespace poetx

@@ -16,12 +16,15 @@ cudaError_t gemm_blockwise_left(DT t, const void* G, const void* N, void* C, int
 cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, int64_t N,
                        int64_t K, bool w_trans, cudaStream_t s);
 // dG_j = A_j^T B_j (contraction over the rows): A, B [rows, width], dG [width/b, b, b] fp32.
-// bf16 operands split the contraction over `grad_splits` ranges of rows; their fp32 partial
-// sums go to `partials` (block_grad_ws_bytes bytes) and are then added in a fixed order.
+// bf16 operands split the contraction over `grad_splits` ranges of rows. With more than one
+// range the fp32 partial products go to `partials` ([splits][width/b][b][b], block_grad_ws_bytes
+// bytes), dG is left untouched and *splits_used says how many ranges there are; the consumer
+// (gemm_dq_from_dg) adds them in a fixed order. With one range the result is written to dG.
 int grad_splits(int64_t nb, int64_t b, int64_t rows);
 size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows);
 cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
-                            int64_t width, int64_t b, void* partials, cudaStream_t s);
+                            int64_t width, int64_t b, void* partials, int* splits_used,
+                            cudaStream_t s);
 // CNP blocks and the dq chain: tensor cores (cnp_tc.cu) when b is a multiple of 128, SIMT fp32
 // (cnp.cu) otherwise; the dq chain of fp32 layers always runs in fp32 SIMT.
 bool tc_blocks_supported(int64_t b);
@@ -29,14 +32,16 @@ size_t cnp_tc_ws_bytes(int64_t nb, int64_t b);
 size_t dq_tc_ws_bytes(int64_t nb, int64_t b);
 cudaError_t cnp_build_tc(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                          void* ws, cudaStream_t s);
-cudaError_t dq_from_dg_tc(const float* q, const float* dG, int64_t nb, int64_t b, float* dq,
-                          void* ws, cudaStream_t s);
+// dG_parts: `splits` fp32 partial sums [splits][nb][b][b] (splits == 1: the gradient itself);
+// dG: [nb][b][b] fp32 buffer that receives the sum when splits > 1.
+cudaError_t dq_from_dg_tc(const float* q, const float* dG_parts, int splits, float* dG,
+                          int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s);
 
 size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b);
 cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                            void* ws, cudaStream_t s);
 size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b);
-cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG, int64_t nb, int64_t b,
-                            float* dq, void* ws, cudaStream_t s);
+cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG_parts, int splits, float* dG,
+                            int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s);
 
 }  // namespace poetx

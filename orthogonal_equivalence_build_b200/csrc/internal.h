@@ -46,10 +46,12 @@ struct Arena {
 // out[r, c] = in[row_map ? row_map[r] : r, col_map[c]]       (gather)
 cudaError_t gather_cols(const void* in, void* out, int64_t rows, int64_t cols,
                         const int32_t* row_map, const int32_t* col_map, int elem_bytes,
-                        cudaStream_t s);
+                        cudaStream_t s, const char* name = nullptr);
 // out[r, col_map[c]] = in[r, c]                              (scatter)
+// With inv_tmp (cols ints, 16-byte aligned) it runs as a gather through the inverse map.
 cudaError_t scatter_cols(const void* in, void* out, int64_t rows, int64_t cols,
-                         const int32_t* col_map, int elem_bytes, cudaStream_t s);
+                         const int32_t* col_map, int elem_bytes, int32_t* inv_tmp,
+                         cudaStream_t s, const char* name = nullptr);
 // rho[i] = inverse(perm_old)[perm_new[i]]; inv_tmp is k ints of scratch
 cudaError_t compose_inverse(const int32_t* perm_old, const int32_t* perm_new, int32_t* inv_tmp,
                             int32_t* rho, int64_t k, cudaStream_t s);

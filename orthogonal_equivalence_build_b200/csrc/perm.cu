@@ -101,6 +101,90 @@ __global__ void scatter_cols_global(const T* __restrict__ in, T* __restrict__ ou
   }
 }
 
+// out[r, c] = in[rmap(r), cmap[c]] for many rows sharing one column map. Rows are staged through
+// shared memory in chunks of R rows with double-buffered cp.async (16-byte pieces, L1 bypassed),
+// so the loads of chunk k+1 overlap the gather of chunk k. Each thread owns up to VPT fixed
+// 16-byte output vectors (vector v = tid + k * blockDim) and keeps their source indices in
+// registers for the whole launch (packed two 16-bit indices per register), so the per-row work
+// is shared-memory reads plus one coalesced 16-byte store per vector. Needs cols <= 65536,
+// 16-byte aligned rows and index array, and cols / (16 / sizeof(T)) <= VPT * blockDim.
+template <typename T, int VPT>
+__global__ void __launch_bounds__(256)
+gather_cols_pipelined(const T* __restrict__ in, T* __restrict__ out, int64_t rows, int cols,
+                      const int32_t* __restrict__ row_map, const int32_t* __restrict__ col_map,
+                      int R) {
+  constexpr int VEC = 16 / sizeof(T);
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T* buf[2] = {reinterpret_cast<T*>(smem_raw),
+               reinterpret_cast<T*>(smem_raw) + (int64_t)R * cols};
+  const int nvec = cols / VEC;
+  const int64_t nchunks = (rows + R - 1) / R;
+  int64_t chunk = blockIdx.x;
+  if (chunk >= nchunks) return;
+  // this thread's source indices, loaded once
+  uint32_t ids[VPT][VEC / 2];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int v = threadIdx.x + k * blockDim.x;
+#pragma unroll
+    for (int h = 0; h < VEC / 2; ++h) ids[k][h] = 0;
+    if (v < nvec) {
+#pragma unroll
+      for (int h = 0; h < VEC / 4; ++h) {
+        const int4 t = __ldg(reinterpret_cast<const int4*>(col_map + v * VEC) + h);
+        ids[k][2 * h] = (uint32_t)t.x | ((uint32_t)t.y << 16);
+        ids[k][2 * h + 1] = (uint32_t)t.z | ((uint32_t)t.w << 16);
+      }
+    }
+  }
+  auto issue = [&](int64_t ch, T* dst) {
+    for (int idx = threadIdx.x; idx < R * nvec; idx += blockDim.x) {
+      const int r = idx / nvec, v = idx - r * nvec;
+      const int64_t row = ch * R + r;
+      if (row >= rows) continue;
+      const int64_t src_row = row_map ? (int64_t)row_map[row] : row;
+      const T* g = in + src_row * cols + (int64_t)v * VEC;
+      const uint32_t sa = static_cast<uint32_t>(__cvta_generic_to_shared(dst + r * cols + v * VEC));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(g) : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  issue(chunk, buf[0]);
+  int cur = 0;
+  for (; chunk < nchunks; chunk += gridDim.x) {
+    const int64_t next = chunk + gridDim.x;
+    if (next < nchunks) issue(next, buf[cur ^ 1]);
+    else asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncthreads();
+    const int64_t left = rows - chunk * R;
+    const int nr = left < R ? (int)left : R;
+    for (int r = 0; r < nr; ++r) {
+      const T* srow = buf[cur] + r * cols;
+      T* orow = out + (chunk * R + r) * cols;
+#pragma unroll
+      for (int k = 0; k < VPT; ++k) {
+        const int v = threadIdx.x + k * blockDim.x;
+        if (v < nvec) {
+          union {
+            int4 v4;
+            T e[VEC];
+          } pack;
+#pragma unroll
+          for (int h = 0; h < VEC / 2; ++h) {
+            pack.e[2 * h] = srow[ids[k][h] & 0xFFFFu];
+            pack.e[2 * h + 1] = srow[ids[k][h] >> 16];
+          }
+          *reinterpret_cast<int4*>(orow + v * VEC) = pack.v4;
+        }
+      }
+    }
+    __syncthreads();
+    cur ^= 1;
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+}
+
 int num_sms() {
   static int sms = 0;
   if (!sms) {
@@ -114,10 +198,36 @@ int num_sms() {
 
 constexpr size_t kMaxRowSmem = 200 * 1024;
 
+bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
 template <typename T>
 cudaError_t launch_gather(const void* in, void* out, int64_t rows, int64_t cols,
-                          const int32_t* row_map, const int32_t* col_map, cudaStream_t s) {
+                          const int32_t* row_map, const int32_t* col_map, cudaStream_t s,
+                          const char* name) {
   if (rows == 0 || cols == 0) return cudaSuccess;
+  const size_t row_bytes = (size_t)cols * sizeof(T);
+  constexpr int VEC = 16 / sizeof(T);
+  const int64_t nvec = cols / VEC;
+  if (row_bytes % 16 == 0 && row_bytes <= 96 * 1024 && cols <= 65536 && nvec <= 8 * 256 &&
+      aligned16p(in) && aligned16p(out) && aligned16p(col_map)) {
+    // chunks of about 24 KB per buffer, two buffers per CTA
+    const int R = (int)std::max<size_t>(1, std::min<size_t>(16, (24 * 1024) / row_bytes));
+    const size_t smem = 2 * (size_t)R * row_bytes;
+    const int per_sm = std::max(1, std::min(8, (int)((200 * 1024) / smem)));
+    const int64_t nchunks = (rows + R - 1) / R;
+    const int64_t grid = std::min<int64_t>(nchunks, (int64_t)num_sms() * per_sm);
+    TraceScope t(name ? name : (sizeof(T) == 2 ? "perm_gather_cols_bf16" : "perm_gather_cols_f32"),
+                 s);
+    auto launch = [&](auto kern) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      kern<<<(unsigned)grid, 256, smem, s>>>(static_cast<const T*>(in), static_cast<T*>(out),
+                                             rows, (int)cols, row_map, col_map, R);
+    };
+    if (nvec <= 2 * 256) launch(gather_cols_pipelined<T, 2>);
+    else if (nvec <= 4 * 256) launch(gather_cols_pipelined<T, 4>);
+    else launch(gather_cols_pipelined<T, 8>);
+    return cudaGetLastError();
+  }
   const size_t smem = 2 * (size_t)pad8(cols) * sizeof(T);
   if (smem <= kMaxRowSmem) {
     cudaFuncSetAttribute(gather_cols_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -229,13 +339,27 @@ __global__ void check_counts_kernel(int32_t* __restrict__ counts, int64_t k) {
 
 cudaError_t gather_cols(const void* in, void* out, int64_t rows, int64_t cols,
                         const int32_t* row_map, const int32_t* col_map, int elem_bytes,
-                        cudaStream_t s) {
-  if (elem_bytes == 2) return launch_gather<__nv_bfloat16>(in, out, rows, cols, row_map, col_map, s);
-  return launch_gather<float>(in, out, rows, cols, row_map, col_map, s);
+                        cudaStream_t s, const char* name) {
+  if (elem_bytes == 2)
+    return launch_gather<__nv_bfloat16>(in, out, rows, cols, row_map, col_map, s, name);
+  return launch_gather<float>(in, out, rows, cols, row_map, col_map, s, name);
 }
 
 cudaError_t scatter_cols(const void* in, void* out, int64_t rows, int64_t cols,
-                         const int32_t* col_map, int elem_bytes, cudaStream_t s) {
+                         const int32_t* col_map, int elem_bytes, int32_t* inv_tmp,
+                         cudaStream_t s, const char* name) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  if (inv_tmp && aligned16p(inv_tmp) && ((size_t)cols * elem_bytes) % 16 == 0) {
+    // out[r, p] = in[r, inverse(col_map)[p]]: the scatter as a pipelined gather
+    const int grid = (int)std::min<int64_t>((cols + 255) / 256, 4096);
+    {
+      TraceScope t("perm_invert", s);
+      invert_kernel<<<grid, 256, 0, s>>>(col_map, inv_tmp, cols);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    return gather_cols(in, out, rows, cols, nullptr, inv_tmp, elem_bytes, s, name);
+  }
   if (elem_bytes == 2) return launch_scatter<__nv_bfloat16>(in, out, rows, cols, col_map, s);
   return launch_scatter<float>(in, out, rows, cols, col_map, s);
 }

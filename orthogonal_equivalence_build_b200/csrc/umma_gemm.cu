@@ -186,6 +186,27 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile) {
   return t;
 }
 
+// Store 32 accumulator columns of one row (already in registers) as fp32 or bf16.
+template <bool OUT_F32>
+__device__ __forceinline__ void store_row32(void* C, long long off, const uint32_t (&r)[32]) {
+  if constexpr (OUT_F32) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(C) + off);
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(C) + off);
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      dst[v] = make_uint4(
+          pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+          pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+          pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+          pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+  }
+}
+
 template <int BN, bool A_MN, bool B_MN, bool OUT_F32, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
@@ -346,24 +367,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
       for (int c = 0; c < BN; c += 32) {
         uint32_t r[32];
         tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + c), r);
-        if (live) {
-          if constexpr (OUT_F32) {
-            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.C) + base + c);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                   __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          } else {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + base + c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(
-                  pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
-          }
-        }
+        if (live) store_row32<OUT_F32>(p.C, base + c, r);
       }
       tc_fence_before();
       __syncwarp();

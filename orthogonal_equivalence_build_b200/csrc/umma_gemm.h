@@ -25,6 +25,7 @@ struct Gemm {
 };
 
 bool supported(const Gemm& g);
+
 // Number of K ranges the kernel actually uses for `splits` requested ranges over K
 // (ranges of whole 64-wide K blocks, none empty).
 int effective_splits(int64_t K, int64_t splits);

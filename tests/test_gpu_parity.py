@@ -73,7 +73,9 @@ def test_validate_permutation():
 # ------------------------------------------------------------------ bit-exact layer cases
 @pytest.mark.parametrize("key,m,b,T", [("tiny_fp32", 512, 64, 200),
                                        ("llama1p3b_attn", 512, 128, 333),
-                                       ("llama1p3b_attn", 1024, 256, 130)])
+                                       ("llama1p3b_attn", 1024, 256, 130),
+                                       ("llama1p3b_attn", 1024, 256, 777),
+                                       ("llama8b_up_proj", 1024, 512, 1100)])
 def test_identity_layer_is_bit_exact(key, m, b, T):
     """q = 0 and W0 = I: G = I exactly and every product is by 1.0 or 0.0, so Y == X and
     dX == dY bit for bit; this pins the gathers, scatters and operand layouts."""
@@ -129,6 +131,8 @@ def test_fp32_layer_shapes(m, n, b, T):
     ("llama8b_up_proj", 1024, 3584, 512, 300),
     ("llama8b_decoder", 512, 1536, 256, 129),
     ("llama1p3b_attn", 512, 512, 128, 1),
+    ("llama8b_up_proj", 1024, 2048, 512, 1000),
+    ("llama1p3b_attn", 768, 512, 256, 2049),
 ])
 def test_bf16_layer_parity(key, m, n, b, T):
     _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), TOL_BF16)
