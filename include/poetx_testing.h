@@ -13,7 +13,9 @@
  *   splits > 1 splits K into that many ranges of whole 64-wide K blocks and writes fp32
  *   partial products to C + s * M * ldc (c_f32 must be 1); the caller adds them. A count that
  *   would leave a range empty (e.g. 5 ranges over 16 blocks) is rejected with INVALID_ARG.
- * Returns POETX_ERR_UNSUPPORTED when the tensor-core tiling does not cover the shape
+ *   variant 0 runs the single-CTA kernel (128 x BN tiles); variant 1 runs the CTA-pair kernel
+ *   (tcgen05.mma.cta_group::2 on a 2-CTA cluster, 256 x 256 tiles; N % 256 == 0, M >= 256).
+ * Returns POETX_ERR_UNSUPPORTED when the chosen kernel's tiling does not cover the shape
  * (N % 64 != 0, K-major extents < 64, misaligned pointers or strides); it never falls back.
  * Asynchronous on `stream`.
  */
@@ -27,7 +29,7 @@ extern "C" {
 poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, int64_t a_cols, int32_t a_mn,
                                      const void* B, int64_t b_rows, int64_t b_cols, int32_t b_mn,
                                      int64_t M, int64_t N, int64_t K, void* C, int32_t c_f32,
-                                     int64_t ldc, int32_t splits, void* stream);
+                                     int64_t ldc, int32_t splits, int32_t variant, void* stream);
 
 #ifdef __cplusplus
 }

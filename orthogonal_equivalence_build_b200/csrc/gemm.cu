@@ -31,6 +31,12 @@ __global__ void sum_partials_kernel(const float* __restrict__ part, float* __res
   }
 }
 
+// CTA-pair tiles where the shape allows (256 x 256 per pair), single-CTA tiles otherwise.
+cudaError_t run(const umma::Gemm& g, cudaStream_t s) {
+  if (umma::pair_supported(g)) return umma::gemm_pair(g, s);
+  return umma::gemm(g, s);
+}
+
 }  // namespace
 
 int grad_splits(int64_t nb, int64_t b, int64_t rows) {
@@ -65,6 +71,7 @@ cudaError_t gemm_blockwise(DT t, const void* A, const void* G, void* C, int64_t 
     else { g.b_mn = true; g.b_gn = 0; g.b_gk = b; }                // B(k, j) = G[k][j]
     g.C = C; g.ldc = width; g.c_gs = b;
     g.name = transpose_g ? "umma_blockwise_T" : "umma_blockwise";
+    // K = b is short: single-CTA 128 x 256 tiles measured faster than CTA pairs here
     if (umma::supported(g)) return umma::gemm(g, s);
   }
   SimtGemm g{};
@@ -86,7 +93,7 @@ cudaError_t gemm_blockwise_left(DT t, const void* G, const void* N, void* C, int
     g.B = N; g.b_rows = m; g.b_cols = n; g.b_ld = n; g.b_mn = true; g.b_gn = 0; g.b_gk = b;
     g.C = C; g.ldc = n; g.c_gs = b * n;
     g.name = "umma_blockwise_left";
-    if (b % 128 == 0 && umma::supported(g)) return umma::gemm(g, s);
+    if (b % 128 == 0 && umma::supported(g)) return run(g, s);
   }
   SimtGemm g{};
   g.M = b; g.N = n; g.K = b; g.batch = m / b;
@@ -108,7 +115,7 @@ cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, i
     else { g.b_rows = K; g.b_cols = N; g.b_ld = N; g.b_mn = true; }
     g.C = C; g.ldc = N;
     g.name = w_trans ? "umma_dense_W0T" : "umma_dense_W0";
-    if (umma::supported(g)) return umma::gemm(g, s);
+    if (umma::supported(g)) return run(g, s);
   }
   SimtGemm g{};
   g.M = M; g.N = N; g.K = K; g.batch = 1;
@@ -144,7 +151,7 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
     g.name = "umma_block_grad";
     if (b % 128 == 0 && umma::supported(g) && (sp == 1 || partials)) {
       *splits_used = sp;
-      return umma::gemm(g, s);
+      return run(g, s);
     }
   }
   SimtGemm g{};

@@ -6,7 +6,8 @@ extern "C" poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, i
                                                 int32_t a_mn, const void* B, int64_t b_rows,
                                                 int64_t b_cols, int32_t b_mn, int64_t M,
                                                 int64_t N, int64_t K, void* C, int32_t c_f32,
-                                                int64_t ldc, int32_t splits, void* stream) {
+                                                int64_t ldc, int32_t splits, int32_t variant,
+                                                void* stream) {
   using namespace poetx;
   if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || splits < 1) {
     set_error("testing_gemm: bad arguments");
@@ -27,12 +28,14 @@ extern "C" poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, i
   g.B = B; g.b_rows = b_rows; g.b_cols = b_cols; g.b_ld = b_cols; g.b_mn = b_mn != 0;
   g.C = C; g.out_f32 = c_f32 != 0; g.ldc = ldc; g.c_split = M * ldc;
   g.name = "umma_testing_gemm";
-  if (!umma::supported(g) || (g.a_mn && g.b_mn && !g.out_f32) ||
-      (g.a_mn && !g.b_mn)) {
+  const bool pair = variant == 1;
+  if (!umma::supported(g) || (g.a_mn && g.b_mn && !g.out_f32) || (g.a_mn && !g.b_mn) ||
+      (pair && !umma::pair_supported(g)) || variant < 0 || variant > 1) {
     set_error("testing_gemm: shape/layout not covered by the tensor-core kernel");
     return POETX_ERR_UNSUPPORTED;
   }
-  cudaError_t e = umma::gemm(g, static_cast<cudaStream_t>(stream));
+  cudaError_t e = pair ? umma::gemm_pair(g, static_cast<cudaStream_t>(stream))
+                       : umma::gemm(g, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) {
     set_error("testing_gemm: %s", cudaGetErrorString(e));
     return POETX_ERR_CUDA;

@@ -303,6 +303,7 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
                        kDrainLimitNs);
       }
     }
+    __syncwarp();  // reconverge before the block-wide barriers below
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -385,6 +386,276 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair kernel
+// The same GEMM on a cluster of two CTAs on two SMs with tcgen05.mma.cta_group::2: one MMA
+// instruction computes a 256 x 256 x 16 product; CTA r of the pair holds rows [128r, 128r+128)
+// of the A tile and rows [128r, 128r+128) of the B tile (N) in its own shared memory and receives
+// rows [128r, 128r+128) x 256 of the accumulator in its own TMEM. Per CTA and 64-deep stage that
+// is 32 KB of operands for 128 x 256 x 64 outputs, two thirds of the single-CTA 128 x 256 tile's
+// 48 KB, which is what bounds that tile by L2 bandwidth.
+//   Both producers load their halves with TMA; the bytes of both complete the transaction count
+//   of the leader's (rank 0) full barrier. The leader's single MMA thread issues the pair MMAs
+//   and commits with a multicast to both CTAs' empty / accumulator-full barriers. Epilogue warps
+//   of both CTAs read their own TMEM and arrive on the leader's accumulator-empty barrier.
+//   No TMA load is multicast.
+struct PairParams {
+  int M, N, K, groups, splits;
+  int tiles_m, tiles_n, kblocks_per_split, total_tiles;   // tiles of 256 x 256
+  int a_gm, a_gk, b_gn, b_gk;
+  void* C;
+  long long ldc, c_gs, c_split;
+  int* err;
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+               "memory");
+}
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// arrive once on `bar` in every CTA of the pair when this thread's MMAs have retired
+__device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+
+// Instruction descriptor for the pair MMA: M = 256, N = 256.
+template <bool A_MN, bool B_MN>
+__device__ __forceinline__ constexpr uint32_t instr_desc_pair() {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((A_MN ? 1u : 0u) << 15) |
+         ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+}
+
+__device__ __forceinline__ TileCoord decode_pair_tile(const PairParams& p, int tile) {
+  constexpr int GROUP_M = 8;   // bands of 8 pair-rows (2048 rows)
+  const int per_group = p.tiles_m * p.tiles_n;
+  const int per_split = per_group * p.groups;
+  TileCoord t;
+  t.split = tile / per_split;
+  const int r = tile - t.split * per_split;
+  t.g = r / per_group;
+  const int local = r - t.g * per_group;
+  const int band = local / (GROUP_M * p.tiles_n);
+  const int first_m = band * GROUP_M;
+  const int gm = min(GROUP_M, p.tiles_m - first_m);
+  const int within = local - band * GROUP_M * p.tiles_n;
+  t.mb = first_m + within % gm;
+  t.nb = within / gm;
+  return t;
+}
+
+template <bool A_MN, bool B_MN, bool OUT_F32>
+__global__ void __launch_bounds__(kThreads, 1)
+umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
+                      const __grid_constant__ CUtensorMap tma_b, const PairParams p) {
+  constexpr int STAGES = 6;
+  constexpr int A_BYTES = 128 * BK * 2;  // this CTA's 128 rows of A, 16 KB
+  constexpr int B_BYTES = 128 * BK * 2;  // this CTA's 128 rows (N) of B, 16 KB
+  constexpr int ACC_COLS = 256;
+  constexpr uint32_t TMEM_COLS = 2 * ACC_COLS;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + STAGES * B_BYTES);
+  uint64_t* full = bars;                   // used in the leader only
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = bars + 2 * STAGES + 2;  // used in the leader only (8 arrivals)
+  uint64_t* drain = bars + 2 * STAGES + 4;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const Ctl ctl{abort_flag, p.err};
+  const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(tfull + a), 1);
+      mbar_init(smem_u32(tempty + a), 8);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
+        const TileCoord tc = decode_pair_tile(p, tile);
+        const int kb0 = tc.split * p.kblocks_per_split;
+        const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
+        const int am = tc.g * p.a_gm + tc.mb * 256 + (int)rank * 128, ak = tc.g * p.a_gk;
+        const int bn = tc.g * p.b_gn + tc.nb * 256 + (int)rank * 128, bk = tc.g * p.b_gk;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_bounded(smem_u32(empty + s), ph ^ 1u, ctl, kErrProducer, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
+          if (leader) mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + B_BYTES));
+          const int k = kb * BK;
+          if constexpr (A_MN) {
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, am, ak + k);
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), &tma_a, fb, am + 64,
+                             ak + k);
+          } else {
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k, am);
+          }
+          if constexpr (B_MN) {
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn, bk + k);
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb, bn + 64,
+                             bk + k);
+          } else {
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k, bn);
+          }
+        }
+      }
+      if (!ok && leader) {
+        // the leader's full barriers count both CTAs' bytes: let them land
+        for (int j = max(0, it - STAGES); j < it; ++j)
+          wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
+                       kDrainLimitNs);
+      }
+    }
+    __syncwarp();  // reconverge before the block-wide barriers below
+  } else if (warp == 1) {
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = instr_desc_pair<A_MN, B_MN>();
+      int it = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
+        const TileCoord tc = decode_pair_tile(p, tile);
+        const int kb0 = tc.split * p.kblocks_per_split;
+        const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
+        const int acc = tcount & 1;
+        const uint32_t use = (uint32_t)(tcount >> 1);
+        if (!wait_bounded(smem_u32(tempty + acc), (use & 1u) ^ 1u, ctl, kErrMma, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(acc * ACC_COLS);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!wait_bounded(smem_u32(full + s), ph, ctl, kErrMma, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sa + s * A_BYTES), b0 = smem_u32(sb + s * B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            const uint64_t ad = A_MN ? smem_desc(a0 + kk * 2048, 64 * BK * 2, 1024)
+                                     : smem_desc(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = B_MN ? smem_desc(b0 + kk * 2048, 64 * BK * 2, 1024)
+                                     : smem_desc(b0 + kk * 32, 16, 1024);
+            umma_bf16_pair(d, ad, bd, idesc, (kb > kb0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit_pair_both(smem_u32(empty + s));
+        }
+        if (!ok) break;
+        umma_commit_pair_both(smem_u32(tfull + acc));
+      }
+      umma_commit_pair_both(smem_u32(drain));
+      wait_bounded(smem_u32(drain), 0, ctl, ok ? kErrMma : 0, ok ? kWaitLimitNs : kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t leader_tempty0 = map_to_rank(smem_u32(tempty), 0);
+    int tcount = 0;
+    for (int tile = cluster_id; tile < p.total_tiles; tile += num_clusters, ++tcount) {
+      const TileCoord tc = decode_pair_tile(p, tile);
+      const int acc = tcount & 1;
+      const uint32_t use = (uint32_t)(tcount >> 1);
+      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
+      tc_fence_after();
+      const int grow = tc.mb * 256 + (int)rank * 128 + row;
+      const bool live = grow < p.M;
+      const long long base = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
+                             (long long)grow * p.ldc + (long long)tc.nb * 256;
+#pragma unroll 1
+      for (int c = 0; c < ACC_COLS; c += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS + c),
+                  r);
+        if (live) store_row32<OUT_F32>(p.C, base + c, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(leader_tempty0 + (uint32_t)(acc * 8));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync_all();   // no remote arrive or copy may target a CTA that has left
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -462,6 +733,53 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   return cudaGetLastError();
 }
 
+template <bool A_MN, bool B_MN, bool OUT_F32>
+cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
+  constexpr int STAGES = 6;
+  constexpr size_t smem = (size_t)STAGES * (128 * BK * 2 * 2) + 1024 + 256;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : 128)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
+  PairParams p;
+  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = (int)g.groups;
+  p.tiles_m = (int)((g.M + 255) / 256);
+  p.tiles_n = (int)(g.N / 256);
+  const int kblocks = (int)((g.K + BK - 1) / BK);
+  p.splits = effective_splits(g.K, g.splits);
+  p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
+  p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
+  p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
+  p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
+  p.err = device_error_word();
+  auto kern = umma_gemm_pair_kernel<A_MN, B_MN, OUT_F32>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;
+  if (!max_clusters) {
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess ||
+        max_clusters <= 0)
+      max_clusters = sm_count() / 2;
+  }
+  const int clusters = std::min(p.total_tiles, max_clusters);
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  TraceScope t(name, s);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int BN>
 cudaError_t dispatch_majors(const Gemm& g, cudaStream_t s) {
 #define POETX_UM(AM, BMJ, F)                                                                   \
@@ -501,6 +819,24 @@ bool supported(const Gemm& g) {
   if (g.a_rows >= lim || g.a_cols >= lim || g.b_rows >= lim || g.b_cols >= lim) return false;
   if ((g.a_gm | g.a_gk | g.b_gn | g.b_gk) % 64) return false;
   return true;
+}
+
+bool pair_supported(const Gemm& g) {
+  return supported(g) && g.N % 256 == 0 && g.M >= 256 && !(g.a_mn && !g.b_mn) &&
+         !(g.a_mn && g.b_mn && !g.out_f32) && (g.groups == 1 || g.a_gm == 0 || g.a_gm % 256 == 0);
+}
+
+cudaError_t gemm_pair(const Gemm& g, cudaStream_t s) {
+  const char* name = g.name ? g.name : "umma_gemm_pair";
+#define POETX_UP(AM, BMJ, F) \
+  if (g.a_mn == AM && g.b_mn == BMJ && g.out_f32 == F) return launch_pair_t<AM, BMJ, F>(g, s, name);
+  POETX_UP(false, false, false)
+  POETX_UP(false, true, false)
+  POETX_UP(true, true, true)
+  POETX_UP(false, false, true)
+  POETX_UP(false, true, true)
+#undef POETX_UP
+  return cudaErrorNotSupported;
 }
 
 cudaError_t gemm(const Gemm& g, cudaStream_t s) {

@@ -25,6 +25,10 @@ struct Gemm {
 };
 
 bool supported(const Gemm& g);
+// The same product on CTA pairs (tcgen05.mma.cta_group::2, 256 x 256 pair tiles); needs
+// N % 256 == 0 and M >= 256.
+bool pair_supported(const Gemm& g);
+cudaError_t gemm_pair(const Gemm& g, cudaStream_t s);
 
 // Number of K ranges the kernel actually uses for `splits` requested ranges over K
 // (ranges of whole 64-wide K blocks, none empty).

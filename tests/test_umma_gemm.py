@@ -67,3 +67,34 @@ def test_umma_gemm_rejects_uncovered_shapes():
     with pytest.raises(poetx.PoetxError) as e:
         poetx.testing_gemm_bf16(a, False, b, False, 128, 48, 64, c)
     assert e.value.status == 7
+
+
+# ------------------------------------------------------------------ CTA-pair kernel
+@pytest.mark.parametrize("a_mn,b_mn,f32", LAYOUTS)
+@pytest.mark.parametrize("M,N,K", [(256, 256, 64), (304, 512, 192), (1000, 256, 1024),
+                                   (512, 768, 320)])
+def test_umma_pair_gemm_matches_fp32_matmul(a_mn, b_mn, f32, M, N, K):
+    a, b, ref = _operands(M, N, K, a_mn, b_mn, seed=M * 3 + N + K)
+    c = torch.empty(M, N, device="cuda", dtype=torch.float32 if f32 else torch.bfloat16)
+    poetx.testing_gemm_bf16(a, a_mn, b, b_mn, M, N, K, c, variant=1)
+    torch.cuda.synchronize()
+    poetx.device_status()
+    err = (c.float().cpu() - ref).abs().max().item() / ref.abs().max().item()
+    assert err < (2e-6 * K ** 0.5 if f32 else 6e-3), err
+
+
+def test_umma_pair_gemm_split_k_and_identity():
+    M, N, K = 512, 256, 1000
+    a, b, ref = _operands(M, N, K, True, True, seed=7)
+    c = torch.full((4, M, N), float("nan"), device="cuda")
+    poetx.testing_gemm_bf16(a, True, b, True, M, N, K, c, splits=4, variant=1)
+    torch.cuda.synchronize()
+    total = c.sum(0).cpu()
+    assert (total - ref).abs().max().item() / ref.abs().max().item() < 1e-5
+    A = torch.randn(384, 256).to(torch.bfloat16).cuda()
+    eye = torch.eye(256, dtype=torch.bfloat16, device="cuda")
+    for b_mn in (False, True):
+        out = torch.empty(384, 256, device="cuda", dtype=torch.bfloat16)
+        poetx.testing_gemm_bf16(A, False, eye, b_mn, 384, 256, 256, out, variant=1)
+        torch.cuda.synchronize()
+        assert torch.equal(out, A)
