@@ -271,7 +271,7 @@ def run_ours(args):
     dq_r = torch.empty_like(q_r)
     dq_p = torch.empty_like(q_p)
     ws = torch.empty(max(poetx.fwd_workspace_bytes(layer, T), poetx.bwd_workspace_bytes(layer, T),
-                         poetx.cnp_workspace_bytes(max(m, n) // b, b)),
+                         poetx.layer_cnp_workspace_bytes(layer)),
                      dtype=torch.uint8, device=dev)
     flat_dq = torch.empty(dq_r.numel() + dq_p.numel(), device=dev) if world > 1 else None
     stream = torch.cuda.current_stream(dev)

@@ -94,6 +94,18 @@ poetx_status poetx_cnp_build(const float* q, int64_t nblocks, int64_t b, float* 
                              int32_t lp_dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * poetx_layer_cnp_build — poetx_cnp_build of both sides of a layer in one launch sequence:
+ *   L->q_r -> L->g_r (and L->g_r_lp for BF16 layers), L->q_p -> L->g_p (L->g_p_lp). The same
+ *   arithmetic as two poetx_cnp_build calls; one pass over all m/b + n/b blocks fills the GPU
+ *   better than two.
+ *   workspace >= poetx_layer_cnp_workspace_bytes(L). Errors: as poetx_cnp_build, plus those of
+ *   the layer descriptor (see poetx_linear_fwd) and INVALID_ARG if q_r or q_p is NULL.
+ * ------------------------------------------------------------------------------------------- */
+size_t poetx_layer_cnp_workspace_bytes(const poetx_layer* L);
+poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * poetx_cnp_build_noalloc — poetx_cnp_build for callers that cannot allocate device memory.
  *   The pages have no counterpart to this call; it exists for library users only. Some callers
  *   may not allocate device memory when they build the blocks (a host program that hands out all

@@ -180,9 +180,9 @@ size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
 
 struct BwdWs {
   void *dC, *dB, *dA1, *A, *dA;
-  float *dG_r, *dG_p;
+  float* dG;             // [m/b + n/b][b][b]: the R blocks, then the P blocks
   void* chain;
-  void* partials;
+  void *part_r, *part_p;  // split-K partial sums of dG_R, dG_P
   int32_t* inv;
 };
 size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
@@ -194,14 +194,11 @@ size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   w.dA1 = a.take(T * L->m * e);
   w.A = a.take(T * L->m * e);
   w.dA = a.take(T * L->m * e);
-  w.dG_r = static_cast<float*>(a.take((size_t)(L->m * L->b) * sizeof(float)));
-  w.dG_p = static_cast<float*>(a.take((size_t)(L->n * L->b) * sizeof(float)));
+  w.dG = static_cast<float*>(a.take((size_t)((L->m + L->n) * L->b) * sizeof(float)));
   const DT t = L->dtype == POETX_BF16 ? DT::BF16 : DT::F32;
-  const size_t chain =
-      std::max(gemm_dq_ws_bytes(t, L->m / L->b, L->b), gemm_dq_ws_bytes(t, L->n / L->b, L->b));
-  w.chain = a.take(chain);
-  w.partials = a.take(std::max(block_grad_ws_bytes(t, L->m, L->b, T),
-                               block_grad_ws_bytes(t, L->n, L->b, T)));
+  w.chain = a.take(gemm_dq_ws_bytes(t, L->m / L->b + L->n / L->b, L->b));
+  w.part_r = a.take(block_grad_ws_bytes(t, L->m, L->b, T));
+  w.part_p = a.take(block_grad_ws_bytes(t, L->n, L->b, T));
   w.inv = static_cast<int32_t*>(a.take(L->m * 4));
   if (o) *o = w;
   return a.used;
@@ -319,6 +316,31 @@ poetx_status poetx_cnp_build(const float* q, int64_t nblocks, int64_t b, float* 
   return POETX_OK;
 }
 
+size_t poetx_layer_cnp_workspace_bytes(const poetx_layer* L) {
+  if (!L || L->b < 2 || L->m <= 0 || L->n <= 0) return 0;
+  return gemm_cnp_ws_bytes(L->m / L->b + L->n / L->b, L->b);
+}
+
+poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  poetx_status st = check_layer(L, true);
+  if (st != POETX_OK) return st;
+  if (!L->q_r || !L->q_p) return fail(POETX_ERR_INVALID_ARG, "layer has no q");
+  if ((st = check_ws(workspace, ws_bytes, poetx_layer_cnp_workspace_bytes(L))) != POETX_OK)
+    return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  BlockRuns r;
+  const bool lp = L->dtype == POETX_BF16;
+  r.q[0] = L->q_r; r.g[0] = L->g_r; r.nb[0] = r.nb0 = (int)(L->m / L->b);
+  r.q[1] = L->q_p; r.g[1] = L->g_p; r.nb[1] = (int)(L->n / L->b);
+  if (lp) {
+    r.g_lp[0] = static_cast<__nv_bfloat16*>(L->g_r_lp);
+    r.g_lp[1] = static_cast<__nv_bfloat16*>(L->g_p_lp);
+  }
+  CHECK_CUDA(gemm_cnp_build_runs(r, L->b, workspace, as_stream(stream)), "layer_cnp_build");
+  return POETX_OK;
+}
+
 // ------------------------------------------------------------------ forward
 size_t poetx_fwd_workspace_bytes(const poetx_layer* L, int64_t T) {
   if (!L || T < 0 || L->m <= 0 || L->n <= 0) return 0;
@@ -383,15 +405,11 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
   CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s, "perm_bwd_gather_dY"), "bwd gather dY");
   CHECK_CUDA(gemm_blockwise(t, w.dC, Gp, w.dB, T, n, b, true, s), "bwd P blocks");
-  const float* parts = static_cast<const float*>(w.partials);
-  if (dq_p) {
-    // dG_P, then its dq chain right away: the split-K partials buffer is shared with the R side
-    int sp = 1;
-    CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, w.dG_p, T, n, b, w.partials, &sp, s), "bwd dG_P");
-    CHECK_CUDA(gemm_dq_from_dg(t, L->q_p, sp > 1 ? parts : w.dG_p, sp, w.dG_p, n / b, b, dq_p,
-                               w.chain, s),
-               "dq_p");
-  }
+  float* dG_r = w.dG;
+  float* dG_p = w.dG + (m / b) * b * b;
+  int sp_r = 1, sp_p = 1;
+  if (dq_p)
+    CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, dG_p, T, n, b, w.part_p, &sp_p, s), "bwd dG_P");
   CHECK_CUDA(gemm_dense(t, w.dB, L->w0m, w.dA1, T, m, n, true, s), "bwd W0'^T GEMM");
   if (dx) {
     CHECK_CUDA(gemm_blockwise(t, w.dA1, Gr, w.dA, T, m, b, true, s), "bwd R blocks");
@@ -399,12 +417,24 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
                "bwd scatter dX");
   }
   if (dq_r) {
-    int sp = 1;
     CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_gather_X"), "bwd gather X");
-    CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, w.dG_r, T, m, b, w.partials, &sp, s), "bwd dG_R");
-    CHECK_CUDA(gemm_dq_from_dg(t, L->q_r, sp > 1 ? parts : w.dG_r, sp, w.dG_r, m / b, b, dq_r,
-                               w.chain, s),
-               "dq_r");
+    CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, dG_r, T, m, b, w.part_r, &sp_r, s), "bwd dG_R");
+  }
+  if (dq_r || dq_p) {
+    // one dq chain over the R blocks and the P blocks
+    BlockRuns r;
+    int k = 0;
+    if (dq_r) {
+      r.q[k] = L->q_r; r.dq[k] = dq_r; r.splits[k] = sp_r; r.nb[k] = (int)(m / b);
+      r.parts[k] = sp_r > 1 ? static_cast<const float*>(w.part_r) : dG_r;
+      ++k;
+    }
+    if (dq_p) {
+      r.q[k] = L->q_p; r.dq[k] = dq_p; r.splits[k] = sp_p; r.nb[k] = (int)(n / b);
+      r.parts[k] = sp_p > 1 ? static_cast<const float*>(w.part_p) : dG_p;
+    }
+    r.nb0 = r.nb[0];
+    CHECK_CUDA(gemm_dq_from_dg_runs(t, r, b, dq_r ? dG_r : dG_p, w.chain, s), "dq chain");
   }
   return POETX_OK;
 }

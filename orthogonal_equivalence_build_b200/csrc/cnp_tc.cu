@@ -52,10 +52,9 @@ __device__ __forceinline__ bool pair_ctx(int b, PairCtx& c) {
   return true;
 }
 
-// up <- Q tile (I, J), I <= J, from the packed strict upper triangle of block g.
-__device__ __forceinline__ void load_q_tile(Tile& up, const float* __restrict__ q, int b,
+// up <- Q tile (I, J), I <= J, from the packed strict upper triangle of one block (qb).
+__device__ __forceinline__ void load_q_tile(Tile& up, const float* __restrict__ qb, int b,
                                             const PairCtx& c) {
-  const float* qb = q + (int64_t)c.g * (b * (b - 1) / 2);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = c.ty + 8 * k;
@@ -101,12 +100,14 @@ __device__ __forceinline__ void put_split(__nv_bfloat16* __restrict__ Acat,
 
 // CNP pass 1: X = Y = Q.
 __global__ void __launch_bounds__(kTileThreads)
-split_q_kernel(const float* __restrict__ q, int b, __nv_bfloat16* __restrict__ Acat,
+split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Acat,
                __nv_bfloat16* __restrict__ Bcat) {
   __shared__ Tile up;
   PairCtx c;
   if (!pair_ctx(b, c)) return;
-  load_q_tile(up, q, b, c);
+  int local;
+  const int run = run_of(r, c.g, local);
+  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = c.ty + 8 * k;
@@ -121,12 +122,14 @@ split_q_kernel(const float* __restrict__ q, int b, __nv_bfloat16* __restrict__ A
 
 // CNP pass 2: X = S, Y = 2I + 2Q + S.
 __global__ void __launch_bounds__(kTileThreads)
-split_sh_kernel(const float* __restrict__ q, const float* __restrict__ S, int b,
+split_sh_kernel(const BlockRuns r, const float* __restrict__ S, int b,
                 __nv_bfloat16* __restrict__ Acat, __nv_bfloat16* __restrict__ Bcat) {
   __shared__ Tile up;
   PairCtx c;
   if (!pair_ctx(b, c)) return;
-  load_q_tile(up, q, b, c);
+  int local;
+  const int run = run_of(r, c.g, local);
+  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
   const float* Sg = S + (int64_t)c.g * c.bb;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -146,13 +149,18 @@ split_sh_kernel(const float* __restrict__ q, const float* __restrict__ S, int b,
 
 // CNP finish: G = I + 2Q + P (fp32 and its bf16 copy).
 __global__ void __launch_bounds__(kTileThreads)
-cnp_finish_kernel(const float* __restrict__ q, const float* __restrict__ P, int b,
-                  float* __restrict__ g, __nv_bfloat16* __restrict__ g_lp) {
+cnp_finish_kernel(const BlockRuns r, const float* __restrict__ Pall, int b) {
   __shared__ Tile up;
   PairCtx c;
   if (!pair_ctx(b, c)) return;
-  load_q_tile(up, q, b, c);
-  const int64_t base = (int64_t)c.g * c.bb;
+  int local;
+  const int run = run_of(r, c.g, local);
+  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
+  // P is indexed by the launch-wide block, the outputs by the block within its run
+  const float* P = Pall + ((int64_t)c.g - local) * c.bb;
+  float* g = r.g[run];
+  __nv_bfloat16* g_lp = r.g_lp[run];
+  const int64_t base = (int64_t)local * c.bb;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = c.ty + 8 * k;
@@ -175,14 +183,20 @@ cnp_finish_kernel(const float* __restrict__ q, const float* __restrict__ P, int 
 
 // dq pass 1: Qh = bf16(Q); dG = sum of the split partials (fixed order), dGh = bf16(dG).
 __global__ void __launch_bounds__(kTileThreads)
-dq_prep_kernel(const float* __restrict__ q, const float* __restrict__ parts, int splits,
-               int64_t split_stride, int b, float* __restrict__ dG,
+dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
                __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ dGh) {
   __shared__ Tile up;
   PairCtx c;
   if (!pair_ctx(b, c)) return;
-  load_q_tile(up, q, b, c);
+  int local;
+  const int run = run_of(r, c.g, local);
+  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
   const int64_t base = (int64_t)c.g * c.bb;
+  // this block's partial sums within its run, [splits][nb_run][b][b]
+  const float* pr = r.parts[run] + (int64_t)local * c.bb;
+  const int splits = r.splits[run];
+  const int64_t split_stride = (int64_t)r.nb[run] * c.bb;
+  const bool in_place = splits == 1 && pr == dG + base;  // written straight into dG
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = c.ty + 8 * k;
@@ -190,10 +204,10 @@ dq_prep_kernel(const float* __restrict__ q, const float* __restrict__ parts, int
     for (int h = 0; h < 2; ++h) {
       if (h == 1 && c.diag) break;
       const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
-      const int64_t e = base + (int64_t)i * b + j;
+      const int64_t off = (int64_t)i * b + j, e = base + off;
       float v = 0.f;
-      for (int sp = 0; sp < splits; ++sp) v += parts[sp * split_stride + e];
-      if (splits > 1) dG[e] = v;
+      for (int sp = 0; sp < splits; ++sp) v += pr[sp * split_stride + off];
+      if (!in_place) dG[e] = v;
       dGh[e] = __float2bfloat16_rn(v);
       Qh[e] = __float2bfloat16_rn(h ? -up.v[c.tx][r] : up.v[r][c.tx]);
     }
@@ -202,12 +216,14 @@ dq_prep_kernel(const float* __restrict__ q, const float* __restrict__ parts, int
 
 // dq pass 2: Sh = bf16(S), SmQ = bf16(S - 2Q).
 __global__ void __launch_bounds__(kTileThreads)
-dq_prep2_kernel(const float* __restrict__ q, const float* __restrict__ S, int b,
+dq_prep2_kernel(const BlockRuns r, const float* __restrict__ S, int b,
                 __nv_bfloat16* __restrict__ Sh, __nv_bfloat16* __restrict__ SmQ) {
   __shared__ Tile up;
   PairCtx c;
   if (!pair_ctx(b, c)) return;
-  load_q_tile(up, q, b, c);
+  int local;
+  const int run = run_of(r, c.g, local);
+  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
   const int64_t base = (int64_t)c.g * c.bb;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
@@ -263,8 +279,8 @@ dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
 
 // dq pass 4: U = V - ZQ; dq_ij = U_ij - U_ji (i < j), written packed.
 __global__ void __launch_bounds__(kTileThreads)
-dq_pack_kernel(const float* __restrict__ V, const float* __restrict__ ZQ, int b,
-               float* __restrict__ dq) {
+dq_pack_kernel(const BlockRuns r, const float* __restrict__ V, const float* __restrict__ ZQ,
+               int b) {
   __shared__ Tile ua, ub;  // U tiles (I, J) and (J, I)
   PairCtx c;
   if (!pair_ctx(b, c)) return;
@@ -282,7 +298,9 @@ dq_pack_kernel(const float* __restrict__ V, const float* __restrict__ ZQ, int b,
     }
   }
   __syncthreads();
-  float* dqb = dq + (int64_t)c.g * (b * (b - 1) / 2);
+  int local;
+  const int run = run_of(r, c.g, local);
+  float* dqb = r.dq[run] + (int64_t)local * (b * (b - 1) / 2);
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int r = c.ty + 8 * k;
@@ -323,8 +341,8 @@ size_t cnp_tc_ws_bytes(int64_t nb, int64_t b) {
   return 2 * cat + 2 * f;
 }
 
-cudaError_t cnp_build_tc(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
-                         void* ws, cudaStream_t s) {
+cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s) {
+  const int64_t nb = (int64_t)r.nb[0] + r.nb[1];
   if (nb == 0) return cudaSuccess;
   Arena a(ws, cnp_tc_ws_bytes(nb, b));
   auto* Acat = static_cast<__nv_bfloat16*>(a.take((size_t)(nb * b * 3 * b) * 2));
@@ -335,18 +353,18 @@ cudaError_t cnp_build_tc(const float* q, int64_t nb, int64_t b, float* g, __nv_b
   const int bi = (int)b;
   {
     TraceScope t("cnp_split_Q", s);
-    split_q_kernel<<<grid, kTileThreads, 0, s>>>(q, bi, Acat, Bcat);
+    split_q_kernel<<<grid, kTileThreads, 0, s>>>(r, bi, Acat, Bcat);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Acat, Bcat, S, nb, b, 3 * b, "umma_cnp_QQ", s));
   {
     TraceScope t("cnp_split_SH", s);
-    split_sh_kernel<<<grid, kTileThreads, 0, s>>>(q, S, bi, Acat, Bcat);
+    split_sh_kernel<<<grid, kTileThreads, 0, s>>>(r, S, bi, Acat, Bcat);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Acat, Bcat, P, nb, b, 3 * b, "umma_cnp_SH", s));
   TraceScope t("cnp_finish", s);
-  cnp_finish_kernel<<<grid, kTileThreads, 0, s>>>(q, P, bi, g, g_lp);
+  cnp_finish_kernel<<<grid, kTileThreads, 0, s>>>(r, P, bi);
   return cudaGetLastError();
 }
 
@@ -356,8 +374,8 @@ size_t dq_tc_ws_bytes(int64_t nb, int64_t b) {
   return 5 * h + 3 * f;
 }
 
-cudaError_t dq_from_dg_tc(const float* q, const float* dG_parts, int splits, float* dG,
-                          int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s) {
+cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cudaStream_t s) {
+  const int64_t nb = (int64_t)r.nb[0] + r.nb[1];
   if (nb == 0) return cudaSuccess;
   Arena a(ws, dq_tc_ws_bytes(nb, b));
   const size_t hb = (size_t)(nb * b * b) * 2, fb = (size_t)(nb * b * b) * 4;
@@ -371,30 +389,27 @@ cudaError_t dq_from_dg_tc(const float* q, const float* dG_parts, int splits, flo
   auto* T1 = static_cast<float*>(a.take(fb));
   const dim3 grid = pair_grid(nb, b);
   const int bi = (int)b;
-  // with one split the gradient is read in place; with several it is summed into dG
-  const float* dGsum = splits > 1 ? dG : dG_parts;
   {
     TraceScope t("dq_prep", s);
-    dq_prep_kernel<<<grid, kTileThreads, 0, s>>>(q, dG_parts, splits, nb * b * b, bi, dG, Qh,
-                                                 dGh);
+    dq_prep_kernel<<<grid, kTileThreads, 0, s>>>(r, bi, dG, Qh, dGh);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Qh, Qh, S, nb, b, b, "umma_dq_QQ", s));
   {
     TraceScope t("dq_prep2", s);
-    dq_prep2_kernel<<<grid, kTileThreads, 0, s>>>(q, S, bi, Sh, SmQ);
+    dq_prep2_kernel<<<grid, kTileThreads, 0, s>>>(r, S, bi, Sh, SmQ);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Sh, dGh, Hb, nb, b, b, "umma_dq_SdG", s));
   POETX_TRY(block_product(dGh, SmQ, T1, nb, b, b, "umma_dq_dGH", s));
   {
     TraceScope t("dq_mid", s);
-    dq_mid_kernel<<<grid, kTileThreads, 0, s>>>(dGsum, T1, Hb, bi, Zh, S);
+    dq_mid_kernel<<<grid, kTileThreads, 0, s>>>(dG, T1, Hb, bi, Zh, S);
     POETX_TRY(cudaGetLastError());
   }
   POETX_TRY(block_product(Zh, Qh, T1, nb, b, b, "umma_dq_ZQ", s));
   TraceScope t("dq_pack", s);
-  dq_pack_kernel<<<grid, kTileThreads, 0, s>>>(S, T1, bi, dq);
+  dq_pack_kernel<<<grid, kTileThreads, 0, s>>>(r, S, T1, bi);
   return cudaGetLastError();
 }
 

@@ -169,28 +169,49 @@ size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b) {
 
 cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                            void* ws, cudaStream_t s) {
-  if (tc_blocks_supported(b)) return cnp_build_tc(q, nb, b, g, g_lp, ws, s);
+  if (tc_blocks_supported(b)) {
+    BlockRuns r;
+    r.q[0] = q; r.g[0] = g; r.g_lp[0] = g_lp; r.nb[0] = r.nb0 = (int)nb;
+    return cnp_build_tc(r, b, ws, s);
+  }
   return cnp_build(q, nb, b, g, g_lp, ws, s);
+}
+
+cudaError_t gemm_cnp_build_runs(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s) {
+  if (tc_blocks_supported(b)) return cnp_build_tc(r, b, ws, s);
+  for (int k = 0; k < 2; ++k) {
+    if (!r.nb[k]) continue;
+    cudaError_t e = cnp_build(r.q[k], r.nb[k], b, r.g[k], r.g_lp[k], ws, s);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b) {
   return (t == DT::BF16 && tc_blocks_supported(b)) ? dq_tc_ws_bytes(nb, b) : dq_ws_bytes(nb, b);
 }
 
-cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG_parts, int splits, float* dG,
-                            int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s) {
-  if (t == DT::BF16 && tc_blocks_supported(b))
-    return dq_from_dg_tc(q, dG_parts, splits, dG, nb, b, dq, ws, s);
-  if (splits > 1) {
-    const int64_t count = nb * b * b;
-    TraceScope tr("sum_split_partials", s);
-    sum_partials_kernel<<<(int)std::min<int64_t>((count + 255) / 256, sms() * 8), 256, 0, s>>>(
-        dG_parts, dG, count, splits);
-    cudaError_t e = cudaGetLastError();
+cudaError_t gemm_dq_from_dg_runs(DT t, const BlockRuns& r, int64_t b, float* dG, void* ws,
+                                 cudaStream_t s) {
+  if (t == DT::BF16 && tc_blocks_supported(b)) return dq_from_dg_tc(r, b, dG, ws, s);
+  // fp32 layers: per run, sum split partials if any, then the fp32 SIMT chain
+  float* dGk = dG;
+  for (int k = 0; k < 2; ++k) {
+    if (!r.nb[k]) continue;
+    const int64_t count = (int64_t)r.nb[k] * b * b;
+    const float* src = r.parts[k];
+    if (r.splits[k] > 1 || src != dGk) {
+      TraceScope tr("sum_split_partials", s);
+      sum_partials_kernel<<<(int)std::min<int64_t>((count + 255) / 256, sms() * 8), 256, 0, s>>>(
+          src, dGk, count, r.splits[k]);
+      cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    cudaError_t e = dq_from_dg(r.q[k], dGk, r.nb[k], b, r.dq[k], ws, s);
     if (e != cudaSuccess) return e;
-    dG_parts = dG;
+    dGk += count;
   }
-  return dq_from_dg(q, dG_parts, nb, b, dq, ws, s);
+  return cudaSuccess;
 }
 
 }  // namespace poetx

@@ -30,18 +30,40 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
 bool tc_blocks_supported(int64_t b);
 size_t cnp_tc_ws_bytes(int64_t nb, int64_t b);
 size_t dq_tc_ws_bytes(int64_t nb, int64_t b);
-cudaError_t cnp_build_tc(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
-                         void* ws, cudaStream_t s);
-// dG_parts: `splits` fp32 partial sums [splits][nb][b][b] (splits == 1: the gradient itself);
-// dG: [nb][b][b] fp32 buffer that receives the sum when splits > 1.
-cudaError_t dq_from_dg_tc(const float* q, const float* dG_parts, int splits, float* dG,
-                          int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s);
+
+// Up to two runs of b x b blocks handled by one launch sequence (the R and the P blocks of a
+// layer): launch-wide block j < nb[0] is block j of run 0, otherwise block j - nb[0] of run 1.
+struct BlockRuns {
+  const float* q[2] = {nullptr, nullptr};     // packed skew parameters of each run
+  float* g[2] = {nullptr, nullptr};           // fp32 CNP blocks (may be null)
+  __nv_bfloat16* g_lp[2] = {nullptr, nullptr};  // bf16 copies (may be null)
+  float* dq[2] = {nullptr, nullptr};          // packed gradients
+  const float* parts[2] = {nullptr, nullptr}; // dG split partials [splits][nb][b][b]
+  int splits[2] = {1, 1};
+  int nb[2] = {0, 0};
+  int nb0 = 0;                                // == nb[0]
+};
+__device__ __forceinline__ int run_of(const BlockRuns& r, int g, int& local) {
+  if (g < r.nb0) {
+    local = g;
+    return 0;
+  }
+  local = g - r.nb0;
+  return 1;
+}
+cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s);
+// dG: [nb[0] + nb[1]][b][b] fp32, receives the summed gradients (a run whose parts pointer is
+// its own slice of dG with one split is read in place).
+cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cudaStream_t s);
 
 size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b);
 cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                            void* ws, cudaStream_t s);
+// both runs of a layer in one sequence (tensor cores), or one after the other (SIMT)
+cudaError_t gemm_cnp_build_runs(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s);
 size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b);
-cudaError_t gemm_dq_from_dg(DT t, const float* q, const float* dG_parts, int splits, float* dG,
-                            int64_t nb, int64_t b, float* dq, void* ws, cudaStream_t s);
+// dq of the runs in r; dG: [nb[0] + nb[1]][b][b] fp32 scratch that receives summed gradients
+cudaError_t gemm_dq_from_dg_runs(DT t, const BlockRuns& r, int64_t b, float* dG, void* ws,
+                                 cudaStream_t s);
 
 }  // namespace poetx

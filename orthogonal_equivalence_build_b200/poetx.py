@@ -50,6 +50,8 @@ def _load() -> ctypes.CDLL:
         "poetx_cnp_workspace_bytes": (SZ, [I64, I64]),
         "poetx_cnp_build": (I32, [V, I64, I64, V, V, I32, V, SZ, V]),
         "poetx_cnp_build_noalloc": (I32, [V, I64, I64, V, V, I32, V]),
+        "poetx_layer_cnp_workspace_bytes": (SZ, [LP]),
+        "poetx_layer_cnp_build": (I32, [LP, V, SZ, V]),
         "poetx_fwd_workspace_bytes": (SZ, [LP, I64]),
         "poetx_linear_fwd": (I32, [LP, V, I64, V, V, V, SZ, V]),
         "poetx_bwd_workspace_bytes": (SZ, [LP, I64]),
@@ -78,6 +80,7 @@ def _load() -> ctypes.CDLL:
 lib = _load()
 EXPORTED = (
     "poetx_cnp_workspace_bytes", "poetx_cnp_build", "poetx_cnp_build_noalloc",
+    "poetx_layer_cnp_workspace_bytes", "poetx_layer_cnp_build",
     "poetx_fwd_workspace_bytes",
     "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
     "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
@@ -180,10 +183,16 @@ def cnp_build_noalloc(q: torch.Tensor, b: int, g: Optional[torch.Tensor] = None,
                                        _stream(stream)))
 
 
+def layer_cnp_workspace_bytes(layer: PoetxLinear) -> int:
+    return int(lib.poetx_layer_cnp_workspace_bytes(ctypes.byref(layer.desc)))
+
+
 def layer_cnp_build(layer: PoetxLinear, workspace: Optional[torch.Tensor] = None,
                     stream=None) -> None:
-    cnp_build(layer.q_r, layer.b, layer.g_r, layer.g_r_lp, workspace, stream)
-    cnp_build(layer.q_p, layer.b, layer.g_p, layer.g_p_lp, workspace, stream)
+    """CNP blocks of both sides of the layer (poetx_layer_cnp_build)."""
+    ws = _workspace(layer_cnp_workspace_bytes(layer), layer.w0m.device, workspace)
+    _check(lib.poetx_layer_cnp_build(ctypes.byref(layer.desc), _ptr(ws),
+                                     0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def fwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:

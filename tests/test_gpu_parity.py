@@ -186,3 +186,36 @@ def test_full_size_sampled(key):
                        h["q_p"], c.b)
     assert rel_err(dq_r, ref["dq_r"]) <= TOL_BF16
     assert rel_err(dq_p, ref["dq_p"]) <= TOL_BF16
+
+
+# ------------------------------------------------------------------ layer-level CNP and one-sided dq
+@pytest.mark.parametrize("key,m,n,b", [("llama8b_up_proj", 1024, 3584, 512),
+                                       ("tiny_fp32", 512, 768, 64)])
+def test_layer_cnp_build_matches_per_side_builds(key, m, n, b):
+    """One launch sequence over the R and P blocks gives the per-side results bit for bit."""
+    c = LayerCase(key, m=m, n=n, b=b, tokens=8)
+    lay = c.layer
+    g_r = torch.empty_like(lay.g_r)
+    g_p = torch.empty_like(lay.g_p)
+    lp_r = torch.empty_like(lay.g_r_lp) if lay.g_r_lp is not None else None
+    lp_p = torch.empty_like(lay.g_p_lp) if lay.g_p_lp is not None else None
+    poetx.cnp_build(c.q_r, b, g_r, lp_r)
+    poetx.cnp_build(c.q_p, b, g_p, lp_p)
+    torch.cuda.synchronize()
+    assert torch.equal(g_r, lay.g_r) and torch.equal(g_p, lay.g_p)
+    if lp_r is not None:
+        assert torch.equal(lp_r, lay.g_r_lp) and torch.equal(lp_p, lay.g_p_lp)
+
+
+@pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 700),
+                                         ("tiny_fp32", 256, 512, 64, 99)])
+def test_one_sided_dq_matches_two_sided(key, m, n, b, T):
+    c = LayerCase(key, m=m, n=n, b=b, tokens=T)
+    y, bsave = c.forward()
+    dx, dq_r, dq_p = c.backward(bsave)
+    only_r = torch.empty_like(dq_r)
+    only_p = torch.empty_like(dq_p)
+    poetx.linear_bwd(c.layer, c.x, c.dy, bsave, None, only_r, None)
+    poetx.linear_bwd(c.layer, c.x, c.dy, bsave, None, None, only_p)
+    torch.cuda.synchronize()
+    assert torch.equal(only_r, dq_r) and torch.equal(only_p, dq_p)
