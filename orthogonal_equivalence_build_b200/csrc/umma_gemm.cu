@@ -186,24 +186,59 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile) {
   return t;
 }
 
-// Store 32 accumulator columns of one row (already in registers) as fp32 or bf16.
+// Epilogue of one warp's 32 accumulator rows: TMEM -> registers -> a swizzled 8 KB stage in
+// shared memory -> global memory, 64 columns at a time. Each store instruction of the warp writes
+// whole row segments (4 rows x 128 B for bf16, 2 rows x 256 B for fp32) instead of one 16 B piece
+// of 32 different rows. tmem_row0: TMEM address of this warp's lane quarter at the tile's first
+// column; off0: element offset of the warp's first row in C at the tile's first column.
+constexpr int kEpiStageBytes = 8192;
+
 template <bool OUT_F32>
-__device__ __forceinline__ void store_row32(void* C, long long off, const uint32_t (&r)[32]) {
-  if constexpr (OUT_F32) {
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(C) + off);
+__device__ __forceinline__ void epilogue_warp_rows(uint32_t tmem_row0, int ncols,
+                                                   uint8_t* __restrict__ stage, void* C,
+                                                   long long off0, long long ldc, int nlive,
+                                                   int lane) {
+  constexpr int ESZ = OUT_F32 ? 4 : 2;
+  constexpr int ROWB = 64 * ESZ;      // bytes of one row per 64-column chunk
+  constexpr int V16 = ROWB / 16;      // 16-byte pieces per row chunk: 8 (bf16) or 16 (fp32)
+  constexpr int RPI = 32 / V16;       // rows per store instruction: 4 or 2
+  uint8_t* myrow = stage + lane * ROWB;
+  const int sub = lane % V16, rsub = lane / V16;
+  char* Cb = static_cast<char*>(C);
+#pragma unroll 1
+  for (int c = 0; c < ncols; c += 64) {
+    uint32_t r0[32], r1[32];
+    tmem_ld32(tmem_row0 + (uint32_t)c, r0);
+    tmem_ld32(tmem_row0 + (uint32_t)(c + 32), r1);
+    if constexpr (OUT_F32) {
 #pragma unroll
-    for (int v = 0; v < 8; ++v)
-      dst[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                           __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-  } else {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(C) + off);
+      for (int v = 0; v < 16; ++v) {
+        const uint32_t* src = v < 8 ? &r0[4 * v] : &r1[4 * (v - 8)];
+        *reinterpret_cast<uint4*>(myrow + ((v ^ (lane & 15)) * 16)) =
+            make_uint4(src[0], src[1], src[2], src[3]);
+      }
+    } else {
 #pragma unroll
-    for (int v = 0; v < 4; ++v)
-      dst[v] = make_uint4(
-          pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-          pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-          pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-          pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+      for (int v = 0; v < 8; ++v) {
+        const uint32_t* src = v < 4 ? &r0[8 * v] : &r1[8 * (v - 4)];
+        *reinterpret_cast<uint4*>(myrow + ((v ^ (lane & 7)) * 16)) = make_uint4(
+            pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+            pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+            pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+            pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 32 / RPI; ++i) {
+      const int r = i * RPI + rsub;
+      if (r < nlive) {
+        const uint4 v =
+            *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
+        *reinterpret_cast<uint4*>(Cb + (off0 + (long long)r * ldc + c) * ESZ + sub * 16) = v;
+      }
+    }
+    __syncwarp();
   }
 }
 
@@ -219,7 +254,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sa = smem;
   uint8_t* sb = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + STAGES * B_BYTES);
+  uint8_t* sepi = sb + STAGES * B_BYTES;   // 4 epilogue warps x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + 4 * kEpiStageBytes);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -352,7 +388,6 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
   } else {
     // ------------------------------------------------------------ epilogue (warps 2..5)
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
     int tcount = 0;
     for (int tile = blockIdx.x; tile < p.total_tiles; tile += gridDim.x, ++tcount) {
       const TileCoord tc = decode_tile(p, tile);
@@ -360,16 +395,13 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
       const uint32_t use = (uint32_t)(tcount >> 1);
       if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
       tc_fence_after();
-      const int grow = tc.mb * BM + row;
-      const bool live = grow < p.M;
-      const long long base = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
-                             (long long)grow * p.ldc + (long long)tc.nb * BN;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN + c), r);
-        if (live) store_row32<OUT_F32>(p.C, base + c, r);
-      }
+      const int row0 = tc.mb * BM + quarter * 32;   // first row of this warp
+      const int nlive = max(0, min(32, p.M - row0));
+      const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
+                             (long long)row0 * p.ldc + (long long)tc.nb * BN;
+      epilogue_warp_rows<OUT_F32>(
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN), BN,
+          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
@@ -491,7 +523,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sa = smem;
   uint8_t* sb = smem + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sb + STAGES * B_BYTES);
+  uint8_t* sepi = sb + STAGES * B_BYTES;   // 4 epilogue warps x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + 4 * kEpiStageBytes);
   uint64_t* full = bars;                   // used in the leader only
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
@@ -620,7 +653,6 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     __syncwarp();
   } else {
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
     const uint32_t leader_tempty0 = map_to_rank(smem_u32(tempty), 0);
     int tcount = 0;
     for (int tile = cluster_id; tile < p.total_tiles; tile += num_clusters, ++tcount) {
@@ -629,17 +661,13 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       const uint32_t use = (uint32_t)(tcount >> 1);
       if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
       tc_fence_after();
-      const int grow = tc.mb * 256 + (int)rank * 128 + row;
-      const bool live = grow < p.M;
-      const long long base = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
-                             (long long)grow * p.ldc + (long long)tc.nb * 256;
-#pragma unroll 1
-      for (int c = 0; c < ACC_COLS; c += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS + c),
-                  r);
-        if (live) store_row32<OUT_F32>(p.C, base + c, r);
-      }
+      const int row0 = tc.mb * 256 + (int)rank * 128 + quarter * 32;
+      const int nlive = max(0, min(32, p.M - row0));
+      const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
+                             (long long)row0 * p.ldc + (long long)tc.nb * 256;
+      epilogue_warp_rows<OUT_F32>(
+          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS), ACC_COLS,
+          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader_tempty0 + (uint32_t)(acc * 8));
@@ -709,7 +737,8 @@ constexpr int stages_for() {
 template <int BN, bool A_MN, bool B_MN, bool OUT_F32>
 cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   constexpr int STAGES = stages_for<BN>();
-  constexpr size_t smem = (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 1024 + 256;
+  constexpr size_t smem =
+      (size_t)STAGES * (BM * BK * 2 + BN * BK * 2) + 4 * kEpiStageBytes + 1024 + 256;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : BM)) return cudaErrorInvalidValue;
   if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : BN)) return cudaErrorInvalidValue;
@@ -736,7 +765,7 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
 template <bool A_MN, bool B_MN, bool OUT_F32>
 cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   constexpr int STAGES = 6;
-  constexpr size_t smem = (size_t)STAGES * (128 * BK * 2 * 2) + 1024 + 256;
+  constexpr size_t smem = (size_t)STAGES * (128 * BK * 2 * 2) + 4 * kEpiStageBytes + 1024 + 256;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : 128)) return cudaErrorInvalidValue;
   if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
