@@ -152,10 +152,15 @@ poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, vo
  *     dA_j = dA'_j (G_R^j)^T;  dG_R^j = A_j^T dA'_j (A = X[:, perm_r]);  dX[:, perm_r] = dA;
  *     dq = skew-packed gradient of the CNP polynomial at q (chain rule through G(Q)).
  *   x [T, m], dy [T, n], saved_b [T, n] (from the forward on the same x and layer state).
+ *   saved_b may be NULL (memory-saving mode, "POET-Xmem" in "POET-X: Memory-efficient LLM
+ *   Training ..." §2 Metodologia / the POET-X blog §第五斧): B is then rebuilt exactly as
+ *   (X[:, perm_r] Diag(G_R)) W0' inside the call, which costs one more W0' product (2 T m n
+ *   FLOP) and needs no [T, n] buffer between forward and backward. (The pages' cheaper
+ *   B = C G_P^T is exact only for orthogonal G, which CNP is not, so it is not used.)
  *   dx [T, m] output (may be NULL to skip it);  dq_r [m/b, b(b-1)/2], dq_p [n/b, b(b-1)/2]
  *   fp32 outputs (either may be NULL to skip that side). Uses L->q_r/q_p and the G blocks.
  *   workspace >= poetx_bwd_workspace_bytes(L, T).
- *   Errors: as poetx_linear_fwd; saved_b and dy must not be NULL.
+ *   Errors: as poetx_linear_fwd; dy must not be NULL.
  * ------------------------------------------------------------------------------------------- */
 size_t poetx_bwd_workspace_bytes(const poetx_layer* L, int64_t T);
 poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* dy,

@@ -180,6 +180,7 @@ size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
 
 struct BwdWs {
   void *dC, *dB, *dA1, *A, *dA;
+  void* B;               // recomputed forward product when the caller did not keep it
   float* dG;             // [m/b + n/b][b][b]: the R blocks, then the P blocks
   void* chain;
   void *part_r, *part_p;  // split-K partial sums of dG_R, dG_P
@@ -194,6 +195,7 @@ size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   w.dA1 = a.take(T * L->m * e);
   w.A = a.take(T * L->m * e);
   w.dA = a.take(T * L->m * e);
+  w.B = a.take(T * L->n * e);
   w.dG = static_cast<float*>(a.take((size_t)((L->m + L->n) * L->b) * sizeof(float)));
   const DT t = L->dtype == POETX_BF16 ? DT::BF16 : DT::F32;
   w.chain = a.take(gemm_dq_ws_bytes(t, L->m / L->b + L->n / L->b, L->b));
@@ -389,8 +391,8 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   if (T < 0) return fail(POETX_ERR_SHAPE, "T < 0");
   if ((dq_r && !L->q_r) || (dq_p && !L->q_p))
     return fail(POETX_ERR_INVALID_ARG, "dq requested but the layer has no q");
-  if (!x || !dy || !saved_b) return fail(POETX_ERR_INVALID_ARG, "x, dy or saved_b is NULL");
-  if (!aligned16(x) || !aligned16(dy) || !aligned16(saved_b) || (dx && !aligned16(dx)) ||
+  if (!x || !dy) return fail(POETX_ERR_INVALID_ARG, "x or dy is NULL");
+  if (!aligned16(x) || !aligned16(dy) || (saved_b && !aligned16(saved_b)) || (dx && !aligned16(dx)) ||
       (dq_r && !aligned16(dq_r)) || (dq_p && !aligned16(dq_p)))
     return fail(POETX_ERR_ALIGN, "backward pointers must be 16-byte aligned");
   if ((st = check_ws(workspace, ws_bytes, poetx_bwd_workspace_bytes(L, T))) != POETX_OK) return st;
@@ -403,6 +405,14 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   const int64_t m = L->m, n = L->n, b = L->b;
   const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
+  if (!saved_b && (dq_p || dq_r)) {
+    // memory-saving mode: rebuild B = (X[:, perm_r] Diag(G_R)) W0' exactly instead of keeping it
+    CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_regather_X"),
+               "bwd recompute gather");
+    CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.dA, T, m, b, false, s), "bwd recompute R blocks");
+    CHECK_CUDA(gemm_dense(t, w.dA, L->w0m, w.B, T, n, m, false, s), "bwd recompute W0' GEMM");
+    saved_b = w.B;
+  }
   CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s, "perm_bwd_gather_dY"), "bwd gather dY");
   CHECK_CUDA(gemm_blockwise(t, w.dC, Gp, w.dB, T, n, b, true, s), "bwd P blocks");
   float* dG_r = w.dG;

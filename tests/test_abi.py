@@ -77,6 +77,7 @@ def test_backward_argument_checks():
     L = _layer()
     bwd = poetx.lib.poetx_linear_bwd
     assert bwd(ctypes.byref(L), 0x100000, None, 0x300000, 128, None, None, None, None, 0, None) == 1
+    assert bwd(ctypes.byref(L), None, 0x200000, None, 128, None, None, None, None, 0, None) == 1
     L2 = _layer(q_r=None)
     assert bwd(ctypes.byref(L2), 0x100000, 0x200000, 0x300000, 128, None, 0x500000, None,
                None, 0, None) == 1
@@ -114,3 +115,21 @@ def test_workspace_queries_scale_with_tokens():
     f = poetx.lib.poetx_fwd_workspace_bytes
     assert f(ctypes.byref(L), 256) > f(ctypes.byref(L), 128) > 0
     assert poetx.lib.poetx_fwd_workspace_bytes(None, 128) == 0
+
+
+def test_workspaces_never_hold_an_m_by_n_buffer():
+    """R W0 P is never formed: the token-independent part of the forward/backward workspace
+    grows linearly with m + n (b x b blocks), not with m * n."""
+    def ws(fn, m, n, T):
+        L = _layer(m=m, n=n, b=512)
+        return fn(ctypes.byref(L), T)
+    for fn in (poetx.lib.poetx_fwd_workspace_bytes, poetx.lib.poetx_bwd_workspace_bytes):
+        base = ws(fn, 4096, 14336, 16)
+        double = ws(fn, 8192, 28672, 16)
+        assert double < 2.2 * base, (fn.__name__, base, double)
+        assert ws(fn, 4096, 14336, 1) < 4096 * 14336 * 2 * 3   # below three copies of W0'
+    # activations scale with T only
+    f = poetx.lib.poetx_fwd_workspace_bytes
+    L = _layer(m=4096, n=14336, b=512)
+    assert f(ctypes.byref(L), 2048) - f(ctypes.byref(L), 1024) == \
+        f(ctypes.byref(L), 4096) - f(ctypes.byref(L), 3072)

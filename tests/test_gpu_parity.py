@@ -219,3 +219,94 @@ def test_one_sided_dq_matches_two_sided(key, m, n, b, T):
     poetx.linear_bwd(c.layer, c.x, c.dy, bsave, None, None, only_p)
     torch.cuda.synchronize()
     assert torch.equal(only_r, dq_r) and torch.equal(only_p, dq_p)
+
+
+# ------------------------------------------------------------------ memory-saving backward
+@pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 700),
+                                         ("tiny_fp32", 256, 512, 64, 99)])
+def test_backward_without_saved_b_is_identical(key, m, n, b, T):
+    """saved_b = NULL rebuilds B exactly with the same kernels: results equal bit for bit."""
+    c = LayerCase(key, m=m, n=n, b=b, tokens=T)
+    y, bsave = c.forward()
+    dx, dq_r, dq_p = c.backward(bsave)
+    dx2 = torch.empty_like(dx)
+    dq_r2, dq_p2 = torch.empty_like(dq_r), torch.empty_like(dq_p)
+    poetx.linear_bwd(c.layer, c.x, c.dy, None, dx2, dq_r2, dq_p2)
+    torch.cuda.synchronize()
+    assert torch.equal(dx2, dx) and torch.equal(dq_r2, dq_r) and torch.equal(dq_p2, dq_p)
+
+
+# ------------------------------------------------------------------ more full-size shapes
+@pytest.mark.parametrize("key,layer", [("llama8b_decoder", 1),    # k_proj 4096 x 1024
+                                       ("llama8b_decoder", 6),    # down_proj 14336 x 4096
+                                       ("llama13b_layers", 4)])   # gate 5120 x 13824
+def test_full_size_sampled_other_linears(key, layer):
+    c = LayerCase(key, layer)
+    h = c.host()
+    rows = np.sort(np.random.default_rng(layer).choice(c.T, 8, replace=False))
+    G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
+    y, bsave = c.forward()
+    dy_sparse = torch.zeros_like(c.dy)
+    idx = torch.from_numpy(rows).cuda()
+    dy_sparse[idx] = c.dy[idx]
+    dx, dq_r, dq_p = c.backward(bsave, dy=dy_sparse)
+    torch.cuda.synchronize()
+    Xs, dYs = h["X"][rows], h["dY"][rows]
+    ref = O.linear_bwd(Xs, dYs, h["W0m"], h["perm_r"], h["perm_p"], G_r, G_p, h["q_r"],
+                       h["q_p"], c.b)
+    assert rel_err(y[rows], ref["Y"]) <= TOL_BF16
+    assert rel_err(dx[rows], ref["dX"]) <= TOL_BF16
+    assert rel_err(dq_r, ref["dq_r"]) <= TOL_BF16
+    assert rel_err(dq_p, ref["dq_p"]) <= TOL_BF16
+
+
+# ------------------------------------------------------------------ 13B layer: 400 steps + merge
+@pytest.mark.slow
+def test_llama13b_layer_400_steps_with_merge_reinit():
+    """The 13B layer-set schedule on its q/k/v/o shape (5120 x 5120, b = 512, 8192 tokens): 400
+    fwd+bwd steps with q += N(0, 1e-4^2) after each, merge_reinit at step 400, one more step.
+    The oracle replays the same float32 q sequence and checks sampled rows of Y at steps 1, 2,
+    400 and 401 and the merged weight."""
+    import poetx_workloads as W
+    wl = W.WORKLOADS["llama13b_layers"]
+    c = LayerCase("llama13b_layers", 0)
+    h = c.host()
+    rows = np.sort(np.random.default_rng(13).choice(c.T, 6, replace=False))
+    Xs = h["X"][rows]
+    q_r, q_p = h["q_r"].astype(np.float32).copy(), h["q_p"].astype(np.float32).copy()
+    W0m = h["W0m"].astype(np.float64)
+    pr, pp = h["perm_r"], h["perm_p"]
+    checks = {1, 2, 400, 401}
+
+    def check(step):
+        y, _ = c.forward()
+        torch.cuda.synchronize()
+        ref = O.linear_fwd_rows(Xs, W0m, pr, pp, O.cnp(q_r, c.b), O.cnp(q_p, c.b))
+        assert rel_err(y[rows], ref) <= TOL_BF16, step
+
+    for step in range(1, 402):
+        poetx.layer_cnp_build(c.layer)
+        if step in checks:
+            check(step)
+        y, bsave = c.forward()
+        poetx.linear_bwd(c.layer, c.x, c.dy, bsave, None, torch.empty_like(c.q_r),
+                         torch.empty_like(c.q_p))
+        if step == 400:
+            seed = 0x13B0400
+            poetx.layer_cnp_build(c.layer)
+            poetx.merge_reinit(c.layer, seed)
+            torch.cuda.synchronize()
+            ref = O.merge_reinit(W0m, pr, pp, q_r, q_p, c.b, seed)
+            assert rel_err(c.layer.w0m, ref["W0m"]) <= TOL_BF16
+            assert np.array_equal(c.perm_r.cpu().numpy(), ref["perm_r"])
+            W0m, pr, pp = ref["W0m"], ref["perm_r"], ref["perm_p"]
+            q_r[:] = 0
+            q_p[:] = 0
+        # harness perturbation, identical float32 arithmetic on both sides
+        d_r = W.q_perturbation(wl, 0, step, 0, q_r.shape)
+        d_p = W.q_perturbation(wl, 0, step, 1, q_p.shape)
+        c.q_r += torch.from_numpy(d_r).cuda()
+        c.q_p += torch.from_numpy(d_p).cuda()
+        q_r += d_r
+        q_p += d_p
+    assert np.array_equal(c.q_r.cpu().numpy(), q_r)
