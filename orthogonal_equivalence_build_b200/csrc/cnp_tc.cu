@@ -22,11 +22,13 @@ namespace poetx {
 namespace {
 
 // ---------------------------------------------------------------- 32 x 32 mirrored tile pairs
-// Every elementwise pass works on a pair of tiles (I, J), (J, I) with I <= J of one b x b block:
-// loads and stores stay coalesced along rows, transposes go through shared memory, and the
-// packed q of the pair is read once (its upper tile is contiguous along each row).
+// Every elementwise pass works on a pair of tiles (I, J), (J, I) with I <= J of one b x b block;
+// only those pairs are launched (nt (nt + 1) / 2 per block). A thread owns one row and four
+// consecutive columns of each tile: 16-byte loads, 8-byte bf16 stores, rows stay coalesced, and
+// the transposes go through shared memory (conflict-free: the padded row stride is 33 floats).
+// The packed q of a pair is read once (its upper tile is contiguous along each row).
 constexpr int TS = 32;
-constexpr int kTileThreads = 256;  // 32 x 8: thread (tx, ty) owns rows ty, ty+8, ty+16, ty+24
+constexpr int kTileThreads = 256;  // thread (tx, ty): row ty, columns 4 tx .. 4 tx + 3
 
 struct Tile {
   float v[TS][TS + 1];
@@ -34,68 +36,97 @@ struct Tile {
 
 struct PairCtx {
   int g, I, J;      // block, tile row, tile column (I <= J)
-  int tx, ty;
+  int r, c0;        // this thread's row in a tile and first of its four columns
   bool diag;
   int64_t bb;       // b * b
 };
 
-__device__ __forceinline__ bool pair_ctx(int b, PairCtx& c) {
+__device__ __forceinline__ void pair_ctx(int b, PairCtx& c) {
   const int nt = b / TS;
-  c.I = blockIdx.x / nt;
-  c.J = blockIdx.x - c.I * nt;
-  if (c.I > c.J) return false;
+  int p = blockIdx.x, I = 0;
+  while (p >= nt - I) {  // tile row I holds the pairs (I, I .. nt - 1)
+    p -= nt - I;
+    ++I;
+  }
+  c.I = I;
+  c.J = I + p;
   c.g = blockIdx.y;
-  c.tx = threadIdx.x & 31;
-  c.ty = threadIdx.x >> 5;
+  c.r = threadIdx.x >> 3;
+  c.c0 = (threadIdx.x & 7) * 4;
   c.diag = c.I == c.J;
   c.bb = (int64_t)b * b;
-  return true;
+}
+
+dim3 pair_grid(int64_t nb, int64_t b) {
+  const int nt = (int)(b / TS);
+  return dim3((unsigned)(nt * (nt + 1) / 2), (unsigned)nb);
 }
 
 // up <- Q tile (I, J), I <= J, from the packed strict upper triangle of one block (qb).
+// The mirrored tile (J, I) is -up^T: its entry (r, col) is -up.v[col][r].
 __device__ __forceinline__ void load_q_tile(Tile& up, const float* __restrict__ qb, int b,
                                             const PairCtx& c) {
+  const int i = c.I * TS + c.r;
+  const int64_t rowbase = (int64_t)i * b - (int64_t)i * (i + 1) / 2 - i - 1;  // + j for j > i
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    const int i = c.I * TS + r, j = c.J * TS + c.tx;
-    up.v[r][c.tx] = (i < j) ? qb[i * b - i * (i + 1) / 2 + (j - i - 1)] : 0.f;
+    const int j = c.J * TS + c.c0 + k;
+    up.v[c.r][c.c0 + k] = (i < j) ? qb[rowbase + j] : 0.f;
   }
   __syncthreads();
   if (c.diag) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const int r = c.ty + 8 * k;
-      if (r > c.tx) up.v[r][c.tx] = -up.v[c.tx][r];
-    }
+    for (int k = 0; k < 4; ++k)
+      if (c.r > c.c0 + k) up.v[c.r][c.c0 + k] = -up.v[c.c0 + k][c.r];
     __syncthreads();
   }
 }
-// Q tile (J, I) entry (r, col) is -up.v[col][r].
 
-__device__ __forceinline__ void split_bf16(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-  hi = __float2bfloat16_rn(x);
-  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+__device__ __forceinline__ float4 ld4(const float* __restrict__ p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ void st4(float* p, float a, float b2, float c, float d) {
+  *reinterpret_cast<float4*>(p) = make_float4(a, b2, c, d);
+}
+__device__ __forceinline__ uint32_t bf2(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ void st4h(__nv_bfloat16* p, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(bf2(v[0], v[1]), bf2(v[2], v[3]));
+}
+__device__ __forceinline__ void split4(const float (&x)[4], float (&hi)[4], float (&lo)[4]) {
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    hi[k] = __bfloat162float(__float2bfloat16_rn(x[k]));
+    lo[k] = x[k] - hi[k];
+  }
 }
 
-// Concatenated split operands of one block product X Y:
+// Concatenated split operands of one block product X Y, four consecutive columns j .. j+3:
 //   Acat [nb*b][3b]: row (g, i) = [Xhi(i, :) | Xhi(i, :) | Xlo(i, :)]
 //   Bcat [nb*3b][b]: rows (g, k') = Yhi (k' < b), Ylo (b <= k' < 2b), Yhi (2b <= k')
-__device__ __forceinline__ void put_split(__nv_bfloat16* __restrict__ Acat,
-                                          __nv_bfloat16* __restrict__ Bcat, int b, int g, int i,
-                                          int j, float x, float y) {
-  __nv_bfloat16 xh, xl, yh, yl;
-  split_bf16(x, xh, xl);
-  split_bf16(y, yh, yl);
-  __nv_bfloat16* arow = Acat + ((int64_t)g * b + i) * (3 * b);
-  arow[j] = xh;
-  arow[b + j] = xh;
-  arow[2 * b + j] = xl;
-  __nv_bfloat16* bblk = Bcat + (int64_t)g * 3 * b * b;
-  const int64_t e = (int64_t)i * b + j, bb = (int64_t)b * b;
-  bblk[e] = yh;
-  bblk[bb + e] = yl;
-  bblk[2 * bb + e] = yh;
+__device__ __forceinline__ void put_split4(__nv_bfloat16* __restrict__ Acat,
+                                           __nv_bfloat16* __restrict__ Bcat, int b, int g, int i,
+                                           int j, const float (&x)[4], const float (&y)[4]) {
+  float xh[4], xl[4], yh[4], yl[4];
+  split4(x, xh, xl);
+  split4(y, yh, yl);
+  __nv_bfloat16* arow = Acat + ((int64_t)g * b + i) * (3 * b) + j;
+  st4h(arow, xh);
+  st4h(arow + b, xh);
+  st4h(arow + 2 * b, xl);
+  const int64_t bb = (int64_t)b * b;
+  __nv_bfloat16* bp = Bcat + (int64_t)g * 3 * bb + (int64_t)i * b + j;
+  st4h(bp, yh);
+  st4h(bp + bb, yl);
+  st4h(bp + 2 * bb, yh);
+}
+
+__device__ __forceinline__ const float* run_q(const BlockRuns& r, int g, int b, int& run,
+                                              int& local) {
+  run = run_of(r, g, local);
+  return r.q[run] + (int64_t)local * (b * (b - 1) / 2);
 }
 
 // CNP pass 1: X = Y = Q.
@@ -104,19 +135,17 @@ split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Acat,
                __nv_bfloat16* __restrict__ Bcat) {
   __shared__ Tile up;
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
-  int local;
-  const int run = run_of(r, c.g, local);
-  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
+  pair_ctx(b, c);
+  int run, local;
+  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
+  float x[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    const float v = up.v[r][c.tx];
-    put_split(Acat, Bcat, b, c.g, c.I * TS + r, c.J * TS + c.tx, v, v);
-    if (!c.diag) {
-      const float w = -up.v[c.tx][r];
-      put_split(Acat, Bcat, b, c.g, c.J * TS + r, c.I * TS + c.tx, w, w);
-    }
+  for (int k = 0; k < 4; ++k) x[k] = up.v[c.r][c.c0 + k];
+  put_split4(Acat, Bcat, b, c.g, c.I * TS + c.r, c.J * TS + c.c0, x, x);
+  if (!c.diag) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) x[k] = -up.v[c.c0 + k][c.r];
+    put_split4(Acat, Bcat, b, c.g, c.J * TS + c.r, c.I * TS + c.c0, x, x);
   }
 }
 
@@ -126,24 +155,27 @@ split_sh_kernel(const BlockRuns r, const float* __restrict__ S, int b,
                 __nv_bfloat16* __restrict__ Acat, __nv_bfloat16* __restrict__ Bcat) {
   __shared__ Tile up;
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
-  int local;
-  const int run = run_of(r, c.g, local);
-  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
+  pair_ctx(b, c);
+  int run, local;
+  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
   const float* Sg = S + (int64_t)c.g * c.bb;
+  float x[4], y[4];
+  {
+    const int i = c.I * TS + c.r, j = c.J * TS + c.c0;
+    const float4 s4 = ld4(Sg + (int64_t)i * b + j);
+    x[0] = s4.x; x[1] = s4.y; x[2] = s4.z; x[3] = s4.w;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    {
-      const int i = c.I * TS + r, j = c.J * TS + c.tx;
-      const float s = Sg[(int64_t)i * b + j];
-      put_split(Acat, Bcat, b, c.g, i, j, s, ((i == j) ? 2.f : 0.f) + 2.f * up.v[r][c.tx] + s);
-    }
-    if (!c.diag) {
-      const int i = c.J * TS + r, j = c.I * TS + c.tx;
-      const float s = Sg[(int64_t)i * b + j];
-      put_split(Acat, Bcat, b, c.g, i, j, s, -2.f * up.v[c.tx][r] + s);
-    }
+    for (int k = 0; k < 4; ++k)
+      y[k] = ((c.diag && c.r == c.c0 + k) ? 2.f : 0.f) + 2.f * up.v[c.r][c.c0 + k] + x[k];
+    put_split4(Acat, Bcat, b, c.g, i, j, x, y);
+  }
+  if (!c.diag) {
+    const int i = c.J * TS + c.r, j = c.I * TS + c.c0;
+    const float4 s4 = ld4(Sg + (int64_t)i * b + j);
+    x[0] = s4.x; x[1] = s4.y; x[2] = s4.z; x[3] = s4.w;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) y[k] = -2.f * up.v[c.c0 + k][c.r] + x[k];
+    put_split4(Acat, Bcat, b, c.g, i, j, x, y);
   }
 }
 
@@ -152,32 +184,28 @@ __global__ void __launch_bounds__(kTileThreads)
 cnp_finish_kernel(const BlockRuns r, const float* __restrict__ Pall, int b) {
   __shared__ Tile up;
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
-  int local;
-  const int run = run_of(r, c.g, local);
-  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
+  pair_ctx(b, c);
+  int run, local;
+  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
   // P is indexed by the launch-wide block, the outputs by the block within its run
-  const float* P = Pall + ((int64_t)c.g - local) * c.bb;
-  float* g = r.g[run];
-  __nv_bfloat16* g_lp = r.g_lp[run];
-  const int64_t base = (int64_t)local * c.bb;
+  const float* P = Pall + (int64_t)c.g * c.bb;
+  float* g = r.g[run] ? r.g[run] + (int64_t)local * c.bb : nullptr;
+  __nv_bfloat16* g_lp = r.g_lp[run] ? r.g_lp[run] + (int64_t)local * c.bb : nullptr;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    {
-      const int i = c.I * TS + r, j = c.J * TS + c.tx;
-      const int64_t e = base + (int64_t)i * b + j;
-      const float v = ((i == j) ? 1.f : 0.f) + 2.f * up.v[r][c.tx] + P[e];
-      if (g) g[e] = v;
-      if (g_lp) g_lp[e] = __float2bfloat16_rn(v);
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && c.diag) break;
+    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
+    const int64_t off = (int64_t)i * b + j;
+    const float4 p4 = ld4(P + off);
+    const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float qv = h ? -up.v[c.c0 + k][c.r] : up.v[c.r][c.c0 + k];
+      v[k] = ((!h && c.diag && c.r == c.c0 + k) ? 1.f : 0.f) + 2.f * qv + pv[k];
     }
-    if (!c.diag) {
-      const int i = c.J * TS + r, j = c.I * TS + c.tx;
-      const int64_t e = base + (int64_t)i * b + j;
-      const float v = -2.f * up.v[c.tx][r] + P[e];
-      if (g) g[e] = v;
-      if (g_lp) g_lp[e] = __float2bfloat16_rn(v);
-    }
+    if (g) st4(g + off, v[0], v[1], v[2], v[3]);
+    if (g_lp) st4h(g_lp + off, v);
   }
 }
 
@@ -187,10 +215,9 @@ dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
                __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ dGh) {
   __shared__ Tile up;
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
-  int local;
-  const int run = run_of(r, c.g, local);
-  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
+  pair_ctx(b, c);
+  int run, local;
+  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
   const int64_t base = (int64_t)c.g * c.bb;
   // this block's partial sums within its run, [splits][nb_run][b][b]
   const float* pr = r.parts[run] + (int64_t)local * c.bb;
@@ -198,19 +225,21 @@ dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
   const int64_t split_stride = (int64_t)r.nb[run] * c.bb;
   const bool in_place = splits == 1 && pr == dG + base;  // written straight into dG
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (h == 1 && c.diag) break;
-      const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
-      const int64_t off = (int64_t)i * b + j, e = base + off;
-      float v = 0.f;
-      for (int sp = 0; sp < splits; ++sp) v += pr[sp * split_stride + off];
-      if (!in_place) dG[e] = v;
-      dGh[e] = __float2bfloat16_rn(v);
-      Qh[e] = __float2bfloat16_rn(h ? -up.v[c.tx][r] : up.v[r][c.tx]);
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && c.diag) break;
+    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
+    const int64_t off = (int64_t)i * b + j;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sp = 0; sp < splits; ++sp) {
+      const float4 t = ld4(pr + sp * split_stride + off);
+      v[0] += t.x; v[1] += t.y; v[2] += t.z; v[3] += t.w;
     }
+    if (!in_place) st4(dG + base + off, v[0], v[1], v[2], v[3]);
+    st4h(dGh + base + off, v);
+    float qv[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) qv[k] = h ? -up.v[c.c0 + k][c.r] : up.v[c.r][c.c0 + k];
+    st4h(Qh + base + off, qv);
   }
 }
 
@@ -220,24 +249,23 @@ dq_prep2_kernel(const BlockRuns r, const float* __restrict__ S, int b,
                 __nv_bfloat16* __restrict__ Sh, __nv_bfloat16* __restrict__ SmQ) {
   __shared__ Tile up;
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
-  int local;
-  const int run = run_of(r, c.g, local);
-  load_q_tile(up, r.q[run] + (int64_t)local * (b * (b - 1) / 2), b, c);
+  pair_ctx(b, c);
+  int run, local;
+  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
   const int64_t base = (int64_t)c.g * c.bb;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && c.diag) break;
+    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
+    const int64_t off = base + (int64_t)i * b + j;
+    const float4 s4 = ld4(S + off);
+    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+    float m[4];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      if (h == 1 && c.diag) break;
-      const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
-      const int64_t e = base + (int64_t)i * b + j;
-      const float s = S[e];
-      const float qv = h ? -up.v[c.tx][r] : up.v[r][c.tx];
-      Sh[e] = __float2bfloat16_rn(s);
-      SmQ[e] = __float2bfloat16_rn(s - 2.f * qv);
-    }
+    for (int k = 0; k < 4; ++k)
+      m[k] = sv[k] - 2.f * (h ? -up.v[c.c0 + k][c.r] : up.v[c.r][c.c0 + k]);
+    st4h(Sh + off, sv);
+    st4h(SmQ + off, m);
   }
 }
 
@@ -248,32 +276,37 @@ dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
               float* __restrict__ V) {
   __shared__ Tile sa, sb;  // Sbar tiles (I, J) and (J, I)
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
+  pair_ctx(b, c);
   const int64_t base = (int64_t)c.g * c.bb;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = (h ? c.J : c.I) * TS + r, j = (h ? c.I : c.J) * TS + c.tx;
-      const int64_t e = base + (int64_t)i * b + j;
-      const float d = dG[e], hb = Hb[e];
-      (h ? sb : sa).v[r][c.tx] = 2.f * d + T1[e] + hb;
-      if (h == 0 || !c.diag) V[e] = 2.f * d + 2.f * hb;
-    }
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && c.diag) break;
+    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
+    const int64_t off = base + (int64_t)i * b + j;
+    const float4 d = ld4(dG + off), t = ld4(T1 + off), hb = ld4(Hb + off);
+    Tile& dst = h ? sb : sa;
+    dst.v[c.r][c.c0 + 0] = 2.f * d.x + t.x + hb.x;
+    dst.v[c.r][c.c0 + 1] = 2.f * d.y + t.y + hb.y;
+    dst.v[c.r][c.c0 + 2] = 2.f * d.z + t.z + hb.z;
+    dst.v[c.r][c.c0 + 3] = 2.f * d.w + t.w + hb.w;
+    st4(V + off, 2.f * d.x + 2.f * hb.x, 2.f * d.y + 2.f * hb.y, 2.f * d.z + 2.f * hb.z,
+        2.f * d.w + 2.f * hb.w);
   }
   __syncthreads();
+  const Tile& tb = c.diag ? sa : sb;
+  {
+    const int i = c.I * TS + c.r, j = c.J * TS + c.c0;
+    float z[4];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    {
-      const int i = c.I * TS + r, j = c.J * TS + c.tx;
-      Zh[base + (int64_t)i * b + j] = __float2bfloat16_rn(sa.v[r][c.tx] + sb.v[c.tx][r]);
-    }
-    if (!c.diag) {
-      const int i = c.J * TS + r, j = c.I * TS + c.tx;
-      Zh[base + (int64_t)i * b + j] = __float2bfloat16_rn(sb.v[r][c.tx] + sa.v[c.tx][r]);
-    }
+    for (int k = 0; k < 4; ++k) z[k] = sa.v[c.r][c.c0 + k] + tb.v[c.c0 + k][c.r];
+    st4h(Zh + base + (int64_t)i * b + j, z);
+  }
+  if (!c.diag) {
+    const int i = c.J * TS + c.r, j = c.I * TS + c.c0;
+    float z[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) z[k] = sb.v[c.r][c.c0 + k] + sa.v[c.c0 + k][c.r];
+    st4h(Zh + base + (int64_t)i * b + j, z);
   }
 }
 
@@ -283,33 +316,33 @@ dq_pack_kernel(const BlockRuns r, const float* __restrict__ V, const float* __re
                int b) {
   __shared__ Tile ua, ub;  // U tiles (I, J) and (J, I)
   PairCtx c;
-  if (!pair_ctx(b, c)) return;
+  pair_ctx(b, c);
   const int64_t base = (int64_t)c.g * c.bb;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    {
-      const int64_t e = base + (int64_t)(c.I * TS + r) * b + c.J * TS + c.tx;
-      ua.v[r][c.tx] = V[e] - ZQ[e];
-    }
-    {
-      const int64_t e = base + (int64_t)(c.J * TS + r) * b + c.I * TS + c.tx;
-      ub.v[r][c.tx] = V[e] - ZQ[e];
-    }
+  for (int h = 0; h < 2; ++h) {
+    if (h == 1 && c.diag) break;
+    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
+    const int64_t off = base + (int64_t)i * b + j;
+    const float4 v = ld4(V + off), z = ld4(ZQ + off);
+    Tile& dst = h ? ub : ua;
+    dst.v[c.r][c.c0 + 0] = v.x - z.x;
+    dst.v[c.r][c.c0 + 1] = v.y - z.y;
+    dst.v[c.r][c.c0 + 2] = v.z - z.z;
+    dst.v[c.r][c.c0 + 3] = v.w - z.w;
   }
   __syncthreads();
+  const Tile& tb = c.diag ? ua : ub;
   int local;
   const int run = run_of(r, c.g, local);
   float* dqb = r.dq[run] + (int64_t)local * (b * (b - 1) / 2);
+  const int i = c.I * TS + c.r;
+  const int64_t rowbase = (int64_t)i * b - (int64_t)i * (i + 1) / 2 - i - 1;
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    const int r = c.ty + 8 * k;
-    const int i = c.I * TS + r, j = c.J * TS + c.tx;
-    if (i < j) dqb[i * b - i * (i + 1) / 2 + (j - i - 1)] = ua.v[r][c.tx] - ub.v[c.tx][r];
+    const int j = c.J * TS + c.c0 + k;
+    if (i < j) dqb[rowbase + j] = ua.v[c.r][c.c0 + k] - tb.v[c.c0 + k][c.r];
   }
 }
-
-dim3 pair_grid(int64_t nb, int64_t b) { return dim3((unsigned)((b / TS) * (b / TS)), (unsigned)nb); }
 
 // C_g = X_g Y_g for nb blocks of b x b (fp32 out), X K-major [nb*b][kx] (kx = K), Y MN-major
 // [nb*K][b]. K = b (single pass) or 3b (split operands).
