@@ -71,8 +71,7 @@ cudaError_t gemm_blockwise(DT t, const void* A, const void* G, void* C, int64_t 
     else { g.b_mn = true; g.b_gn = 0; g.b_gk = b; }                // B(k, j) = G[k][j]
     g.C = C; g.ldc = width; g.c_gs = b;
     g.name = transpose_g ? "umma_blockwise_T" : "umma_blockwise";
-    // K = b is short: single-CTA 128 x 256 tiles measured faster than CTA pairs here
-    if (umma::supported(g)) return umma::gemm(g, s);
+    if (umma::supported(g)) return run(g, s);
   }
   SimtGemm g{};
   g.M = rows; g.N = b; g.K = b; g.batch = width / b;
