@@ -242,50 +242,64 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     wl = W.WORKLOADS[args.workload]
-    lin = wl.linears[0]
-    m, n, b = lin.m, lin.n, wl.b
+    b = wl.b
     T = args.tokens or wl.tokens
     dt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
     esz = 2 if dt == torch.bfloat16 else 4
+    nlin = len(wl.linears) if args.all_linears else 1
 
-    # ---- inputs: same layer on every rank, each rank its own tokens
-    p = W.layer_params(wl)
-    a = W.layer_acts(wl, tokens=T, seed=W.WORKLOAD_SEED[wl.key] * 1000 + rank)
-    w0 = torch.from_numpy(p["W0"]).to(dt).to(dev)
-    pr = torch.from_numpy(p["perm_r"]).to(dev)
-    pp = torch.from_numpy(p["perm_p"]).to(dev)
-    q_r = torch.from_numpy(p["q_r"]).to(dev)
-    q_p = torch.from_numpy(p["q_p"]).to(dev)
-    x_host = torch.from_numpy(a["X"]).to(dt).pin_memory()
-    dy_host = torch.from_numpy(a["dY"]).to(dt).pin_memory()
-    del a
-    x = x_host.to(dev)
-    dy = dy_host.to(dev)
-    w0m = torch.empty_like(w0)
-    poetx.merge_permutations(w0, pr, pp, w0m)
-    del w0
-    layer = poetx.PoetxLinear(w0m, pr, pp, q_r, q_p, b)
-    y = torch.empty(T, n, dtype=dt, device=dev)
-    bsave = torch.empty(T, n, dtype=dt, device=dev)
-    dx = torch.empty(T, m, dtype=dt, device=dev)
-    dq_r = torch.empty_like(q_r)
-    dq_p = torch.empty_like(q_p)
-    ws = torch.empty(max(poetx.fwd_workspace_bytes(layer, T), poetx.bwd_workspace_bytes(layer, T),
-                         poetx.layer_cnp_workspace_bytes(layer)),
+    # ---- every linear of the workload (the same layers on every rank, each rank its own tokens)
+    layers = []
+    for li in range(nlin):
+        lin = wl.linears[li]
+        p = W.layer_params(wl, li)
+        a = W.layer_acts(wl, li, tokens=T, seed=W.WORKLOAD_SEED[wl.key] * 1000 + rank)
+        w0 = torch.from_numpy(p["W0"]).to(dt).to(dev)
+        pr = torch.from_numpy(p["perm_r"]).to(dev)
+        pp = torch.from_numpy(p["perm_p"]).to(dev)
+        w0m = torch.empty_like(w0)
+        poetx.merge_permutations(w0, pr, pp, w0m)
+        del w0
+        L = poetx.PoetxLinear(w0m, pr, pp, torch.from_numpy(p["q_r"]).to(dev),
+                              torch.from_numpy(p["q_p"]).to(dev), b)
+        d = {"lin": lin, "layer": L,
+             "x_host": torch.from_numpy(a["X"]).to(dt).pin_memory(),
+             "dy_host": torch.from_numpy(a["dY"]).to(dt).pin_memory()}
+        del a
+        d["x"] = d["x_host"].to(dev)
+        d["dy"] = d["dy_host"].to(dev)
+        d["y"] = torch.empty(T, lin.n, dtype=dt, device=dev)
+        d["bsave"] = torch.empty(T, lin.n, dtype=dt, device=dev)
+        d["dx"] = torch.empty(T, lin.m, dtype=dt, device=dev)
+        d["dq_r"] = torch.empty_like(L.q_r)
+        d["dq_p"] = torch.empty_like(L.q_p)
+        layers.append(d)
+        poetx.layer_cnp_build(L)
+    ws = torch.empty(max(max(poetx.fwd_workspace_bytes(d["layer"], T),
+                             poetx.bwd_workspace_bytes(d["layer"], T),
+                             poetx.layer_cnp_workspace_bytes(d["layer"])) for d in layers),
                      dtype=torch.uint8, device=dev)
-    flat_dq = torch.empty(dq_r.numel() + dq_p.numel(), device=dev) if world > 1 else None
+    ndq = sum(d["dq_r"].numel() + d["dq_p"].numel() for d in layers)
+    flat_dq = torch.empty(ndq, device=dev) if world > 1 else None
     stream = torch.cuda.current_stream(dev)
-    flush = None
-    if (x.numel() + dy.numel()) * esz <= L2_BYTES:
-        flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    in_bytes = sum((d["x"].numel() + d["dy"].numel()) * esz for d in layers)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
 
-    def step(xin, dyin):
-        poetx.layer_cnp_build(layer, ws)
-        poetx.linear_fwd(layer, xin, y, bsave, ws)
-        poetx.linear_bwd(layer, xin, dyin, bsave, dx, dq_r, dq_p, ws)
+    def step(xs=None, dys=None):
+        for i, d in enumerate(layers):
+            L = d["layer"]
+            xin = d["x"] if xs is None else xs[i]
+            dyin = d["dy"] if dys is None else dys[i]
+            if wl.cnp_in_step:
+                poetx.layer_cnp_build(L, ws)
+            poetx.linear_fwd(L, xin, d["y"], d["bsave"], ws)
+            poetx.linear_bwd(L, xin, dyin, d["bsave"], d["dx"], d["dq_r"], d["dq_p"], ws)
         if world > 1:
-            flat_dq[:dq_r.numel()].copy_(dq_r.view(-1))
-            flat_dq[dq_r.numel():].copy_(dq_p.view(-1))
+            o = 0
+            for d in layers:
+                for t in (d["dq_r"], d["dq_p"]):
+                    flat_dq[o:o + t.numel()].copy_(t.view(-1))
+                    o += t.numel()
             sum_over_ranks_(flat_dq)
 
     def barrier():
@@ -293,7 +307,7 @@ def run_ours(args):
             dist.barrier(device_ids=[local])
 
     for _ in range(args.warmup):
-        step(x, dy)
+        step()
     torch.cuda.synchronize()
     poetx.device_status()
 
@@ -310,91 +324,114 @@ def run_ours(args):
         if flush is not None:
             flush.zero_()
         ev[i][0].record(stream)
-        step(x, dy)
+        step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
     poetx.trace_enable(False)
     trace = poetx.trace_read()
-    step_ms = [s.elapsed_time(e) for s, e in ev]
-    total_ms = max_over_ranks(sum(step_ms), dev)
-    ms_per_step = total_ms / args.steps
-    value = T * world * args.steps / (total_ms / 1e3)
+    step_ms_local = sum(s.elapsed_time(e) for s, e in ev) / args.steps
 
-    # ---- dominant kernel: the two W0' GEMMs
-    w0_launches = [ms for name, ms in trace if name in ("umma_dense_W0", "umma_dense_W0T")]
+    # ---- merge-then-reinitialize, when the workload's schedule has it (amortised per step)
+    merge_ms = 0.0
+    if wl.merge_every:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for d in layers:
+            poetx.merge_reinit(d["layer"], 0x5EED + rank)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        merge_ms = e0.elapsed_time(e1)
+        for d in layers:   # restore a non-trivial q for any later use
+            poetx.layer_cnp_build(d["layer"])
+    step_ms_local += merge_ms / max(wl.merge_every, 1) if wl.merge_every else 0.0
+    ms_per_step = max_over_ranks(step_ms_local, dev)
+    value = T * world / (ms_per_step / 1e3)
+
+    # ---- dominant kernel: the W0' GEMMs of all linears
+    w0_ms = [ms for name, ms in trace if name in ("umma_dense_W0", "umma_dense_W0T")]
     launches = len(trace)
     peaks, peak_src = measured_peaks()
     roofline = None
-    if w0_launches:
-        avg_ms = statistics.mean(w0_launches)
-        flops = 2.0 * T * m * n
-        achieved = flops / (avg_ms / 1e3) / 1e12
+    if w0_ms:
+        flops = sum(2.0 * 2 * T * d["lin"].m * d["lin"].n for d in layers) * args.steps
+        total_ms = sum(w0_ms)
+        achieved = flops / (total_ms / 1e3) / 1e12
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
                     "kernel": "umma_dense_W0 / umma_dense_W0T (B = A' W0', dA' = dB W0'^T)",
                     "peak_source": f"{peak_src} bf16_tflops_sustained",
                     "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
-                    "avg_launch_ms": avg_ms, "launches": len(w0_launches)}
+                    "avg_launch_ms": total_ms / len(w0_ms), "launches": len(w0_ms)}
         tr = os.path.join(ROOT, "profiles", "traffic.txt")
-        if os.path.exists(tr):
+        if os.path.exists(tr) and nlin == 1:
             for ln in open(tr):
                 parts = ln.split()
                 if len(parts) >= 3 and parts[0] == "umma_dense" and parts[1] == str(T):
                     roofline["traffic"] = float(parts[2])
-    F = layer_flops(T, m, n, b)
-    Bb = layer_bytes(T, m, n, b, esz)
+    F = sum(layer_flops(T, d["lin"].m, d["lin"].n, b, wl.cnp_in_step) for d in layers)
+    Bb = sum(layer_bytes(T, d["lin"].m, d["lin"].n, b, esz) for d in layers)
     t_roof = max(F / (peaks["bf16_tflops"] * 1e12), Bb / (peaks["hbm_gbs"] * 1e9))
     per_kernel = {}
     for name, ms in trace:
         per_kernel[name] = per_kernel.get(name, 0.0) + ms
 
     # ---- end to end through the API: pinned host inputs in, dq out, every step
-    dq_host = torch.empty(dq_r.numel() + dq_p.numel(), dtype=torch.float32).pin_memory()
-    x_dev2 = torch.empty_like(x)
-    dy_dev2 = torch.empty_like(dy)
+    dq_host = torch.empty(ndq, dtype=torch.float32).pin_memory()
+    xs = [torch.empty_like(d["x"]) for d in layers]
+    dys = [torch.empty_like(d["dy"]) for d in layers]
     e2e_steps = max(2, min(args.steps, 5))
-    for _ in range(1):
-        x_dev2.copy_(x_host, non_blocking=True)
-        dy_dev2.copy_(dy_host, non_blocking=True)
-        step(x_dev2, dy_dev2)
+
+    def e2e_step():
+        for i, d in enumerate(layers):
+            xs[i].copy_(d["x_host"], non_blocking=True)
+            dys[i].copy_(d["dy_host"], non_blocking=True)
+        step(xs, dys)
+        o = 0
+        for d in layers:
+            for t in (d["dq_r"], d["dq_p"]):
+                dq_host[o:o + t.numel()].copy_(t.view(-1), non_blocking=True)
+                o += t.numel()
+
+    e2e_step()
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(e2e_steps):
-        x_dev2.copy_(x_host, non_blocking=True)
-        dy_dev2.copy_(dy_host, non_blocking=True)
-        step(x_dev2, dy_dev2)
-        dq_host[:dq_r.numel()].copy_(dq_r.view(-1), non_blocking=True)
-        dq_host[dq_r.numel():].copy_(dq_p.view(-1), non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e = {"value": T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": (x.numel() + dy.numel()) * esz,
-           "d2h_bytes_per_step": dq_host.numel() * 4}
+           "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": ndq * 4}
 
-    line = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             cpu = cpu_baseline(wl, args.ref_tokens)
             cpu.pop("seconds", None)
+        shapes = [f"{d['lin'].name} {d['lin'].m}x{d['lin'].n}" for d in layers]
+        cfg = {"workload": wl.key, "linears": shapes, "b": b, "tokens_per_gpu": T,
+               "global_batch_tokens": T * world, "parallelism": f"dp{world}",
+               "step": ("cnp_build(R,P) + " if wl.cnp_in_step else "")
+               + "linear_fwd + linear_bwd(dx, dq) per linear"
+               + (" + NCCL all-reduce of dq" if world > 1 else ""),
+               "l2": (f"inputs larger than L2: X + dY = {in_bytes / 2**20:.0f} MiB per step"
+                      if flush is None else "L2 flushed (2x126 MiB write) between steps")}
+        if nlin == 1:
+            cfg.update({"m": layers[0]["lin"].m, "n": layers[0]["lin"].n})
+        if wl.merge_every:
+            cfg["merge_reinit"] = (f"every {wl.merge_every} steps: {merge_ms:.3f} ms for all "
+                                   f"linears, amortised into ms_per_step")
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if dt == torch.bfloat16 else "f32", "data": "synthetic",
-            "config": {"workload": wl.key, "m": m, "n": n, "b": b, "tokens_per_gpu": T,
-                       "global_batch_tokens": T * world, "parallelism": f"dp{world}",
-                       "step": "cnp_build(R,P) + linear_fwd + linear_bwd(dx, dq)"
-                               + (" + NCCL all-reduce of dq" if world > 1 else ""),
-                       "l2": ("inputs larger than L2: X + dY = "
-                              f"{(x.numel() + dy.numel()) * esz / 2**20:.0f} MiB per step")
-                       if flush is None else "L2 flushed (2x126 MiB write) between steps"},
+            "config": cfg,
             "tflops": F * world / (ms_per_step / 1e3) / 1e12,
             "step_roofline": {"t_roof_ms": t_roof * 1e3, "frac": t_roof * 1e3 / ms_per_step,
                               "flops": F, "bytes": Bb, "peaks": peak_src},
@@ -424,6 +461,8 @@ def main(argv=None):
     ap.add_argument("--ref-tokens", type=int, default=256,
                     help="tokens in the oracle's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--first-linear-only", dest="all_linears", action="store_false",
+                    help="time only the first linear of a multi-linear workload")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours" and not os.environ.get("POETX_BENCH_ALLOW_SHORT"):
         args.warmup = 3
