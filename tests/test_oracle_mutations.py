@@ -101,3 +101,50 @@ def test_pins_catch_flipped_packing_gradient(monkeypatch):
     _patch(monkeypatch, "grad_through_packing", lambda S: -orig(S))
     with pytest.raises(AssertionError):
         pins.test_dq_matches_central_finite_differences()
+
+
+# ---------------------------------------------------------------- 8-bit weight storage (POET-XQ)
+import oracle.quant as QM  # noqa: E402
+import tests.test_oracle_quant as qpins  # noqa: E402
+
+
+def _quant_variant(divisor=127.0, axis=0, rounder=np.rint):
+    def quantize(W0m):
+        w = np.asarray(W0m, dtype=np.float32)
+        amax = np.max(np.abs(w), axis=axis, keepdims=True)
+        scale = (amax / np.float32(divisor)).astype(np.float32)
+        safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+        q = np.clip(rounder((w / safe).astype(np.float32)), -127, 127)
+        q = np.where(scale > 0, q, 0.0).astype(np.int8)
+        return q, (scale.reshape(-1) if axis == 0 else scale.reshape(-1)[: w.shape[1]])
+    return quantize
+
+
+QUANT_MUTATIONS = {
+    "divide_by_128": _quant_variant(divisor=128.0),
+    "per_row_scale": _quant_variant(axis=1),
+    "truncate": _quant_variant(rounder=np.trunc),
+    "half_away_from_zero": _quant_variant(
+        rounder=lambda r: np.sign(r) * np.floor(np.abs(r) + np.float32(0.5))),
+}
+
+
+@pytest.mark.parametrize("name", sorted(QUANT_MUTATIONS))
+def test_quant_pins_catch_planted_mistake(monkeypatch, name):
+    monkeypatch.setattr(QM, "quantize_w0_int8", QUANT_MUTATIONS[name])
+    failed = 0
+    for check in (qpins.test_exact_lattice_round_trips, qpins.test_ties_round_half_to_even,
+                  qpins.test_uniform_rounding_error_bound_and_range,
+                  qpins.test_scales_are_per_column, qpins.test_codes_match_exact_rational_rounding):
+        try:
+            check()
+        except (AssertionError, ValueError, IndexError):
+            failed += 1
+    assert failed >= 1, name
+
+
+def test_quant_pins_catch_unrounded_dequantisation(monkeypatch):
+    monkeypatch.setattr(QM, "dequantize_w0_int8",
+                        lambda q, s: q.astype(np.float64) * np.asarray(s, np.float64)[None, :])
+    with pytest.raises(AssertionError):
+        qpins.test_dequantised_values_are_bf16_of_fp32_product()
