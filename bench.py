@@ -47,6 +47,29 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def kernel_source_tag() -> str:
+    """First 12 hex digits of the SHA-256 of the tensor-core GEMM source: DRAM traffic figures
+    taken with ncu are used only while the kernel is the one they were taken on."""
+    import hashlib
+    src = os.path.join(ROOT, "orthogonal_equivalence_build_b200", "csrc", "umma_gemm.cu")
+    return hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+
+
+def measured_traffic(names, T):
+    """Mean dram__bytes_read.sum + dram__bytes_write.sum per launch of the kernels `names` at T
+    tokens, from profiles/traffic.txt (lines "<kernel> <T> <bytes per launch> <source tag>"),
+    or None when there is no figure for this kernel source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    tag, vals = kernel_source_tag(), []
+    for ln in open(path):
+        parts = ln.split()
+        if (len(parts) == 4 and parts[0] in names and parts[1] == str(T) and parts[3] == tag):
+            vals.append(float(parts[2]))
+    return sum(vals) / len(vals) if vals else None
+
+
 def layer_flops(T, m, n, b, cnp=True):
     """Algorithmic FLOPs of one step: fwd 2T(mb+mn+nb), bwd dx 2T(mn+mb+nb), dG 2T(mb+nb),
     CNP 2 products per block (S = QQ and S(2I+2Q+S)), dq 4 products per block."""
@@ -57,14 +80,16 @@ def layer_flops(T, m, n, b, cnp=True):
     return f
 
 
-def layer_bytes(T, m, n, b, e=2):
+def layer_bytes(T, m, n, b, e=2, w_e=None):
     """Algorithmic HBM bytes of one step: boundary tensors plus the saved B.
     fwd reads X, W0', G and writes Y, B; bwd reads dY, X, B, W0', G and writes dX;
-    q, G, dq in fp32."""
+    q, G, dq in fp32.  w_e: bytes per W0' element (1 for 8-bit storage, plus its column
+    scales)."""
     gblk = (m // b + n // b) * b * b
     qn = (m // b + n // b) * b * (b - 1) // 2
-    fwd = e * (T * m + m * n + T * n + T * n) + e * gblk
-    bwd = e * (T * n + T * m + T * n + m * n + T * m) + e * gblk
+    w = (e if w_e is None else w_e) * m * n + (4 * n if w_e == 1 else 0)
+    fwd = e * (T * m + T * n + T * n) + w + e * gblk
+    bwd = e * (T * n + T * m + T * n + T * m) + w + e * gblk
     cnp = 4 * qn + 4 * gblk + 2 * gblk
     dq = 4 * qn * 2
     return fwd + bwd + cnp + dq
@@ -260,8 +285,14 @@ def run_ours(args):
         w0m = torch.empty_like(w0)
         poetx.merge_permutations(w0, pr, pp, w0m)
         del w0
+        scale = None
+        if args.xq:   # 8-bit W0' (int8 codes + fp32 column scales)
+            wq = torch.empty(w0m.shape, dtype=torch.int8, device=dev)
+            scale = torch.empty(w0m.shape[1], dtype=torch.float32, device=dev)
+            poetx.quantize_w0(w0m, wq, scale)
+            w0m = wq
         L = poetx.PoetxLinear(w0m, pr, pp, torch.from_numpy(p["q_r"]).to(dev),
-                              torch.from_numpy(p["q_p"]).to(dev), b)
+                              torch.from_numpy(p["q_p"]).to(dev), b, w0m_scale=scale)
         d = {"lin": lin, "layer": L,
              "x_host": torch.from_numpy(a["X"]).to(dt).pin_memory(),
              "dy_host": torch.from_numpy(a["dY"]).to(dt).pin_memory()}
@@ -350,7 +381,9 @@ def run_ours(args):
     value = T * world / (ms_per_step / 1e3)
 
     # ---- dominant kernel: the W0' GEMMs of all linears
-    w0_ms = [ms for name, ms in trace if name in ("umma_dense_W0", "umma_dense_W0T")]
+    w0_names = (("umma_dense_W0_i8", "umma_dense_W0T_i8") if args.xq
+                else ("umma_dense_W0", "umma_dense_W0T"))
+    w0_ms = [ms for name, ms in trace if name in w0_names]
     launches = len(trace)
     peaks, peak_src = measured_peaks()
     roofline = None
@@ -361,52 +394,70 @@ def run_ours(args):
         peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
-                    "kernel": "umma_dense_W0 / umma_dense_W0T (B = A' W0', dA' = dB W0'^T)",
+                    "kernel": f"{w0_names[0]} / {w0_names[1]} (B = A' W0', dA' = dB W0'^T)",
                     "peak_source": f"{peak_src} bf16_tflops_sustained",
                     "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
                     "avg_launch_ms": total_ms / len(w0_ms), "launches": len(w0_ms)}
-        tr = os.path.join(ROOT, "profiles", "traffic.txt")
-        if os.path.exists(tr) and nlin == 1:
-            for ln in open(tr):
-                parts = ln.split()
-                if len(parts) >= 3 and parts[0] == "umma_dense" and parts[1] == str(T):
-                    roofline["traffic"] = float(parts[2])
+        if nlin == 1:
+            roofline["traffic"] = measured_traffic(w0_names, T)
     F = sum(layer_flops(T, d["lin"].m, d["lin"].n, b, wl.cnp_in_step) for d in layers)
-    Bb = sum(layer_bytes(T, d["lin"].m, d["lin"].n, b, esz) for d in layers)
+    Bb = sum(layer_bytes(T, d["lin"].m, d["lin"].n, b, esz, 1 if args.xq else None)
+             for d in layers)
     t_roof = max(F / (peaks["bf16_tflops"] * 1e12), Bb / (peaks["hbm_gbs"] * 1e9))
     per_kernel = {}
     for name, ms in trace:
         per_kernel[name] = per_kernel.get(name, 0.0) + ms
 
-    # ---- end to end through the API: pinned host inputs in, dq out, every step
+    # ---- end to end through the API: pinned host inputs in, dq out, every step. Two input
+    # buffers: the upload of step i+1's X and dY (copy stream) overlaps step i's kernels; a step
+    # starts when its own inputs have landed, an upload starts when the step that last read its
+    # buffer has finished.
     dq_host = torch.empty(ndq, dtype=torch.float32).pin_memory()
-    xs = [torch.empty_like(d["x"]) for d in layers]
-    dys = [torch.empty_like(d["dy"]) for d in layers]
-    e2e_steps = max(2, min(args.steps, 5))
+    bufs = [([torch.empty_like(d["x"]) for d in layers], [torch.empty_like(d["dy"]) for d in layers])
+            for _ in range(2)]
+    copy_stream = torch.cuda.Stream(dev)
+    copied = [torch.cuda.Event() for _ in range(2)]
+    consumed = [torch.cuda.Event() for _ in range(2)]
+    e2e_steps = max(3, min(args.steps, 6))
 
-    def e2e_step():
-        for i, d in enumerate(layers):
-            xs[i].copy_(d["x_host"], non_blocking=True)
-            dys[i].copy_(d["dy_host"], non_blocking=True)
-        step(xs, dys)
+    def upload(k):
+        copy_stream.wait_event(consumed[k])
+        with torch.cuda.stream(copy_stream):
+            for i, d in enumerate(layers):
+                bufs[k][0][i].copy_(d["x_host"], non_blocking=True)
+                bufs[k][1][i].copy_(d["dy_host"], non_blocking=True)
+        copied[k].record(copy_stream)
+
+    def run_step(k):
+        stream.wait_event(copied[k])
+        step(bufs[k][0], bufs[k][1])
+        consumed[k].record(stream)
         o = 0
         for d in layers:
             for t in (d["dq_r"], d["dq_p"]):
                 dq_host[o:o + t.numel()].copy_(t.view(-1), non_blocking=True)
                 o += t.numel()
 
-    e2e_step()
+    def e2e_run(n):
+        copy_stream.wait_stream(stream)
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload((i + 1) % 2)
+            run_step(i % 2)
+
+    e2e_run(2)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    e2e_run(e2e_steps)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     e2e = {"value": T * world * e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
-           "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": ndq * 4}
+           "h2d_bytes_per_step": in_bytes, "d2h_bytes_per_step": ndq * 4,
+           "pipeline": "inputs of step i+1 upload on a copy stream during step i"}
 
     if rank == 0:
         cpu = None
@@ -423,6 +474,9 @@ def run_ours(args):
                       if flush is None else "L2 flushed (2x126 MiB write) between steps")}
         if nlin == 1:
             cfg.update({"m": layers[0]["lin"].m, "n": layers[0]["lin"].n})
+        if args.xq:
+            cfg["w0m_storage"] = ("int8 codes + fp32 column scales, dequantised to bf16 in the "
+                                  "W0' GEMMs' shared-memory operand stages")
         if wl.merge_every:
             cfg["merge_reinit"] = (f"every {wl.merge_every} steps: {merge_ms:.3f} ms for all "
                                    f"linears, amortised into ms_per_step")
@@ -463,6 +517,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--first-linear-only", dest="all_linears", action="store_false",
                     help="time only the first linear of a multi-linear workload")
+    ap.add_argument("--xq", action="store_true",
+                    help="store W0' in 8 bits (int8 + column scales) and time that layer")
     args = ap.parse_args(argv)
     if args.warmup < 3 and args.impl == "ours" and not os.environ.get("POETX_BENCH_ALLOW_SHORT"):
         args.warmup = 3

@@ -59,14 +59,27 @@ typedef enum {
 
 typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
 
+/* poetx_layer.flags bit: W0' is stored in 8 bits ("POET-XQ": only the low-precision weights are
+ * kept and dequantised on demand — "[Project POET-X] Scaling Orthogonal Equivalence ..."
+ * §Quantized Training (POET-XQ); "POET-X: Memory-efficient LLM Training ..." (gist.science)
+ * §Resumo técnico 2 Metodologia). The pages give no format; this library uses symmetric int8
+ * codes with one fp32 scale per column of W0' (poetx_quantize_w0). w0m then points to int8
+ * [m, n] codes, w0m_scale to fp32 [n] scales, and the layer computes exactly as the BF16 layer
+ * whose W0' is bf16(code * scale) (poetx_dequantize_w0): the W0' products dequantise each int8
+ * tile in shared memory inside the tensor-core kernel (T >= 256 and n, m multiples of 256;
+ * other shapes dequantise into the workspace first). Requires dtype == POETX_BF16 and m, n
+ * multiples of 16. */
+#define POETX_LAYER_W0M_I8 1
+
 /* One POET-X linear. Every pointer is a device pointer owned by the caller. */
 typedef struct {
   int64_t m;       /* in-features: rows of W0 */
   int64_t n;       /* out-features: columns of W0 */
   int64_t b;       /* block size; must divide m and n */
   int32_t dtype;   /* poetx_dtype of w0m, activations, saved_b, gradients and g_*_lp */
-  int32_t flags;   /* reserved, must be 0 */
-  void* w0m;       /* [m, n] merged weight W0' (see poetx_merge_permutations) */
+  int32_t flags;   /* 0, or POETX_LAYER_W0M_I8 */
+  void* w0m;       /* [m, n] merged weight W0' (see poetx_merge_permutations); int8 codes
+                      when flags has POETX_LAYER_W0M_I8 */
   int32_t* perm_r; /* [m] permutation of R */
   int32_t* perm_p; /* [n] permutation of P */
   float* q_r;      /* [m/b, b(b-1)/2] packed skew parameters of R */
@@ -75,6 +88,7 @@ typedef struct {
   float* g_p;      /* [n/b, b, b] fp32 CNP blocks of P */
   void* g_r_lp;    /* [m/b, b, b] bf16 copy of g_r; required when dtype == POETX_BF16 */
   void* g_p_lp;    /* [n/b, b, b] bf16 copy of g_p; required when dtype == POETX_BF16 */
+  float* w0m_scale; /* [n] fp32 column scales of the int8 W0' (POETX_LAYER_W0M_I8), else NULL */
 } poetx_layer;
 
 /* ---------------------------------------------------------------------------------------------
@@ -117,8 +131,8 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t
  *   Arguments, outputs and accuracy are those of poetx_cnp_build; any nblocks is accepted (the
  *   blocks are processed in chunks that fit the buffer).
  *   Limit: b must need at most POETX_CNP_NOALLOC_SCRATCH_BYTES of scratch for ONE block
- *   (20*b*b bytes when b is a multiple of 128, else 12*b*b): b <= 896 for multiples of 128,
- *   b <= 1024 otherwise; larger b returns POETX_ERR_SHAPE with a message.
+ *   (12*b*b bytes, in slices rounded up to 256 bytes): b <= 836; larger b returns
+ *   POETX_ERR_SHAPE with a message.
  *   The first call on each device looks up the buffer's device address (cudaGetSymbolAddress)
  *   with that device current; make that first call before any stream capture.
  *   All calls on a device share the one buffer and it keeps the last call's contents (nothing in
@@ -126,7 +140,7 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t
  *   work overlaps on the GPU (e.g. on two streams without ordering) race on the buffer: order
  *   them on one stream or with events.
  * ------------------------------------------------------------------------------------------- */
-#define POETX_CNP_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+#define POETX_CNP_NOALLOC_SCRATCH_BYTES (8u * 1024u * 1024u)
 poetx_status poetx_cnp_build_noalloc(const float* q, int64_t nblocks, int64_t b, float* g,
                                      void* g_lp, int32_t lp_dtype, void* stream);
 
@@ -183,6 +197,8 @@ poetx_status poetx_merge_permutations(const void* w0, const int32_t* perm_r,
  *   drawn from `seed`, W0' <- the new merge of W, q <- 0. In place on L->w0m, L->perm_r,
  *   L->perm_p, L->q_r, L->q_p. The G blocks are NOT reset: rebuild them with poetx_cnp_build
  *   (q = 0 gives G = I exactly). The layer function is preserved up to rounding of W0'.
+ *   For POETX_LAYER_W0M_I8 layers the new W0' is computed from the dequantised one and stored
+ *   again as int8 codes and column scales (poetx_quantize_w0), in L->w0m and L->w0m_scale.
  *   Permutation draw: key_l[i] = SplitMix64 output i of the stream started at
  *   SplitMix64 output l of `seed` (l = 0 for R, 1 for P); pi_l sorts indices by (key, index).
  *   workspace >= poetx_merge_reinit_workspace_bytes(L).
@@ -190,6 +206,21 @@ poetx_status poetx_merge_permutations(const void* w0, const int32_t* perm_r,
 size_t poetx_merge_reinit_workspace_bytes(const poetx_layer* L);
 poetx_status poetx_merge_reinit(poetx_layer* L, uint64_t seed, void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_quantize_w0 — 8-bit storage of a weight for POETX_LAYER_W0M_I8 layers:
+ *     scale[j] = max_i |w[i, j]| / 127,   wq[i, j] = round_half_even(w[i, j] / scale[j]),
+ *   both in IEEE fp32 (|wq| <= 127; an all-zero column gets scale 0 and codes 0).
+ *   w [m, n] F32 or BF16 (dtype), read only;  wq [m, n] int8 and scale [n] fp32 outputs.
+ *   Deterministic: the column maxima are order-independent.
+ *   Errors: INVALID_ARG, SHAPE (m or n < 0), DTYPE, ALIGN.
+ * poetx_dequantize_w0 — w [m, n] bf16 = bf16(wq[i, j] * scale[j]) (fp32 product, rounded to
+ *   nearest even): the exact operand the int8 layer's products use.
+ * ------------------------------------------------------------------------------------------- */
+poetx_status poetx_quantize_w0(const void* w, int64_t m, int64_t n, int32_t dtype, int8_t* wq,
+                               float* scale, void* stream);
+poetx_status poetx_dequantize_w0(const int8_t* wq, const float* scale, int64_t m, int64_t n,
+                                 void* w_bf16, void* stream);
 
 /* Draw the permutation that poetx_merge_reinit would use for (seed, lane) into perm [k]. */
 poetx_status poetx_resample_permutation(uint64_t seed, int32_t lane, int64_t k, int32_t* perm,

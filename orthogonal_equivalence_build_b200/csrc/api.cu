@@ -131,7 +131,16 @@ poetx_status check_layer(const poetx_layer* L, bool need_lp) {
   if (!L) return fail(POETX_ERR_INVALID_ARG, "layer is NULL");
   if (L->dtype != POETX_F32 && L->dtype != POETX_BF16)
     return fail(POETX_ERR_DTYPE, "unknown layer dtype %d", L->dtype);
-  if (L->flags != 0) return fail(POETX_ERR_INVALID_ARG, "layer flags must be 0");
+  if (L->flags != 0 && L->flags != POETX_LAYER_W0M_I8)
+    return fail(POETX_ERR_INVALID_ARG, "unknown layer flags %d", L->flags);
+  if (L->flags == POETX_LAYER_W0M_I8) {
+    if (L->dtype != POETX_BF16)
+      return fail(POETX_ERR_DTYPE, "an int8 W0' needs a BF16 layer");
+    if (!L->w0m_scale) return fail(POETX_ERR_INVALID_ARG, "int8 W0' without w0m_scale");
+    if (!aligned16(L->w0m_scale)) return fail(POETX_ERR_ALIGN, "w0m_scale not 16-byte aligned");
+    if (L->m % 16 || L->n % 16)
+      return fail(POETX_ERR_SHAPE, "an int8 W0' needs m and n multiples of 16");
+  }
   if (L->m <= 0 || L->n <= 0 || L->b < 2)
     return fail(POETX_ERR_SHAPE, "bad layer shape m=%lld n=%lld b=%lld", (long long)L->m,
                 (long long)L->n, (long long)L->b);
@@ -160,10 +169,13 @@ poetx_status check_ws(void* ws, size_t have, size_t need) {
   return POETX_OK;
 }
 
+size_t xq_deq_bytes(const poetx_layer* L, int64_t T, bool fwd_product, bool bwd_product);
+
 // ---- workspace layouts (each buffer 256-byte aligned)
 struct FwdWs {
   void *A, *A1, *B, *C;
   int32_t* inv;
+  void* Wd;   // dequantised W0' (int8 layers whose product shape is not fused)
 };
 size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
   Arena a(base, SIZE_MAX);
@@ -174,6 +186,8 @@ size_t fwd_layout(const poetx_layer* L, int64_t T, void* base, FwdWs* o) {
   w.C = a.take(T * L->n * e);
   w.B = a.take(T * L->n * e);  // used only when the caller does not keep B
   w.inv = static_cast<int32_t*>(a.take(L->n * 4));
+  const size_t wd = xq_deq_bytes(L, T, true, false);
+  w.Wd = wd ? a.take(wd) : nullptr;
   if (o) *o = w;
   return a.used;
 }
@@ -185,6 +199,7 @@ struct BwdWs {
   void* chain;
   void *part_r, *part_p;  // split-K partial sums of dG_R, dG_P
   int32_t* inv;
+  void* Wd;               // dequantised W0' (int8 layers whose product shapes are not fused)
 };
 size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   Arena a(base, SIZE_MAX);
@@ -202,6 +217,8 @@ size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   w.part_r = a.take(block_grad_ws_bytes(t, L->m, L->b, T));
   w.part_p = a.take(block_grad_ws_bytes(t, L->n, L->b, T));
   w.inv = static_cast<int32_t*>(a.take(L->m * 4));
+  const size_t wd = xq_deq_bytes(L, T, true, true);
+  w.Wd = wd ? a.take(wd) : nullptr;
   if (o) *o = w;
   return a.used;
 }
@@ -227,11 +244,31 @@ size_t merge_layout(const poetx_layer* L, void* base, MergeWs* o) {
 
 DT dt_of(int32_t d) { return d == POETX_BF16 ? DT::BF16 : DT::F32; }
 
+bool w0m_i8(const poetx_layer* L) { return L->flags == POETX_LAYER_W0M_I8; }
+
+// bf16 scratch for an explicit dequantisation of an int8 W0' when a product shape is not fused
+size_t xq_deq_bytes(const poetx_layer* L, int64_t T, bool fwd_product, bool bwd_product) {
+  if (!w0m_i8(L)) return 0;
+  const bool need = (fwd_product && !dense_i8_fused(T, L->n)) ||
+                    (bwd_product && !dense_i8_fused(T, L->m));
+  return need ? (size_t)(L->m * L->n) * 2 : 0;
+}
+
+// B = A W0' (trans = false, A [T, m]) or dA' = dB W0'^T (trans = true, dB [T, n])
+cudaError_t w0_product(const poetx_layer* L, const void* A, void* C, int64_t T, bool trans,
+                       void* deq_ws, cudaStream_t s) {
+  const int64_t N = trans ? L->m : L->n, K = trans ? L->n : L->m;
+  if (w0m_i8(L))
+    return gemm_dense_i8(A, static_cast<const int8_t*>(L->w0m), L->w0m_scale, C, T, N, K, trans,
+                         deq_ws, s);
+  return gemm_dense(dt_of(L->dtype), A, L->w0m, C, T, N, K, trans, s);
+}
+
 }  // namespace
 
 extern "C" {
 
-int32_t poetx_abi_version(void) { return 1; }
+int32_t poetx_abi_version(void) { return 2; }
 
 const char* poetx_status_string(int32_t st) {
   switch (st) {
@@ -371,7 +408,7 @@ poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, vo
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
   CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_fwd_gather_X"), "fwd gather");
   CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.A1, T, m, b, false, s), "fwd R blocks");
-  CHECK_CUDA(gemm_dense(t, w.A1, L->w0m, B, T, n, m, false, s), "fwd W0' GEMM");
+  CHECK_CUDA(w0_product(L, w.A1, B, T, false, w.Wd, s), "fwd W0' GEMM");
   CHECK_CUDA(gemm_blockwise(t, B, Gp, w.C, T, n, b, false, s), "fwd P blocks");
   CHECK_CUDA(scatter_cols(w.C, y, T, n, L->perm_p, e, w.inv, s, "perm_fwd_scatter_Y"), "fwd scatter");
   return POETX_OK;
@@ -410,7 +447,7 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
     CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_regather_X"),
                "bwd recompute gather");
     CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.dA, T, m, b, false, s), "bwd recompute R blocks");
-    CHECK_CUDA(gemm_dense(t, w.dA, L->w0m, w.B, T, n, m, false, s), "bwd recompute W0' GEMM");
+    CHECK_CUDA(w0_product(L, w.dA, w.B, T, false, w.Wd, s), "bwd recompute W0' GEMM");
     saved_b = w.B;
   }
   CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s, "perm_bwd_gather_dY"), "bwd gather dY");
@@ -420,7 +457,7 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   int sp_r = 1, sp_p = 1;
   if (dq_p)
     CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, dG_p, T, n, b, w.part_p, &sp_p, s), "bwd dG_P");
-  CHECK_CUDA(gemm_dense(t, w.dB, L->w0m, w.dA1, T, m, n, true, s), "bwd W0'^T GEMM");
+  CHECK_CUDA(w0_product(L, w.dB, w.dA1, T, true, w.Wd, s), "bwd W0'^T GEMM");
   if (dx) {
     CHECK_CUDA(gemm_blockwise(t, w.dA1, Gr, w.dA, T, m, b, true, s), "bwd R blocks");
     CHECK_CUDA(scatter_cols(w.dA, dx, T, m, L->perm_r, e, w.inv, s, "perm_bwd_scatter_dX"),
@@ -467,6 +504,36 @@ poetx_status poetx_merge_permutations(const void* w0, const int32_t* perm_r,
   if (st != POETX_OK) return st;
   CHECK_CUDA(gather_cols(w0, w0m, m, n, perm_r, perm_p, elem_size(dtype), as_stream(stream)),
              "merge_permutations");
+  return POETX_OK;
+}
+
+// ------------------------------------------------------------------ 8-bit W0'
+poetx_status poetx_quantize_w0(const void* w, int64_t m, int64_t n, int32_t dtype, int8_t* wq,
+                               float* scale, void* stream) {
+  if (dtype != POETX_F32 && dtype != POETX_BF16) return fail(POETX_ERR_DTYPE, "bad dtype");
+  if (m < 0 || n < 0) return fail(POETX_ERR_SHAPE, "negative size");
+  if (m == 0 || n == 0) return POETX_OK;
+  if (!w || !wq || !scale) return fail(POETX_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(w) || !aligned16(wq) || !aligned16(scale))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  poetx_status st = check_device();
+  if (st != POETX_OK) return st;
+  CHECK_CUDA(quantize_cols_i8(w, dt_of(dtype), m, n, wq, scale, as_stream(stream)), "quantize_w0");
+  return POETX_OK;
+}
+
+poetx_status poetx_dequantize_w0(const int8_t* wq, const float* scale, int64_t m, int64_t n,
+                                 void* w_bf16, void* stream) {
+  if (m < 0 || n < 0) return fail(POETX_ERR_SHAPE, "negative size");
+  if (m == 0 || n == 0) return POETX_OK;
+  if (!wq || !scale || !w_bf16) return fail(POETX_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(wq) || !aligned16(scale) || !aligned16(w_bf16))
+    return fail(POETX_ERR_ALIGN, "pointers must be 16-byte aligned");
+  poetx_status st = check_device();
+  if (st != POETX_OK) return st;
+  CHECK_CUDA(dequantize_cols_i8(wq, scale, m, n, static_cast<__nv_bfloat16*>(w_bf16),
+                                as_stream(stream)),
+             "dequantize_w0");
   return POETX_OK;
 }
 
@@ -522,16 +589,32 @@ poetx_status poetx_merge_reinit(poetx_layer* L, uint64_t seed, void* workspace, 
   const int64_t m = L->m, n = L->n, b = L->b;
   const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
-  // M = Diag(G_R) W0' Diag(G_P), block by block
-  CHECK_CUDA(gemm_blockwise(t, L->w0m, Gp, w.N1, m, n, b, false, s), "merge W0' G_P");
+  const bool i8 = w0m_i8(L);
+  // M = Diag(G_R) W0' Diag(G_P), block by block (an int8 W0' is dequantised into M's buffer
+  // first; that buffer is free again once W0' Diag(G_P) is formed)
+  const void* W0m = L->w0m;
+  if (i8) {
+    CHECK_CUDA(dequantize_cols_i8(static_cast<const int8_t*>(L->w0m), L->w0m_scale, m, n,
+                                  static_cast<__nv_bfloat16*>(w.M), s),
+               "merge dequantise W0'");
+    W0m = w.M;
+  }
+  CHECK_CUDA(gemm_blockwise(t, W0m, Gp, w.N1, m, n, b, false, s), "merge W0' G_P");
   CHECK_CUDA(gemm_blockwise_left(t, Gr, w.N1, w.M, m, n, b, s), "merge G_R (.)");
   // new permutations, composed index maps rho = perm_old^{-1} o perm_new
   CHECK_CUDA(resample_permutation(seed, 0, m, w.pr_new, s), "resample R");
   CHECK_CUDA(resample_permutation(seed, 1, n, w.pp_new, s), "resample P");
   CHECK_CUDA(compose_inverse(L->perm_r, w.pr_new, w.inv, w.rho_r, m, s), "compose R");
   CHECK_CUDA(compose_inverse(L->perm_p, w.pp_new, w.inv, w.rho_p, n, s), "compose P");
-  // W0'_new[i, j] = M[rho_r[i], rho_p[j]]
-  CHECK_CUDA(gather_cols(w.M, L->w0m, m, n, w.rho_r, w.rho_p, e, s), "merge regather");
+  // W0'_new[i, j] = M[rho_r[i], rho_p[j]]; int8 layers store it as codes and column scales
+  if (i8) {
+    CHECK_CUDA(gather_cols(w.M, w.N1, m, n, w.rho_r, w.rho_p, e, s), "merge regather");
+    CHECK_CUDA(quantize_cols_i8(w.N1, DT::BF16, m, n, static_cast<int8_t*>(L->w0m), L->w0m_scale,
+                                s),
+               "merge quantise W0'");
+  } else {
+    CHECK_CUDA(gather_cols(w.M, L->w0m, m, n, w.rho_r, w.rho_p, e, s), "merge regather");
+  }
   CHECK_CUDA(cudaMemcpyAsync(L->perm_r, w.pr_new, m * 4, cudaMemcpyDeviceToDevice, s), "perm_r");
   CHECK_CUDA(cudaMemcpyAsync(L->perm_p, w.pp_new, n * 4, cudaMemcpyDeviceToDevice, s), "perm_p");
   CHECK_CUDA(fill_zero_f32(L->q_r, m / b * (b * (b - 1) / 2), s), "zero q_r");

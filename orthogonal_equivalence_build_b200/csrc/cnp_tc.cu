@@ -4,15 +4,22 @@
 // as G = (I + 2Q) + S H with S = Q Q and H = 2I + 2Q + S: two b x b products per block, on the
 // bf16 tcgen05 kernel with fp32 accumulation. Each fp32 operand x is split into
 // x_hi = bf16(x) and x_lo = bf16(x - x_hi); x y is taken as x_hi y_hi + x_hi y_lo + x_lo y_hi,
-// i.e. ONE GEMM with the contraction tripled over concatenated operands
-//     [x_hi | x_hi | x_lo] . [y_hi ; y_lo ; y_hi],
-// which keeps about 16 significant bits per product (the dropped x_lo y_lo is ~2^-16 relative):
-// fp32-class G for the 1e-5 bar.
+// one accumulator over three K segments that read the hi and lo halves from their own buffers
+// (the dropped x_lo y_lo is ~2^-16 relative): fp32-class G for the 1e-5 bar.
+//   pass 1 (elementwise): q -> Q_hi, Q_lo
+//   product 1: S = Q Q; its epilogue writes S_hi, S_lo and H_hi, H_lo (H = 2I + 2Q + S)
+//   product 2: P = S H; its epilogue writes G = I + 2Q + P (fp32 and bf16)
+// Q in the epilogues is Q_hi + Q_lo (within |Q| 2^-17 of Q).
 //
 // Gradient, for bf16 layers (tolerance 1e-2): with Hbar = S dG, Sbar = dG (2I - 2Q + S) + Hbar,
-// Z = Sbar + Sbar^T, U = 2 dG + 2 Hbar - Z Q, dq_ij = U_ij - U_ji (i < j). The four products
-// S = QQ, S dG, dG (S - 2Q) and Z Q run single-pass bf16 with fp32 accumulation; the exact
-// 2 dG terms are added in fp32.
+// Z = Sbar + Sbar^T, U = 2 dG + 2 Hbar - Z Q, dq_ij = U_ij - U_ji (i < j). The products S = QQ,
+// S dG and dG (S - 2Q) (the last two in one launch) and Z Q run single-pass bf16 with fp32
+// accumulation; the exact 2 dG terms are added in fp32.
+//   pass 1: dG = sum of split partials, dG_h = bf16(dG), Q_h, Q_l
+//   product 1: S = Q_h Q_h; epilogue writes S_h = bf16(S), SmQ = bf16(S - 2Q)
+//   products 2, 3 (one launch over 2 nb groups): Hbar = S_h dG_h, T1 = dG_h SmQ
+//   pass 2: Z_h = bf16(Sbar + Sbar^T), V = 2 dG + 2 Hbar
+//   product 4: Z_h Q_h;  pass 3: U = V - Z Q, dq packed.
 #include "gemm.h"
 #include "umma_gemm.h"
 
@@ -103,116 +110,49 @@ __device__ __forceinline__ void split4(const float (&x)[4], float (&hi)[4], floa
   }
 }
 
-// Concatenated split operands of one block product X Y, four consecutive columns j .. j+3:
-//   Acat [nb*b][3b]: row (g, i) = [Xhi(i, :) | Xhi(i, :) | Xlo(i, :)]
-//   Bcat [nb*3b][b]: rows (g, k') = Yhi (k' < b), Ylo (b <= k' < 2b), Yhi (2b <= k')
-__device__ __forceinline__ void put_split4(__nv_bfloat16* __restrict__ Acat,
-                                           __nv_bfloat16* __restrict__ Bcat, int b, int g, int i,
-                                           int j, const float (&x)[4], const float (&y)[4]) {
-  float xh[4], xl[4], yh[4], yl[4];
-  split4(x, xh, xl);
-  split4(y, yh, yl);
-  __nv_bfloat16* arow = Acat + ((int64_t)g * b + i) * (3 * b) + j;
-  st4h(arow, xh);
-  st4h(arow + b, xh);
-  st4h(arow + 2 * b, xl);
-  const int64_t bb = (int64_t)b * b;
-  __nv_bfloat16* bp = Bcat + (int64_t)g * 3 * bb + (int64_t)i * b + j;
-  st4h(bp, yh);
-  st4h(bp + bb, yl);
-  st4h(bp + 2 * bb, yh);
-}
-
 __device__ __forceinline__ const float* run_q(const BlockRuns& r, int g, int b, int& run,
                                               int& local) {
   run = run_of(r, g, local);
   return r.q[run] + (int64_t)local * (b * (b - 1) / 2);
 }
 
-// CNP pass 1: X = Y = Q.
+// hi / lo parts of four values, stored at p_hi + off and p_lo + off
+__device__ __forceinline__ void put_hilo4(__nv_bfloat16* __restrict__ p_hi,
+                                          __nv_bfloat16* __restrict__ p_lo, int64_t off,
+                                          const float (&x)[4]) {
+  float h[4], l[4];
+  split4(x, h, l);
+  st4h(p_hi + off, h);
+  st4h(p_lo + off, l);
+}
+
+// CNP pass 1: Q_hi, Q_lo [nb][b][b] from the packed strict upper triangles.
 __global__ void __launch_bounds__(kTileThreads)
-split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Acat,
-               __nv_bfloat16* __restrict__ Bcat) {
+split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
+               __nv_bfloat16* __restrict__ Qlo) {
   __shared__ Tile up;
   PairCtx c;
   pair_ctx(b, c);
   int run, local;
   load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
+  const int64_t base = (int64_t)c.g * c.bb;
   float x[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) x[k] = up.v[c.r][c.c0 + k];
-  put_split4(Acat, Bcat, b, c.g, c.I * TS + c.r, c.J * TS + c.c0, x, x);
+  put_hilo4(Qhi, Qlo, base + (int64_t)(c.I * TS + c.r) * b + c.J * TS + c.c0, x);
   if (!c.diag) {
 #pragma unroll
     for (int k = 0; k < 4; ++k) x[k] = -up.v[c.c0 + k][c.r];
-    put_split4(Acat, Bcat, b, c.g, c.J * TS + c.r, c.I * TS + c.c0, x, x);
+    put_hilo4(Qhi, Qlo, base + (int64_t)(c.J * TS + c.r) * b + c.I * TS + c.c0, x);
   }
 }
 
-// CNP pass 2: X = S, Y = 2I + 2Q + S.
-__global__ void __launch_bounds__(kTileThreads)
-split_sh_kernel(const BlockRuns r, const float* __restrict__ S, int b,
-                __nv_bfloat16* __restrict__ Acat, __nv_bfloat16* __restrict__ Bcat) {
-  __shared__ Tile up;
-  PairCtx c;
-  pair_ctx(b, c);
-  int run, local;
-  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
-  const float* Sg = S + (int64_t)c.g * c.bb;
-  float x[4], y[4];
-  {
-    const int i = c.I * TS + c.r, j = c.J * TS + c.c0;
-    const float4 s4 = ld4(Sg + (int64_t)i * b + j);
-    x[0] = s4.x; x[1] = s4.y; x[2] = s4.z; x[3] = s4.w;
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      y[k] = ((c.diag && c.r == c.c0 + k) ? 2.f : 0.f) + 2.f * up.v[c.r][c.c0 + k] + x[k];
-    put_split4(Acat, Bcat, b, c.g, i, j, x, y);
-  }
-  if (!c.diag) {
-    const int i = c.J * TS + c.r, j = c.I * TS + c.c0;
-    const float4 s4 = ld4(Sg + (int64_t)i * b + j);
-    x[0] = s4.x; x[1] = s4.y; x[2] = s4.z; x[3] = s4.w;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) y[k] = -2.f * up.v[c.c0 + k][c.r] + x[k];
-    put_split4(Acat, Bcat, b, c.g, i, j, x, y);
-  }
-}
-
-// CNP finish: G = I + 2Q + P (fp32 and its bf16 copy).
-__global__ void __launch_bounds__(kTileThreads)
-cnp_finish_kernel(const BlockRuns r, const float* __restrict__ Pall, int b) {
-  __shared__ Tile up;
-  PairCtx c;
-  pair_ctx(b, c);
-  int run, local;
-  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
-  // P is indexed by the launch-wide block, the outputs by the block within its run
-  const float* P = Pall + (int64_t)c.g * c.bb;
-  float* g = r.g[run] ? r.g[run] + (int64_t)local * c.bb : nullptr;
-  __nv_bfloat16* g_lp = r.g_lp[run] ? r.g_lp[run] + (int64_t)local * c.bb : nullptr;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    if (h == 1 && c.diag) break;
-    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
-    const int64_t off = (int64_t)i * b + j;
-    const float4 p4 = ld4(P + off);
-    const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
-    float v[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float qv = h ? -up.v[c.c0 + k][c.r] : up.v[c.r][c.c0 + k];
-      v[k] = ((!h && c.diag && c.r == c.c0 + k) ? 1.f : 0.f) + 2.f * qv + pv[k];
-    }
-    if (g) st4(g + off, v[0], v[1], v[2], v[3]);
-    if (g_lp) st4h(g_lp + off, v);
-  }
-}
-
-// dq pass 1: Qh = bf16(Q); dG = sum of the split partials (fixed order), dGh = bf16(dG).
+// dq pass 1: Qh = bf16(Q), Ql = bf16(Q - Qh); dG = sum of the split partials (fixed order),
+// dGh = bf16(dG).
 __global__ void __launch_bounds__(kTileThreads)
 dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
-               __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ dGh) {
+               __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ Ql,
+               __nv_bfloat16* __restrict__ dGh) {
   __shared__ Tile up;
   PairCtx c;
   pair_ctx(b, c);
@@ -239,33 +179,7 @@ dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
     float qv[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) qv[k] = h ? -up.v[c.c0 + k][c.r] : up.v[c.r][c.c0 + k];
-    st4h(Qh + base + off, qv);
-  }
-}
-
-// dq pass 2: Sh = bf16(S), SmQ = bf16(S - 2Q).
-__global__ void __launch_bounds__(kTileThreads)
-dq_prep2_kernel(const BlockRuns r, const float* __restrict__ S, int b,
-                __nv_bfloat16* __restrict__ Sh, __nv_bfloat16* __restrict__ SmQ) {
-  __shared__ Tile up;
-  PairCtx c;
-  pair_ctx(b, c);
-  int run, local;
-  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
-  const int64_t base = (int64_t)c.g * c.bb;
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    if (h == 1 && c.diag) break;
-    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
-    const int64_t off = base + (int64_t)i * b + j;
-    const float4 s4 = ld4(S + off);
-    const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-    float m[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k)
-      m[k] = sv[k] - 2.f * (h ? -up.v[c.c0 + k][c.r] : up.v[c.r][c.c0 + k]);
-    st4h(Sh + off, sv);
-    st4h(SmQ + off, m);
+    put_hilo4(Qh, Ql, base + off, qv);
   }
 }
 
@@ -344,17 +258,32 @@ dq_pack_kernel(const BlockRuns r, const float* __restrict__ V, const float* __re
   }
 }
 
-// C_g = X_g Y_g for nb blocks of b x b (fp32 out), X K-major [nb*b][kx] (kx = K), Y MN-major
-// [nb*K][b]. K = b (single pass) or 3b (split operands).
-cudaError_t block_product(const void* X, const void* Y, float* C, int64_t nb, int64_t b,
-                          int64_t K, const char* name, cudaStream_t s) {
+// C_g = X_g Y_g for `groups` blocks of b x b (fp32 accumulators), X K-major [groups*b][kx],
+// Y MN-major [groups*K][b] (K = b), with an optional epilogue mode and K segments.
+umma::Gemm block_gemm(const void* X, int64_t x_rows, const void* Y, int64_t y_rows, int64_t groups,
+                      int64_t b, int64_t K, const char* name) {
   umma::Gemm g;
-  g.M = b; g.N = b; g.K = K; g.groups = nb;
-  g.A = X; g.a_rows = nb * b; g.a_cols = K; g.a_ld = K; g.a_mn = false; g.a_gm = b; g.a_gk = 0;
-  g.B = Y; g.b_rows = nb * K; g.b_cols = b; g.b_ld = b; g.b_mn = true; g.b_gn = 0; g.b_gk = K;
-  g.C = C; g.out_f32 = true; g.ldc = b; g.c_gs = b * b;
+  g.M = b; g.N = b; g.K = K; g.groups = groups;
+  g.A = X; g.a_rows = x_rows; g.a_cols = b; g.a_ld = b; g.a_mn = false; g.a_gm = b; g.a_gk = 0;
+  g.B = Y; g.b_rows = y_rows; g.b_cols = b; g.b_ld = b; g.b_mn = true; g.b_gn = 0; g.b_gk = b;
+  g.out_f32 = true; g.ldc = b; g.c_gs = b * b;
   g.name = name;
+  return g;
+}
+
+// x_hi y_hi + x_hi y_lo + x_lo y_hi over three K segments: X = [X_hi; X_lo] and
+// Y = [Y_hi; Y_lo] stacked as [2 nb b][b] (the lo halves nb*b rows below the hi halves)
+void three_pass(umma::Gemm& g, int64_t nb, int64_t b) {
+  g.K = 3 * b;
+  g.nseg = 3;
+  g.a_dy[0] = 0; g.a_dy[1] = 0; g.a_dy[2] = nb * b;
+  g.b_dy[0] = 0; g.b_dy[1] = nb * b; g.b_dy[2] = 0;
+}
+
+cudaError_t run_block_gemm(const umma::Gemm& g, cudaStream_t s) {
   if (!umma::supported(g)) return cudaErrorNotSupported;
+  // CTA pairs (256 x 256 tiles, half the operand traffic per MMA) for b a multiple of 256
+  if (umma::pair_supported(g)) return umma::gemm_pair(g, s);
   return umma::gemm(g, s);
 }
 
@@ -369,80 +298,103 @@ cudaError_t block_product(const void* X, const void* Y, float* C, int64_t nb, in
 bool tc_blocks_supported(int64_t b) { return b % 128 == 0 && b >= 128; }
 
 size_t cnp_tc_ws_bytes(int64_t nb, int64_t b) {
-  const size_t cat = align_up((size_t)(nb * b * 3 * b) * 2, 256);
-  const size_t f = align_up((size_t)(nb * b * b) * 4, 256);
-  return 2 * cat + 2 * f;
+  // [Q_hi; Q_lo], [S_hi; S_lo], [H_hi; H_lo]
+  return 3 * align_up((size_t)(2 * nb * b * b) * 2, 256);
 }
 
 cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s) {
   const int64_t nb = (int64_t)r.nb[0] + r.nb[1];
   if (nb == 0) return cudaSuccess;
+  const int64_t bb = b * b;
   Arena a(ws, cnp_tc_ws_bytes(nb, b));
-  auto* Acat = static_cast<__nv_bfloat16*>(a.take((size_t)(nb * b * 3 * b) * 2));
-  auto* Bcat = static_cast<__nv_bfloat16*>(a.take((size_t)(nb * b * 3 * b) * 2));
-  auto* S = static_cast<float*>(a.take((size_t)(nb * b * b) * 4));
-  auto* P = static_cast<float*>(a.take((size_t)(nb * b * b) * 4));
+  auto* Qst = static_cast<__nv_bfloat16*>(a.take((size_t)(2 * nb * bb) * 2));
+  auto* Sst = static_cast<__nv_bfloat16*>(a.take((size_t)(2 * nb * bb) * 2));
+  auto* Hst = static_cast<__nv_bfloat16*>(a.take((size_t)(2 * nb * bb) * 2));
   const dim3 grid = pair_grid(nb, b);
-  const int bi = (int)b;
   {
     TraceScope t("cnp_split_Q", s);
-    split_q_kernel<<<grid, kTileThreads, 0, s>>>(r, bi, Acat, Bcat);
+    split_q_kernel<<<grid, kTileThreads, 0, s>>>(r, (int)b, Qst, Qst + nb * bb);
     POETX_TRY(cudaGetLastError());
   }
-  POETX_TRY(block_product(Acat, Bcat, S, nb, b, 3 * b, "umma_cnp_QQ", s));
   {
-    TraceScope t("cnp_split_SH", s);
-    split_sh_kernel<<<grid, kTileThreads, 0, s>>>(r, S, bi, Acat, Bcat);
-    POETX_TRY(cudaGetLastError());
+    umma::Gemm g = block_gemm(Qst, 2 * nb * b, Qst, 2 * nb * b, nb, b, b, "umma_cnp_QQ");
+    three_pass(g, nb, b);
+    g.epi.mode = umma::kEpiCnpS;
+    g.epi.b = (int)b;
+    g.epi.qh = Qst; g.epi.ql = Qst + nb * bb;
+    g.epi.o[0] = Sst; g.epi.o[1] = Sst + nb * bb; g.epi.o[2] = Hst; g.epi.o[3] = Hst + nb * bb;
+    POETX_TRY(run_block_gemm(g, s));
   }
-  POETX_TRY(block_product(Acat, Bcat, P, nb, b, 3 * b, "umma_cnp_SH", s));
-  TraceScope t("cnp_finish", s);
-  cnp_finish_kernel<<<grid, kTileThreads, 0, s>>>(r, P, bi);
-  return cudaGetLastError();
+  umma::Gemm g = block_gemm(Sst, 2 * nb * b, Hst, 2 * nb * b, nb, b, b, "umma_cnp_SH");
+  three_pass(g, nb, b);
+  g.epi.mode = umma::kEpiCnpG;
+  g.epi.b = (int)b;
+  g.epi.nb0 = r.nb0;
+  g.epi.qh = Qst; g.epi.ql = Qst + nb * bb;
+  for (int k = 0; k < 2; ++k) {
+    g.epi.g[k] = r.g[k];
+    g.epi.g_lp[k] = r.g_lp[k];
+  }
+  return run_block_gemm(g, s);
 }
 
 size_t dq_tc_ws_bytes(int64_t nb, int64_t b) {
   const size_t h = align_up((size_t)(nb * b * b) * 2, 256);
   const size_t f = align_up((size_t)(nb * b * b) * 4, 256);
-  return 5 * h + 3 * f;
+  return 6 * h + 3 * f;
 }
 
 cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cudaStream_t s) {
   const int64_t nb = (int64_t)r.nb[0] + r.nb[1];
   if (nb == 0) return cudaSuccess;
+  const int64_t bb = b * b;
+  // element offsets of 256-byte-aligned slices: nb * b * b is a multiple of 128 here
   Arena a(ws, dq_tc_ws_bytes(nb, b));
-  const size_t hb = (size_t)(nb * b * b) * 2, fb = (size_t)(nb * b * b) * 4;
+  const size_t hb = (size_t)(nb * bb) * 2, fb = (size_t)(nb * bb) * 4;
   auto* Qh = static_cast<__nv_bfloat16*>(a.take(hb));
-  auto* dGh = static_cast<__nv_bfloat16*>(a.take(hb));
-  auto* Sh = static_cast<__nv_bfloat16*>(a.take(hb));
-  auto* SmQ = static_cast<__nv_bfloat16*>(a.take(hb));
+  auto* Ql = static_cast<__nv_bfloat16*>(a.take(hb));
+  auto* hst = static_cast<__nv_bfloat16*>(a.take(3 * hb));   // S_h, dG_h, SmQ, contiguous
+  __nv_bfloat16* Sh = hst;
+  __nv_bfloat16* dGh = hst + nb * bb;
+  __nv_bfloat16* SmQ = hst + 2 * nb * bb;
   auto* Zh = static_cast<__nv_bfloat16*>(a.take(hb));
-  auto* S = static_cast<float*>(a.take(fb));
-  auto* Hb = static_cast<float*>(a.take(fb));
-  auto* T1 = static_cast<float*>(a.take(fb));
+  auto* fst = static_cast<float*>(a.take(2 * fb));            // Hbar, T1, contiguous
+  float* Hb = fst;
+  float* T1 = fst + nb * bb;
+  auto* V = static_cast<float*>(a.take(fb));
   const dim3 grid = pair_grid(nb, b);
   const int bi = (int)b;
   {
     TraceScope t("dq_prep", s);
-    dq_prep_kernel<<<grid, kTileThreads, 0, s>>>(r, bi, dG, Qh, dGh);
+    dq_prep_kernel<<<grid, kTileThreads, 0, s>>>(r, bi, dG, Qh, Ql, dGh);
     POETX_TRY(cudaGetLastError());
   }
-  POETX_TRY(block_product(Qh, Qh, S, nb, b, b, "umma_dq_QQ", s));
   {
-    TraceScope t("dq_prep2", s);
-    dq_prep2_kernel<<<grid, kTileThreads, 0, s>>>(r, S, bi, Sh, SmQ);
-    POETX_TRY(cudaGetLastError());
+    umma::Gemm g = block_gemm(Qh, nb * b, Qh, nb * b, nb, b, b, "umma_dq_QQ");
+    g.epi.mode = umma::kEpiDqS;
+    g.epi.b = bi;
+    g.epi.qh = Qh; g.epi.ql = Ql;
+    g.epi.o[0] = Sh; g.epi.o[1] = SmQ;
+    POETX_TRY(run_block_gemm(g, s));
   }
-  POETX_TRY(block_product(Sh, dGh, Hb, nb, b, b, "umma_dq_SdG", s));
-  POETX_TRY(block_product(dGh, SmQ, T1, nb, b, b, "umma_dq_dGH", s));
+  {
+    // Hbar_g = S_g dG_g (groups 0..nb-1) and T1_g = dG_g SmQ_g (groups nb..2nb-1)
+    umma::Gemm g = block_gemm(Sh, 2 * nb * b, dGh, 2 * nb * b, 2 * nb, b, b, "umma_dq_SdG_dGH");
+    g.C = fst;
+    POETX_TRY(run_block_gemm(g, s));
+  }
   {
     TraceScope t("dq_mid", s);
-    dq_mid_kernel<<<grid, kTileThreads, 0, s>>>(dG, T1, Hb, bi, Zh, S);
+    dq_mid_kernel<<<grid, kTileThreads, 0, s>>>(dG, T1, Hb, bi, Zh, V);
     POETX_TRY(cudaGetLastError());
   }
-  POETX_TRY(block_product(Zh, Qh, T1, nb, b, b, "umma_dq_ZQ", s));
+  {
+    umma::Gemm g = block_gemm(Zh, nb * b, Qh, nb * b, nb, b, b, "umma_dq_ZQ");
+    g.C = T1;
+    POETX_TRY(run_block_gemm(g, s));
+  }
   TraceScope t("dq_pack", s);
-  dq_pack_kernel<<<grid, kTileThreads, 0, s>>>(r, S, T1, bi);
+  dq_pack_kernel<<<grid, kTileThreads, 0, s>>>(r, V, T1, bi);
   return cudaGetLastError();
 }
 

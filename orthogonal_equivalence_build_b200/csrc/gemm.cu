@@ -126,6 +126,30 @@ cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, i
   return simt_gemm(g, s);
 }
 
+bool dense_i8_fused(int64_t M, int64_t N) { return M >= 256 && N % 256 == 0; }
+
+cudaError_t gemm_dense_i8(const void* A, const int8_t* Wq, const float* scale, void* C, int64_t M,
+                          int64_t N, int64_t K, bool w_trans, void* deq_ws, cudaStream_t s) {
+  if (dense_i8_fused(M, N)) {
+    umma::Gemm g;
+    g.M = M; g.N = N; g.K = K;
+    g.A = A; g.a_rows = M; g.a_cols = K; g.a_ld = K; g.a_mn = false;
+    g.B = Wq; g.b_i8 = true; g.b_scale = scale;
+    if (w_trans) { g.b_rows = N; g.b_cols = K; g.b_ld = K; g.b_mn = false; }
+    else { g.b_rows = K; g.b_cols = N; g.b_ld = N; g.b_mn = true; }
+    g.C = C; g.ldc = N;
+    g.name = w_trans ? "umma_dense_W0T_i8" : "umma_dense_W0_i8";
+    if (!umma::pair_supported(g)) return cudaErrorNotSupported;
+    return umma::gemm_pair(g, s);
+  }
+  if (!deq_ws) return cudaErrorInvalidValue;
+  auto* W = static_cast<__nv_bfloat16*>(deq_ws);
+  const int64_t rows = w_trans ? N : K, cols = w_trans ? K : N;
+  cudaError_t e = dequantize_cols_i8(Wq, scale, rows, cols, W, s);
+  if (e != cudaSuccess) return e;
+  return gemm_dense(DT::BF16, A, W, C, M, N, K, w_trans, s);
+}
+
 size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows) {
   if (t != DT::BF16) return 0;
   const int sp = umma::effective_splits(rows, grad_splits(width / b, b, rows));

@@ -15,6 +15,13 @@ cudaError_t gemm_blockwise_left(DT t, const void* G, const void* N, void* C, int
 // C [M, N] = A [M, K] W, with W [K, N] (w_trans = false) or W^T for W [N, K] (w_trans = true).
 cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, int64_t N,
                        int64_t K, bool w_trans, cudaStream_t s);
+// The same product with an 8-bit W ("POET-XQ"): int8 codes Wq (layout as W above) with fp32
+// scales per column of the stored tensor, used as bf16(code * scale). The dequantisation runs
+// inside the CTA-pair kernel's operand pipeline when dense_i8_fused(M, N); otherwise Wq is first
+// dequantised into deq_ws (K * N bf16) and the bf16 product runs.
+bool dense_i8_fused(int64_t M, int64_t N);
+cudaError_t gemm_dense_i8(const void* A, const int8_t* Wq, const float* scale, void* C, int64_t M,
+                          int64_t N, int64_t K, bool w_trans, void* deq_ws, cudaStream_t s);
 // dG_j = A_j^T B_j (contraction over the rows): A, B [rows, width], dG [width/b, b, b] fp32.
 // bf16 operands split the contraction over `grad_splits` ranges of rows. With more than one
 // range the fp32 partial products go to `partials` ([splits][width/b][b][b], block_grad_ws_bytes

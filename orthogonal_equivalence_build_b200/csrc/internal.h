@@ -3,6 +3,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stddef.h>
 #include <stdint.h>
 
@@ -18,11 +19,18 @@ void trace_end(int slot, cudaStream_t s);
 // Device error word (bounded waits that expired write a nonzero code here).
 int* device_error_word();
 
+// Also an NVTX range of the same name around the launch (a no-op unless a tool such as ncu is
+// attached), so profilers can select a kernel by the library's name for it.
 struct TraceScope {
   int slot;
   cudaStream_t s;
-  TraceScope(const char* name, cudaStream_t st) : slot(trace_begin(name, st)), s(st) {}
-  ~TraceScope() { trace_end(slot, s); }
+  TraceScope(const char* name, cudaStream_t st) : slot(trace_begin(name, st)), s(st) {
+    nvtxRangePushA(name);
+  }
+  ~TraceScope() {
+    trace_end(slot, s);
+    nvtxRangePop();
+  }
 };
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -74,6 +82,14 @@ struct SimtGemm {
   float alpha, beta, diag;
 };
 cudaError_t simt_gemm(const SimtGemm& g, cudaStream_t s);
+
+// ------------------------------------------------------------------ 8-bit W0' (quant.cu)
+// Per-column symmetric int8 codes of w [m, n] (bf16 or fp32) and their fp32 scales [n].
+cudaError_t quantize_cols_i8(const void* w, DT t, int64_t m, int64_t n, int8_t* q, float* scale,
+                             cudaStream_t s);
+// out [m, n] = bf16(q * scale[col])
+cudaError_t dequantize_cols_i8(const int8_t* q, const float* scale, int64_t m, int64_t n,
+                               __nv_bfloat16* out, cudaStream_t s);
 
 // ------------------------------------------------------------------ CNP and dq (cnp.cu)
 size_t cnp_ws_bytes(int64_t nb, int64_t b);

@@ -36,16 +36,34 @@ constexpr int kThreads = 192;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per drain wait
 
-enum : int { kErrProducer = 0x101, kErrMma = 0x102, kErrEpilogue = 0x103 };
+enum : int { kErrProducer = 0x101, kErrMma = 0x102, kErrEpilogue = 0x103, kErrConvert = 0x104 };
 
 struct Params {
   int M, N, K, groups, splits;
   int tiles_m, tiles_n, kblocks_per_split, total_tiles;
   int a_gm, a_gk, b_gn, b_gk;   // per-group coordinate offsets (elements)
+  int nseg, kb_per_seg;         // K segments (see umma_gemm.h)
+  int a_dx[3], a_dy[3], b_dx[3], b_dy[3];
   void* C;
   long long ldc, c_gs, c_split;
+  Epi epi;
   int* err;
 };
+
+// TMA coordinate shifts of K block kb: k restarts at 0 in every segment.
+struct KCoord {
+  int k, adx, ady, bdx, bdy;
+};
+template <typename P>
+__device__ __forceinline__ KCoord k_coord(const P& p, int kb) {
+  KCoord c{kb * BK, 0, 0, 0, 0};
+  if (p.nseg > 1) {
+    const int s = kb / p.kb_per_seg;
+    c.k = (kb - s * p.kb_per_seg) * BK;
+    c.adx = p.a_dx[s]; c.ady = p.a_dy[s]; c.bdx = p.b_dx[s]; c.bdy = p.b_dy[s];
+  }
+  return c;
+}
 
 // ------------------------------------------------------------------ PTX wrappers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -72,6 +90,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// The same test with cluster-scope acquire: for barriers that other CTAs of the cluster
+// release into (their arrivals order their own shared-memory writes before this thread's reads).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -84,12 +115,14 @@ struct Ctl {
 };
 
 // Wait for `parity` on `bar`; false if the CTA is aborting or the wait expired.
+template <bool CLUSTER = false>
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl c, int code,
                                           uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (test()) return true;
     if ((it & 31) == 0) {
       if (*c.abort) return false;
       if (global_ns() - t0 > limit_ns) {
@@ -193,11 +226,61 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile) {
 // column; off0: element offset of the warp's first row in C at the tile's first column.
 constexpr int kEpiStageBytes = 8192;
 
+__device__ __forceinline__ void st4h(__nv_bfloat16* p, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+}
+// hi = bf16(x), lo = bf16(x - hi): x = hi + lo to about 16 significant bits
+__device__ __forceinline__ void st4_split(__nv_bfloat16* hi, __nv_bfloat16* lo, const float (&x)[4]) {
+  float h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    h[k] = __bfloat162float(__float2bfloat16_rn(x[k]));
+    l[k] = x[k] - h[k];
+  }
+  st4h(hi, h);
+  st4h(lo, l);
+}
+
+__device__ __forceinline__ void unpack4h(uint2 u, float (&v)[4]) {
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+  v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
+}
+
+// Elementwise step after a grouped b x b product at (g; i, j..j+3): acc = the four sums, q = Q.
+__device__ __forceinline__ void epi_apply(const Epi& e, int g, int i, int j, const float (&acc)[4],
+                                          const float (&q)[4]) {
+  const long long bb = (long long)e.b * e.b;
+  const long long off = (long long)g * bb + (long long)i * e.b + j;
+  if (e.mode == kEpiCnpS) {
+    float h[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) h[k] = (i == j + k ? 2.f : 0.f) + 2.f * q[k] + acc[k];
+    st4_split(e.o[0] + off, e.o[1] + off, acc);
+    st4_split(e.o[2] + off, e.o[3] + off, h);
+  } else if (e.mode == kEpiCnpG) {
+    float v[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) v[k] = (i == j + k ? 1.f : 0.f) + 2.f * q[k] + acc[k];
+    const int run = g < e.nb0 ? 0 : 1;
+    const long long loc = (long long)(g - (run ? e.nb0 : 0)) * bb + (long long)i * e.b + j;
+    if (e.g[run]) *reinterpret_cast<float4*>(e.g[run] + loc) = make_float4(v[0], v[1], v[2], v[3]);
+    if (e.g_lp[run]) st4h(e.g_lp[run] + loc, v);
+  } else if (e.mode == kEpiDqS) {
+    float m[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) m[k] = acc[k] - 2.f * q[k];
+    st4h(e.o[0] + off, acc);
+    st4h(e.o[1] + off, m);
+  }
+}
+
 template <bool OUT_F32>
 __device__ __forceinline__ void epilogue_warp_rows(uint32_t tmem_row0, int ncols,
                                                    uint8_t* __restrict__ stage, void* C,
                                                    long long off0, long long ldc, int nlive,
-                                                   int lane) {
+                                                   int lane, const Epi& epi, int g, int row0,
+                                                   int col0) {
   constexpr int ESZ = OUT_F32 ? 4 : 2;
   constexpr int ROWB = 64 * ESZ;      // bytes of one row per 64-column chunk
   constexpr int V16 = ROWB / 16;      // 16-byte pieces per row chunk: 8 (bf16) or 16 (fp32)
@@ -229,13 +312,45 @@ __device__ __forceinline__ void epilogue_warp_rows(uint32_t tmem_row0, int ncols
       }
     }
     __syncwarp();
+    if (OUT_F32 && epi.mode != kEpiStore) {
+      // Q at this lane's 32 / RPI positions of the chunk: every load issued before any use
+      constexpr int NR = 32 / RPI;
+      const long long bb = (long long)epi.b * epi.b;
+      const long long qoff0 = (long long)g * bb + (long long)(row0 + rsub) * epi.b + col0 + c + sub * 4;
+      uint2 qh[NR], ql[NR];
 #pragma unroll
-    for (int i = 0; i < 32 / RPI; ++i) {
-      const int r = i * RPI + rsub;
-      if (r < nlive) {
-        const uint4 v =
-            *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
-        *reinterpret_cast<uint4*>(Cb + (off0 + (long long)r * ldc + c) * ESZ + sub * 16) = v;
+      for (int i = 0; i < NR; ++i) {
+        const int r = i * RPI + rsub;
+        const long long o = qoff0 + (long long)(i * RPI) * epi.b;
+        qh[i] = r < nlive ? __ldg(reinterpret_cast<const uint2*>(epi.qh + o)) : make_uint2(0, 0);
+        ql[i] = (r < nlive && epi.ql) ? __ldg(reinterpret_cast<const uint2*>(epi.ql + o))
+                                      : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        const int r = i * RPI + rsub;
+        if (r < nlive) {
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
+          const float a[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
+                              __uint_as_float(v.w)};
+          float q[4], l[4];
+          unpack4h(qh[i], q);
+          unpack4h(ql[i], l);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) q[k] += l[k];
+          epi_apply(epi, g, row0 + r, col0 + c + sub * 4, a, q);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32 / RPI; ++i) {
+        const int r = i * RPI + rsub;
+        if (r < nlive) {
+          const uint4 v =
+              *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
+          *reinterpret_cast<uint4*>(Cb + (off0 + (long long)r * ldc + c) * ESZ + sub * 16) = v;
+        }
       }
     }
     __syncwarp();
@@ -313,22 +428,23 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
           }
           const uint32_t fb = smem_u32(full + s);
           mbar_expect_tx(fb, A_BYTES + B_BYTES);
-          const int k = kb * BK;
+          const KCoord kc = k_coord(p, kb);
+          const int k = kc.k;
           if constexpr (A_MN) {
 #pragma unroll
             for (int h = 0; h < BM / 64; ++h)
-              tma_load_2d(smem_u32(sa + s * A_BYTES + h * 64 * BK * 2), &tma_a, fb, am + 64 * h,
-                          ak + k);
+              tma_load_2d(smem_u32(sa + s * A_BYTES + h * 64 * BK * 2), &tma_a, fb,
+                          am + 64 * h + kc.adx, ak + k + kc.ady);
           } else {
-            tma_load_2d(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k, am);
+            tma_load_2d(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx, am + kc.ady);
           }
           if constexpr (B_MN) {
 #pragma unroll
             for (int h = 0; h < BN / 64; ++h)
-              tma_load_2d(smem_u32(sb + s * B_BYTES + h * 64 * BK * 2), &tma_b, fb, bn + 64 * h,
-                          bk + k);
+              tma_load_2d(smem_u32(sb + s * B_BYTES + h * 64 * BK * 2), &tma_b, fb,
+                          bn + 64 * h + kc.bdx, bk + k + kc.bdy);
           } else {
-            tma_load_2d(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k, bn);
+            tma_load_2d(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx, bn + kc.bdy);
           }
         }
       }
@@ -401,7 +517,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
                              (long long)row0 * p.ldc + (long long)tc.nb * BN;
       epilogue_warp_rows<OUT_F32>(
           tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN), BN,
-          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane);
+          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane, p.epi, tc.g, row0,
+          tc.nb * BN);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
@@ -434,8 +551,12 @@ struct PairParams {
   int M, N, K, groups, splits;
   int tiles_m, tiles_n, kblocks_per_split, total_tiles;   // tiles of 256 x 256
   int a_gm, a_gk, b_gn, b_gk;
+  int nseg, kb_per_seg;
+  int a_dx[3], a_dy[3], b_dx[3], b_dy[3];
   void* C;
   long long ldc, c_gs, c_split;
+  const float* b_scale;   // int8 B only: one scale per column of the stored B tensor
+  Epi epi;
   int* err;
 };
 
@@ -509,11 +630,57 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const PairParams& p, int t
   return t;
 }
 
-template <bool A_MN, bool B_MN, bool OUT_F32>
-__global__ void __launch_bounds__(kThreads, 1)
+// int8 B operand (8-bit weight storage, "POET-XQ"): B is stored as int8 codes with one fp32
+// scale per column of the stored tensor. The producer streams the int8 tile (8 KB per CTA and
+// stage) into a separate staging ring; four converter warps turn it into the bf16 operand
+// bf16(code * scale) in the 128-byte-swizzled stage the MMA reads, then arrive on the leader's
+// full barrier (which also counts the A bytes of both CTAs). The MMA and epilogue are unchanged.
+constexpr int kPairConvThreads = 128;
+
+// float(q) for a signed byte q without a conversion instruction: q + 128 = byte ^ 0x80 placed in
+// the low mantissa bits of 2^23 (0x4B000000) is the float 2^23 + 128 + q; subtracting 2^23 + 128
+// is exact. Then the fp32 product with the column scale (round to nearest), as in the reference
+// definition bf16(fp32(q) * s).
+__device__ __forceinline__ float byte_to_float(uint32_t flipped_word, int byte) {
+  return __uint_as_float(__byte_perm(flipped_word, 0x4B000000u, 0x7540u | (uint32_t)byte)) -
+         8388736.0f;
+}
+__device__ __forceinline__ uint4 dequant8(uint2 w, const float (&sc)[8]) {
+  const uint32_t x0 = w.x ^ 0x80808080u, x1 = w.y ^ 0x80808080u;
+  float f[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[i] = __fmul_rn(byte_to_float(x0, i), sc[i]);
+    f[4 + i] = __fmul_rn(byte_to_float(x1, i), sc[4 + i]);
+  }
+  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                    pack_bf16x2(f[6], f[7]));
+}
+
+__device__ __forceinline__ void load_scales8(const float* __restrict__ p, float (&sc)[8]) {
+  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
+  sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
+}
+
+template <bool B_I8>
+struct PairCfg {
+  static constexpr int STAGES = B_I8 ? 5 : 6;
+  static constexpr int RAW = B_I8 ? 4 : 0;          // int8 staging slots
+  static constexpr int RAW_BYTES = 128 * BK;        // this CTA's 128 B rows (or columns) x 64
+  static constexpr int THREADS = kThreads + (B_I8 ? kPairConvThreads : 0);
+  static constexpr size_t SMEM = (size_t)STAGES * (128 * BK * 2 * 2) + (size_t)RAW * RAW_BYTES +
+                                 4 * kEpiStageBytes + 1024 + 256;
+};
+
+template <bool A_MN, bool B_MN, bool OUT_F32, bool B_I8>
+__global__ void __launch_bounds__(PairCfg<B_I8>::THREADS, 1)
 umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b, const PairParams p) {
-  constexpr int STAGES = 6;
+  using Cfg = PairCfg<B_I8>;
+  constexpr int STAGES = Cfg::STAGES;
+  constexpr int RAW = Cfg::RAW;
   constexpr int A_BYTES = 128 * BK * 2;  // this CTA's 128 rows of A, 16 KB
   constexpr int B_BYTES = 128 * BK * 2;  // this CTA's 128 rows (N) of B, 16 KB
   constexpr int ACC_COLS = 256;
@@ -523,14 +690,17 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                                              ~static_cast<uintptr_t>(1023));
   uint8_t* sa = smem;
   uint8_t* sb = smem + STAGES * A_BYTES;
-  uint8_t* sepi = sb + STAGES * B_BYTES;   // 4 epilogue warps x 8 KB
+  uint8_t* sq = sb + STAGES * B_BYTES;     // int8 staging (B_I8)
+  uint8_t* sepi = sq + RAW * Cfg::RAW_BYTES;   // 4 epilogue warps x 8 KB
   uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + 4 * kEpiStageBytes);
   uint64_t* full = bars;                   // used in the leader only
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = bars + 2 * STAGES + 2;  // used in the leader only (8 arrivals)
-  uint64_t* drain = bars + 2 * STAGES + 4;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+  uint64_t* tempty = tfull + 2;            // used in the leader only (8 arrivals)
+  uint64_t* drain = tempty + 2;
+  uint64_t* qfull = drain + 1;             // int8 staging slot loaded (local)
+  uint64_t* qempty = qfull + RAW;          // int8 staging slot read by the converters (local)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(qempty + RAW);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -541,7 +711,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(smem_u32(full + s), 1);
+      // B_I8: the producer's arrive plus one per converter warp of both CTAs
+      mbar_init(smem_u32(full + s), B_I8 ? 1 + 2 * (kPairConvThreads / 32) : 1);
       mbar_init(smem_u32(empty + s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -549,6 +720,10 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       mbar_init(smem_u32(tempty + a), 8);
     }
     mbar_init(smem_u32(drain), 1);
+    for (int r = 0; r < RAW; ++r) {
+      mbar_init(smem_u32(qfull + r), 1);
+      mbar_init(smem_u32(qempty + r), kPairConvThreads / 32);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -581,30 +756,52 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             ok = false;
             break;
           }
-          const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
-          if (leader) mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + B_BYTES));
-          const int k = kb * BK;
-          if constexpr (A_MN) {
-            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, am, ak + k);
-            tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), &tma_a, fb, am + 64,
-                             ak + k);
-          } else {
-            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k, am);
+          if constexpr (B_I8) {
+            const int r = it % RAW;
+            if (!wait_bounded(smem_u32(qempty + r), ((uint32_t)(it / RAW) & 1u) ^ 1u, ctl,
+                              kErrProducer, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
           }
-          if constexpr (B_MN) {
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn, bk + k);
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb, bn + 64,
-                             bk + k);
+          const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
+          if (leader)
+            mbar_expect_tx(smem_u32(full + s), B_I8 ? 2 * A_BYTES : 2 * (A_BYTES + B_BYTES));
+          const KCoord kc = k_coord(p, kb);
+          const int k = kc.k;
+          if constexpr (A_MN) {
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, am + kc.adx, ak + k + kc.ady);
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), &tma_a, fb,
+                             am + 64 + kc.adx, ak + k + kc.ady);
           } else {
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k, bn);
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx, am + kc.ady);
+          }
+          if constexpr (B_I8) {
+            // int8 tile into this CTA's staging slot, completing its own local barrier
+            const int r = it % RAW;
+            const uint32_t qb = smem_u32(qfull + r);
+            mbar_expect_tx(qb, Cfg::RAW_BYTES);
+            if constexpr (B_MN) tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bn, bk + k);
+            else tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bk + k, bn);
+          } else if constexpr (B_MN) {
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx, bk + k + kc.bdy);
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
+                             bn + 64 + kc.bdx, bk + k + kc.bdy);
+          } else {
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx, bn + kc.bdy);
           }
         }
       }
-      if (!ok && leader) {
-        // the leader's full barriers count both CTAs' bytes: let them land
-        for (int j = max(0, it - STAGES); j < it; ++j)
-          wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
-                       kDrainLimitNs);
+      if (!ok) {
+        // the leader's full barriers count both CTAs' A (and bf16 B) bytes: let them land
+        if (leader)
+          for (int j = max(0, it - STAGES); j < it; ++j)
+            wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
+                         kDrainLimitNs);
+        if constexpr (B_I8)
+          for (int j = max(0, it - RAW); j < it; ++j)
+            wait_bounded(smem_u32(qfull + j % RAW), (uint32_t)(j / RAW) & 1u, ctl, 0,
+                         kDrainLimitNs);
       }
     }
     __syncwarp();  // reconverge before the block-wide barriers below
@@ -628,7 +825,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!wait_bounded(smem_u32(full + s), ph, ctl, kErrMma, kWaitLimitNs)) {
+          if (!wait_bounded<B_I8>(smem_u32(full + s), ph, ctl, kErrMma, kWaitLimitNs)) {
             ok = false;
             break;
           }
@@ -651,7 +848,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       wait_bounded(smem_u32(drain), 0, ctl, ok ? kErrMma : 0, ok ? kWaitLimitNs : kDrainLimitNs);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     const int quarter = warp & 3;
     const uint32_t leader_tempty0 = map_to_rank(smem_u32(tempty), 0);
     int tcount = 0;
@@ -667,11 +864,79 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                              (long long)row0 * p.ldc + (long long)tc.nb * 256;
       epilogue_warp_rows<OUT_F32>(
           tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS), ACC_COLS,
-          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane);
+          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane, p.epi, tc.g, row0,
+          tc.nb * 256);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(leader_tempty0 + (uint32_t)(acc * 8));
     }
+  } else if constexpr (B_I8) {
+    // ------------------------------------------------------------ int8 -> bf16 converters
+    // Thread ct owns one 8-element unit column of the staged tile and 8 of its 64 (B_MN) or
+    // 128 (K-major) lines: 8-byte conflict-free reads, 16-byte swizzled conflict-free writes.
+    const int ct = threadIdx.x - kThreads;
+    const uint32_t leader_full0 = map_to_rank(smem_u32(full), 0);
+    int it = 0;
+    bool ok = true;
+    for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
+      const TileCoord tc = decode_pair_tile(p, tile);
+      const int kb0 = tc.split * p.kblocks_per_split;
+      const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
+      const int bn = tc.g * p.b_gn + tc.nb * 256 + (int)rank * 128;
+      float sc[8];
+      if constexpr (B_MN) load_scales8(p.b_scale + bn + 8 * (ct & 15), sc);   // per N column
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES, r = it % RAW;
+        bool got = wait_bounded(smem_u32(qfull + r), (uint32_t)(it / RAW) & 1u, ctl, kErrConvert,
+                                kWaitLimitNs);
+        got = got && wait_bounded(smem_u32(empty + s), ((uint32_t)(it / STAGES) & 1u) ^ 1u, ctl,
+                                  kErrConvert, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* q = sq + r * Cfg::RAW_BYTES;
+        uint8_t* dst = sb + s * B_BYTES;
+        if constexpr (B_MN) {
+          // staged int8 tile: 64 K lines of 128 N bytes; bf16 stage: two 64-column chunks of
+          // 64 K lines x 128 B, 16-byte unit u of line k at (u ^ (k & 7))
+          const int nu = ct & 15, k0 = ct >> 4;
+          uint8_t* d0 = dst + (nu >> 3) * (64 * BK * 2) + ((((nu & 7) ^ k0) << 4));
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int k = k0 + 8 * i;
+            const uint2 w = *reinterpret_cast<const uint2*>(q + k * 128 + nu * 8);
+            *reinterpret_cast<uint4*>(d0 + k * 128) = dequant8(w, sc);
+          }
+        } else {
+          // staged int8 tile: 128 N lines of 64 K bytes; bf16 stage: 128 lines x 128 B,
+          // 16-byte unit u of line j at (u ^ (j & 7)); the scale runs along K
+          const int u = ct & 7, j0 = ct >> 3;
+          const int kq = kb * BK + 8 * u;   // K is a multiple of 8: a unit is all in or all out
+          if (kq < p.K) {
+            load_scales8(p.b_scale + tc.g * p.b_gk + kq, sc);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sc[e] = 0.f;
+          }
+          uint8_t* d0 = dst + ((u ^ (j0 & 7)) << 4);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = j0 + 16 * i;
+            const uint2 w = *reinterpret_cast<const uint2*>(q + j * 64 + u * 8);
+            *reinterpret_cast<uint4*>(d0 + j * 128) = dequant8(w, sc);
+          }
+        }
+        // make the generic-proxy stores visible to the tensor core's reads, then publish
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(qempty + r));
+          mbar_arrive_remote(leader_full0 + (uint32_t)(s * 8));
+        }
+      }
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -718,6 +983,20 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int6
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D int8 tensor [rows][cols] (row stride ld bytes), box {box_x, box_y}, no swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t ld,
+                 int box_x, int box_y) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld};
+  cuuint32_t box[2] = {(cuuint32_t)box_x, (cuuint32_t)box_y};
+  cuuint32_t estr[2] = {1u, 1u};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int sm_count() {
   static int n = 0;
   if (!n) {
@@ -727,6 +1006,17 @@ int sm_count() {
     if (n <= 0) n = 148;
   }
   return n;
+}
+
+template <typename P>
+void fill_segments(const Gemm& g, P& p) {
+  p.nseg = g.nseg > 1 ? g.nseg : 1;
+  p.kb_per_seg = (int)((g.K / p.nseg + BK - 1) / BK);
+  for (int s = 0; s < 3; ++s) {
+    const bool on = s < p.nseg && p.nseg > 1;
+    p.a_dx[s] = on ? (int)g.a_dx[s] : 0; p.a_dy[s] = on ? (int)g.a_dy[s] : 0;
+    p.b_dx[s] = on ? (int)g.b_dx[s] : 0; p.b_dy[s] = on ? (int)g.b_dy[s] : 0;
+  }
 }
 
 template <int BN>
@@ -751,7 +1041,9 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
   p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
   p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
+  fill_segments(g, p);
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
+  p.epi = g.epi;
   p.err = device_error_word();
   auto kern = umma_gemm_kernel<BN, A_MN, B_MN, OUT_F32, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -762,13 +1054,19 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   return cudaGetLastError();
 }
 
-template <bool A_MN, bool B_MN, bool OUT_F32>
+template <bool A_MN, bool B_MN, bool OUT_F32, bool B_I8>
 cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
-  constexpr int STAGES = 6;
-  constexpr size_t smem = (size_t)STAGES * (128 * BK * 2 * 2) + 4 * kEpiStageBytes + 1024 + 256;
+  using Cfg = PairCfg<B_I8>;
+  constexpr size_t smem = Cfg::SMEM;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : 128)) return cudaErrorInvalidValue;
-  if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
+  if constexpr (B_I8) {
+    // B_MN: 64 K lines of 128 N bytes; K-major: 128 N lines of 64 K bytes
+    if (!make_map_u8(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? 128 : BK, B_MN ? BK : 128))
+      return cudaErrorInvalidValue;
+  } else {
+    if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
+  }
   PairParams p;
   p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = (int)g.groups;
   p.tiles_m = (int)((g.M + 255) / 256);
@@ -778,9 +1076,12 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
   p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
   p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
+  fill_segments(g, p);
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
+  p.b_scale = g.b_scale;
+  p.epi = g.epi;
   p.err = device_error_word();
-  auto kern = umma_gemm_pair_kernel<A_MN, B_MN, OUT_F32>;
+  auto kern = umma_gemm_pair_kernel<A_MN, B_MN, OUT_F32, B_I8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -789,7 +1090,7 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
@@ -834,6 +1135,7 @@ int effective_splits(int64_t K, int64_t splits) {
 
 bool supported(const Gemm& g) {
   if (!encode_fn()) return false;
+  if (g.b_i8) return false;   // int8 B: CTA-pair kernel only (pair_supported)
   if (g.M <= 0 || g.N <= 0 || g.K <= 0 || g.groups <= 0) return false;
   if (g.K % BK != 0 && g.groups > 1 && g.a_gk + g.b_gk != 0) return false;
   if (g.N % 64 != 0) return false;
@@ -847,18 +1149,46 @@ bool supported(const Gemm& g) {
   const int64_t lim = (int64_t)1 << 31;
   if (g.a_rows >= lim || g.a_cols >= lim || g.b_rows >= lim || g.b_cols >= lim) return false;
   if ((g.a_gm | g.a_gk | g.b_gn | g.b_gk) % 64) return false;
+  if (g.nseg < 1 || g.nseg > 3) return false;
+  if (g.nseg > 1) {
+    if (g.K % (64 * g.nseg) || g.splits != 1) return false;
+    for (int s = 0; s < g.nseg; ++s)
+      if ((g.a_dx[s] | g.b_dx[s]) % 64 || g.a_dx[s] < 0 || g.a_dy[s] < 0 || g.b_dx[s] < 0 ||
+          g.b_dy[s] < 0)
+        return false;
+  }
+  if (g.epi.mode != kEpiStore) {
+    // grouped b x b blocks with fp32 accumulators; 16-byte aligned rows of 4 elements
+    if (!g.out_f32 || g.M != g.epi.b || g.N != g.epi.b || g.epi.b % 8 || !g.epi.qh ||
+        g.splits != 1)
+      return false;
+  }
   return true;
 }
 
 bool pair_supported(const Gemm& g) {
+  if (g.b_i8) {
+    // int8 B with per-column scales: one dense product, bf16 A K-major, bf16 out
+    Gemm h = g;
+    h.b_i8 = false;
+    return supported(h) && g.N % 256 == 0 && g.M >= 256 && g.groups == 1 && g.splits == 1 &&
+           !g.a_mn && !g.out_f32 && g.b_scale && g.b_ld % 16 == 0 && g.b_cols % 16 == 0 &&
+           (reinterpret_cast<uintptr_t>(g.b_scale) & 15) == 0;
+  }
   return supported(g) && g.N % 256 == 0 && g.M >= 256 && !(g.a_mn && !g.b_mn) &&
          !(g.a_mn && g.b_mn && !g.out_f32) && (g.groups == 1 || g.a_gm == 0 || g.a_gm % 256 == 0);
 }
 
 cudaError_t gemm_pair(const Gemm& g, cudaStream_t s) {
   const char* name = g.name ? g.name : "umma_gemm_pair";
+  if (g.b_i8) {
+    if (g.a_mn || g.out_f32) return cudaErrorNotSupported;
+    return g.b_mn ? launch_pair_t<false, true, false, true>(g, s, name)
+                  : launch_pair_t<false, false, false, true>(g, s, name);
+  }
 #define POETX_UP(AM, BMJ, F) \
-  if (g.a_mn == AM && g.b_mn == BMJ && g.out_f32 == F) return launch_pair_t<AM, BMJ, F>(g, s, name);
+  if (g.a_mn == AM && g.b_mn == BMJ && g.out_f32 == F) \
+    return launch_pair_t<AM, BMJ, F, false>(g, s, name);
   POETX_UP(false, false, false)
   POETX_UP(false, true, false)
   POETX_UP(true, true, true)

@@ -14,12 +14,44 @@ namespace umma {
 //   B MN-major (b_mn = true):  B(g; k, j) = B[b_gk*g + k][b_gn*g + j]
 // Reads beyond a tensor's rows/cols are zeros. C is bf16 or fp32 row-major:
 //   C[split * c_split + g * c_gs + i * ldc + j].
+// b_i8: B is an int8 tensor [rows][cols] (row stride ld bytes) with fp32 scales b_scale[cols];
+// the product uses B = bf16(code * b_scale[col]) (CTA-pair kernel, one dense product only).
+// K segments (nseg > 1): the contraction is nseg equal segments of K / nseg; within segment s
+// the k index restarts at 0 and the TMA coordinates of A and B are shifted by (a_dx[s], a_dy[s])
+// and (b_dx[s], b_dy[s]) (x = column, y = row of the 2-D tensor). One accumulator sums
+// A_s B_s over the segments, e.g. Xhi Yhi + Xhi Ylo + Xlo Yhi from separate hi / lo buffers.
+//
+// Epilogue modes (fp32 accumulators of grouped b x b products, groups = blocks, M = N = b):
+// instead of storing C, the epilogue evaluates the next elementwise step of the Cayley-Neumann
+// blocks or of their gradient at each element (g; i, j) and stores its results. Q(g; i, j) is
+// qh + ql (bf16 hi / lo parts of the skew block, ql may be null), all arrays [groups][b][b].
+enum EpiMode : int {
+  kEpiStore = 0,
+  kEpiCnpS = 1,   // acc = S = Q Q: o0, o1 = hi / lo of S; o2, o3 = hi / lo of H = 2I + 2Q + S
+  kEpiCnpG = 2,   // acc = S H:  G = I + 2Q + acc to g[run] (fp32) and g_lp[run] (bf16); block g
+                  // is block g of run 0 when g < nb0, else block g - nb0 of run 1
+  kEpiDqS = 3,    // acc = S = Q Q: o0 = bf16(S), o1 = bf16(S - 2Q)
+};
+struct Epi {
+  int mode = kEpiStore;
+  int b = 0, nb0 = 0;
+  const __nv_bfloat16* qh = nullptr;
+  const __nv_bfloat16* ql = nullptr;
+  __nv_bfloat16* o[4] = {nullptr, nullptr, nullptr, nullptr};
+  float* g[2] = {nullptr, nullptr};
+  __nv_bfloat16* g_lp[2] = {nullptr, nullptr};
+};
+
 struct Gemm {
   int64_t M = 0, N = 0, K = 0, groups = 1, splits = 1;
   const void* A = nullptr; int64_t a_rows = 0, a_cols = 0, a_ld = 0; bool a_mn = false;
   int64_t a_gm = 0, a_gk = 0;
   const void* B = nullptr; int64_t b_rows = 0, b_cols = 0, b_ld = 0; bool b_mn = false;
   int64_t b_gn = 0, b_gk = 0;
+  bool b_i8 = false; const float* b_scale = nullptr;
+  int nseg = 1;
+  int64_t a_dx[3] = {0, 0, 0}, a_dy[3] = {0, 0, 0}, b_dx[3] = {0, 0, 0}, b_dy[3] = {0, 0, 0};
+  Epi epi;
   void* C = nullptr; bool out_f32 = false; int64_t ldc = 0, c_gs = 0, c_split = 0;
   const char* name = nullptr;
 };

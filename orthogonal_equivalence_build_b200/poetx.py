@@ -35,7 +35,11 @@ class Layer(ctypes.Structure):
                 ("w0m", ctypes.c_void_p), ("perm_r", ctypes.c_void_p),
                 ("perm_p", ctypes.c_void_p), ("q_r", ctypes.c_void_p), ("q_p", ctypes.c_void_p),
                 ("g_r", ctypes.c_void_p), ("g_p", ctypes.c_void_p),
-                ("g_r_lp", ctypes.c_void_p), ("g_p_lp", ctypes.c_void_p)]
+                ("g_r_lp", ctypes.c_void_p), ("g_p_lp", ctypes.c_void_p),
+                ("w0m_scale", ctypes.c_void_p)]
+
+
+LAYER_W0M_I8 = 1
 
 
 def _load() -> ctypes.CDLL:
@@ -59,6 +63,8 @@ def _load() -> ctypes.CDLL:
         "poetx_merge_permutations": (I32, [V, V, V, I64, I64, I32, V, V]),
         "poetx_merge_reinit_workspace_bytes": (SZ, [LP]),
         "poetx_merge_reinit": (I32, [LP, U64, V, SZ, V]),
+        "poetx_quantize_w0": (I32, [V, I64, I64, I32, V, V, V]),
+        "poetx_dequantize_w0": (I32, [V, V, I64, I64, V, V]),
         "poetx_resample_permutation": (I32, [U64, I32, I64, V, V]),
         "poetx_validate_permutation": (I32, [V, I64, V, SZ, V]),
         "poetx_device_status": (I32, [V]),
@@ -84,7 +90,7 @@ EXPORTED = (
     "poetx_fwd_workspace_bytes",
     "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
     "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
-    "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
+    "poetx_quantize_w0", "poetx_dequantize_w0", "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
     "poetx_trace_enable", "poetx_trace_read", "poetx_status_string",
     "poetx_last_error_message", "poetx_abi_version", "poetx_testing_gemm_bf16")
 
@@ -130,24 +136,33 @@ class PoetxLinear:
 
     w0m [m, n] (dtype), perm_r [m], perm_p [n] (int32), q_r [m/b, b(b-1)/2], q_p (fp32),
     g_r [m/b, b, b], g_p (fp32) and, for bf16 layers, g_r_lp / g_p_lp (bf16).
+    An int8 w0m with its fp32 column scales w0m_scale [n] makes an 8-bit-weight layer
+    (POETX_LAYER_W0M_I8; activations and gradients bf16).
     """
 
     def __init__(self, w0m: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,
-                 q_r: torch.Tensor, q_p: torch.Tensor, b: int):
+                 q_r: torch.Tensor, q_p: torch.Tensor, b: int,
+                 w0m_scale: Optional[torch.Tensor] = None):
         m, n = w0m.shape
         dev = w0m.device
         self.b = int(b)
         self.w0m, self.perm_r, self.perm_p = w0m, perm_r, perm_p
+        self.w0m_scale = w0m_scale
         self.q_r, self.q_p = q_r, q_p
         self.g_r = torch.empty(m // b, b, b, dtype=torch.float32, device=dev)
         self.g_p = torch.empty(n // b, b, b, dtype=torch.float32, device=dev)
-        lp = w0m.dtype == torch.bfloat16
+        i8 = w0m.dtype == torch.int8
+        if i8 and w0m_scale is None:
+            raise ValueError("an int8 w0m needs w0m_scale")
+        lp = i8 or w0m.dtype == torch.bfloat16
         self.g_r_lp = torch.empty(m // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
         self.g_p_lp = torch.empty(n // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
-        self.desc = Layer(m=m, n=n, b=self.b, dtype=dtype_code(w0m.dtype), flags=0,
+        self.desc = Layer(m=m, n=n, b=self.b, dtype=BF16 if i8 else dtype_code(w0m.dtype),
+                          flags=LAYER_W0M_I8 if i8 else 0,
                           w0m=_ptr(w0m), perm_r=_ptr(perm_r), perm_p=_ptr(perm_p),
                           q_r=_ptr(q_r), q_p=_ptr(q_p), g_r=_ptr(self.g_r), g_p=_ptr(self.g_p),
-                          g_r_lp=_ptr(self.g_r_lp), g_p_lp=_ptr(self.g_p_lp))
+                          g_r_lp=_ptr(self.g_r_lp), g_p_lp=_ptr(self.g_p_lp),
+                          w0m_scale=_ptr(w0m_scale) if i8 else None)
 
     @property
     def m(self) -> int:
@@ -159,7 +174,8 @@ class PoetxLinear:
 
     @property
     def dtype(self) -> torch.dtype:
-        return self.w0m.dtype
+        """Activation / gradient dtype (bf16 for 8-bit-weight layers)."""
+        return torch.bfloat16 if self.w0m.dtype == torch.int8 else self.w0m.dtype
 
 
 # ----------------------------------------------------------------------------- entry points
@@ -239,6 +255,19 @@ def merge_reinit(layer: PoetxLinear, seed: int, workspace: Optional[torch.Tensor
     ws = _workspace(merge_reinit_workspace_bytes(layer), layer.w0m.device, workspace)
     _check(lib.poetx_merge_reinit(ctypes.byref(layer.desc), seed & ((1 << 64) - 1), _ptr(ws),
                                   0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def quantize_w0(w: torch.Tensor, wq: torch.Tensor, scale: torch.Tensor, stream=None) -> None:
+    """wq [m, n] int8, scale [n] fp32 <- per-column symmetric 8-bit codes of w (poetx_quantize_w0)."""
+    m, n = w.shape
+    _check(lib.poetx_quantize_w0(_ptr(w), m, n, dtype_code(w.dtype), _ptr(wq), _ptr(scale),
+                                 _stream(stream)))
+
+
+def dequantize_w0(wq: torch.Tensor, scale: torch.Tensor, out: torch.Tensor, stream=None) -> None:
+    """out [m, n] bf16 <- bf16(wq * scale[col]) (poetx_dequantize_w0)."""
+    m, n = wq.shape
+    _check(lib.poetx_dequantize_w0(_ptr(wq), _ptr(scale), m, n, _ptr(out), _stream(stream)))
 
 
 def resample_permutation(seed: int, lane: int, perm: torch.Tensor, stream=None) -> None:

@@ -29,7 +29,7 @@ def test_header_symbols_are_exported():
 
 
 def test_abi_version_and_strings():
-    assert poetx.abi_version() == 1
+    assert poetx.abi_version() == 2
     assert poetx.lib.poetx_status_string(0) == b"ok"
     assert poetx.lib.poetx_status_string(8) == b"workspace too small"
 
@@ -56,6 +56,10 @@ def _fwd(L, x=0x100000, T=128, y=0x200000, ws=None, wsb=0):
     (dict(g_r_lp=None), 1),                     # bf16 layer needs the bf16 copies
     (dict(perm_r=0x20004), 3),                  # misaligned
     (dict(b=2048, m=4096, n=4096), 2),          # b too large
+    (dict(flags=2), 1),                         # unknown flag
+    (dict(flags=1, w0m_scale=0xA0000, dtype=poetx.F32), 4),   # int8 W0' needs a bf16 layer
+    (dict(flags=1, w0m_scale=0xA0004), 3),      # misaligned scales
+    (dict(flags=1, w0m_scale=0xA0000, m=520, n=1040, b=8), 2),  # int8 W0' rows of 16 bytes
 ])
 def test_layer_validation(kw, status):
     assert _fwd(_layer(**kw)) == status
@@ -133,3 +137,29 @@ def test_workspaces_never_hold_an_m_by_n_buffer():
     L = _layer(m=4096, n=14336, b=512)
     assert f(ctypes.byref(L), 2048) - f(ctypes.byref(L), 1024) == \
         f(ctypes.byref(L), 4096) - f(ctypes.byref(L), 3072)
+
+
+def test_int8_w0_workspace_only_where_the_product_is_not_fused():
+    """8-bit W0' layers dequantise inside the tensor-core kernel when T >= 256 and m, n are
+    multiples of 256; other shapes need one bf16 copy of W0' in the workspace."""
+    L16 = _layer(m=4096, n=14336, b=512)
+    L8 = _layer(m=4096, n=14336, b=512, flags=1, w0m_scale=0xA0000)
+    for fn in (poetx.lib.poetx_fwd_workspace_bytes, poetx.lib.poetx_bwd_workspace_bytes):
+        assert fn(ctypes.byref(L8), 4096) == fn(ctypes.byref(L16), 4096)
+        extra = fn(ctypes.byref(L8), 128) - fn(ctypes.byref(L16), 128)
+        assert 4096 * 14336 * 2 <= extra < 4096 * 14336 * 2 + 4096
+    assert poetx.lib.poetx_merge_reinit_workspace_bytes(ctypes.byref(L8)) == \
+        poetx.lib.poetx_merge_reinit_workspace_bytes(ctypes.byref(L16))
+
+
+def test_quantize_argument_checks():
+    q = poetx.lib.poetx_quantize_w0
+    assert q(0x1000, 64, 64, 5, 0x2000, 0x3000, None) == 4
+    assert q(None, 64, 64, 1, 0x2000, 0x3000, None) == 1
+    assert q(0x1000, -1, 64, 1, 0x2000, 0x3000, None) == 2
+    assert q(0x1000, 64, 64, 1, 0x2000, 0x3004, None) == 3
+    assert q(0x1000, 0, 64, 1, 0x2000, 0x3000, None) == 0
+    d = poetx.lib.poetx_dequantize_w0
+    assert d(None, 0x3000, 64, 64, 0x4000, None) == 1
+    assert d(0x2000, 0x3000, 64, 64, 0x4008, None) == 3
+    assert d(0x2000, 0x3000, 64, 0, 0x4000, None) == 0
