@@ -348,7 +348,12 @@ def run_ours(args):
           for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize()
+    # events only around the dominant kernel inside the timed region: an event between two
+    # launches keeps the second from overlapping the first one's tail
+    w0_names = (("umma_dense_W0_i8", "umma_dense_W0T_i8") if args.xq
+                else ("umma_dense_W0", "umma_dense_W0T"))
     poetx.trace_read()
+    poetx.trace_select(w0_names)
     poetx.trace_enable(True)
     sampler.start()
     for i in range(args.steps):
@@ -381,10 +386,20 @@ def run_ours(args):
     value = T * world / (ms_per_step / 1e3)
 
     # ---- dominant kernel: the W0' GEMMs of all linears
-    w0_names = (("umma_dense_W0_i8", "umma_dense_W0T_i8") if args.xq
-                else ("umma_dense_W0", "umma_dense_W0T"))
     w0_ms = [ms for name, ms in trace if name in w0_names]
-    launches = len(trace)
+    # every library launch of a step, with its device time: a separate traced pass (3 steps)
+    poetx.trace_select(None)
+    poetx.trace_enable(True)
+    n_pass = 3
+    for _ in range(n_pass):
+        step()
+    torch.cuda.synchronize()
+    poetx.trace_enable(False)
+    full = poetx.trace_read()
+    launches = len(full) // n_pass * args.steps
+    per_kernel = {}
+    for name, ms in full:
+        per_kernel[name] = per_kernel.get(name, 0.0) + ms / n_pass
     peaks, peak_src = measured_peaks()
     roofline = None
     if w0_ms:
@@ -404,9 +419,6 @@ def run_ours(args):
     Bb = sum(layer_bytes(T, d["lin"].m, d["lin"].n, b, esz, 1 if args.xq else None)
              for d in layers)
     t_roof = max(F / (peaks["bf16_tflops"] * 1e12), Bb / (peaks["hbm_gbs"] * 1e9))
-    per_kernel = {}
-    for name, ms in trace:
-        per_kernel[name] = per_kernel.get(name, 0.0) + ms
 
     # ---- end to end through the API: pinned host inputs in, dq out, every step. Two input
     # buffers: the upload of step i+1's X and dY (copy stream) overlaps step i's kernels; a step
@@ -494,8 +506,11 @@ def run_ours(args):
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,
-            "kernel_ms_per_step": {k: v / args.steps for k, v in sorted(per_kernel.items(),
+            "kernel_ms_per_step": {k: v for k, v in sorted(per_kernel.items(),
                                                                         key=lambda kv: -kv[1])},
+            "kernel_ms_source": ("CUDA events around every library launch, separate pass of "
+                                 f"{n_pass} steps after the timed region (which records events "
+                                 "around the W0' GEMMs only)"),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -241,6 +241,13 @@ poetx_status poetx_device_status(void* stream);
  * Returns the number of launches recorded. */
 poetx_status poetx_trace_enable(int32_t on);
 int64_t poetx_trace_read(char* buf, size_t len);
+/* Record only launches whose name is one of `names` (comma-separated, exact match); NULL or ""
+ * records every launch again. Events between two launches keep the second from starting early
+ * (see below), so a selective trace disturbs the timing of the untraced launches less.
+ * Kernels on the layer's path are launched with programmatic stream serialisation: a kernel may
+ * run its set-up while the previous one finishes and waits for it before touching memory.
+ * POETX_PDL=0 in the environment turns that off. */
+poetx_status poetx_trace_select(const char* names);
 
 const char* poetx_status_string(int32_t status);
 const char* poetx_last_error_message(void);

@@ -9,6 +9,7 @@
 #include "gemm.h"
 
 #include <cstdarg>
+#include <cstdlib>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -39,6 +40,14 @@ std::mutex g_trace_mu;
 bool g_trace_on = false;
 std::vector<TraceRec> g_trace;
 std::vector<cudaEvent_t> g_event_pool;
+std::vector<std::string> g_trace_only;   // empty: every launch
+
+bool traced(const char* name) {
+  if (g_trace_only.empty()) return true;
+  for (const auto& n : g_trace_only)
+    if (n == name) return true;
+  return false;
+}
 
 cudaEvent_t pool_event() {
   if (!g_event_pool.empty()) {
@@ -55,6 +64,7 @@ cudaEvent_t pool_event() {
 int trace_begin(const char* name, cudaStream_t s) {
   if (!g_trace_on) return -1;
   std::lock_guard<std::mutex> lk(g_trace_mu);
+  if (!traced(name)) return -1;
   TraceRec r{name, pool_event(), pool_event()};
   cudaEventRecord(r.start, s);
   g_trace.push_back(r);
@@ -65,6 +75,21 @@ void trace_end(int slot, cudaStream_t s) {
   if (slot < 0) return;
   std::lock_guard<std::mutex> lk(g_trace_mu);
   if (slot < (int)g_trace.size()) cudaEventRecord(g_trace[slot].stop, s);
+}
+
+// ------------------------------------------------------------------ programmatic launch
+bool pdl_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* v = getenv("POETX_PDL");
+    on = (v && v[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
+void set_pdl_attr(cudaLaunchAttribute& a) {
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = pdl_enabled() ? 1 : 0;
 }
 
 // ------------------------------------------------------------------ device error word
@@ -291,6 +316,23 @@ const char* poetx_last_error_message(void) { return g_last_error.c_str(); }
 poetx_status poetx_trace_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(g_trace_mu);
   g_trace_on = on != 0;
+  return POETX_OK;
+}
+
+poetx_status poetx_trace_select(const char* names) {
+  std::lock_guard<std::mutex> lk(g_trace_mu);
+  g_trace_only.clear();
+  if (!names) return POETX_OK;
+  std::string cur;
+  for (const char* p = names;; ++p) {
+    if (*p == ',' || *p == 0) {
+      if (!cur.empty()) g_trace_only.push_back(cur);
+      cur.clear();
+      if (*p == 0) break;
+    } else {
+      cur.push_back(*p);
+    }
+  }
   return POETX_OK;
 }
 

@@ -130,6 +130,8 @@ __device__ __forceinline__ void put_hilo4(__nv_bfloat16* __restrict__ p_hi,
 __global__ void __launch_bounds__(kTileThreads)
 split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
                __nv_bfloat16* __restrict__ Qlo) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ Tile up;
   PairCtx c;
   pair_ctx(b, c);
@@ -153,6 +155,8 @@ __global__ void __launch_bounds__(kTileThreads)
 dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
                __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ Ql,
                __nv_bfloat16* __restrict__ dGh) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ Tile up;
   PairCtx c;
   pair_ctx(b, c);
@@ -188,6 +192,8 @@ __global__ void __launch_bounds__(kTileThreads)
 dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
               const float* __restrict__ Hb, int b, __nv_bfloat16* __restrict__ Zh,
               float* __restrict__ V) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ Tile sa, sb;  // Sbar tiles (I, J) and (J, I)
   PairCtx c;
   pair_ctx(b, c);
@@ -228,6 +234,8 @@ dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
 __global__ void __launch_bounds__(kTileThreads)
 dq_pack_kernel(const BlockRuns r, const float* __restrict__ V, const float* __restrict__ ZQ,
                int b) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ Tile ua, ub;  // U tiles (I, J) and (J, I)
   PairCtx c;
   pair_ctx(b, c);
@@ -313,8 +321,7 @@ cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s
   const dim3 grid = pair_grid(nb, b);
   {
     TraceScope t("cnp_split_Q", s);
-    split_q_kernel<<<grid, kTileThreads, 0, s>>>(r, (int)b, Qst, Qst + nb * bb);
-    POETX_TRY(cudaGetLastError());
+    POETX_TRY(launch_k(split_q_kernel, grid, dim3(kTileThreads), 0, s, r, (int)b, Qst, Qst + nb * bb));
   }
   {
     umma::Gemm g = block_gemm(Qst, 2 * nb * b, Qst, 2 * nb * b, nb, b, b, "umma_cnp_QQ");
@@ -366,8 +373,7 @@ cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cu
   const int bi = (int)b;
   {
     TraceScope t("dq_prep", s);
-    dq_prep_kernel<<<grid, kTileThreads, 0, s>>>(r, bi, dG, Qh, Ql, dGh);
-    POETX_TRY(cudaGetLastError());
+    POETX_TRY(launch_k(dq_prep_kernel, grid, dim3(kTileThreads), 0, s, r, bi, dG, Qh, Ql, dGh));
   }
   {
     umma::Gemm g = block_gemm(Qh, nb * b, Qh, nb * b, nb, b, b, "umma_dq_QQ");
@@ -385,8 +391,8 @@ cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cu
   }
   {
     TraceScope t("dq_mid", s);
-    dq_mid_kernel<<<grid, kTileThreads, 0, s>>>(dG, T1, Hb, bi, Zh, V);
-    POETX_TRY(cudaGetLastError());
+    POETX_TRY(launch_k(dq_mid_kernel, grid, dim3(kTileThreads), 0, s, (const float*)dG,
+                       (const float*)T1, (const float*)Hb, bi, Zh, V));
   }
   {
     umma::Gemm g = block_gemm(Zh, nb * b, Qh, nb * b, nb, b, b, "umma_dq_ZQ");
@@ -394,8 +400,8 @@ cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cu
     POETX_TRY(run_block_gemm(g, s));
   }
   TraceScope t("dq_pack", s);
-  dq_pack_kernel<<<grid, kTileThreads, 0, s>>>(r, V, T1, bi);
-  return cudaGetLastError();
+  return launch_k(dq_pack_kernel, grid, dim3(kTileThreads), 0, s, r, (const float*)V,
+                  (const float*)T1, bi);
 }
 
 }  // namespace poetx

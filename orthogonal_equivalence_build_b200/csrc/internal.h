@@ -33,6 +33,36 @@ struct TraceScope {
   }
 };
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// The hot-path kernels are launched with programmatic stream serialisation: a kernel may be
+// scheduled, and run its prologue (barrier set-up, TMEM allocation), while the previous kernel
+// of the stream finishes. Every such kernel calls pdl_wait() before its first global-memory
+// access; it returns once the previous grid has completed and its writes are visible, so reads
+// after writes and writes after reads across kernels keep stream order. pdl_trigger() allows the
+// next launch to be scheduled. Both are no-ops in a kernel launched without the attribute.
+// POETX_PDL=0 in the environment launches without it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+bool pdl_enabled();
+void set_pdl_attr(cudaLaunchAttribute& a);
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                     Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  set_pdl_attr(attr[0]);
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // element count rounded up to a multiple of 8 (16-byte aligned offsets for 2- and 4-byte types)
 __host__ __device__ inline int64_t pad8(int64_t x) { return (x + 7) & ~(int64_t)7; }

@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(256)
 gather_cols_pipelined(const T* __restrict__ in, T* __restrict__ out, int64_t rows, int cols,
                       const int32_t* __restrict__ row_map, const int32_t* __restrict__ col_map,
                       int R) {
+  pdl_wait();
+  pdl_trigger();
   constexpr int VEC = 16 / sizeof(T);
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T* buf[2] = {reinterpret_cast<T*>(smem_raw),
@@ -220,8 +222,8 @@ cudaError_t launch_gather(const void* in, void* out, int64_t rows, int64_t cols,
                  s);
     auto launch = [&](auto kern) {
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      kern<<<(unsigned)grid, 256, smem, s>>>(static_cast<const T*>(in), static_cast<T*>(out),
-                                             rows, (int)cols, row_map, col_map, R);
+      launch_k(kern, dim3((unsigned)grid), dim3(256), smem, s, static_cast<const T*>(in),
+               static_cast<T*>(out), rows, (int)cols, row_map, col_map, R);
     };
     if (nvec <= 2 * 256) launch(gather_cols_pipelined<T, 2>);
     else if (nvec <= 4 * 256) launch(gather_cols_pipelined<T, 4>);
@@ -270,6 +272,8 @@ cudaError_t launch_scatter(const void* in, void* out, int64_t rows, int64_t cols
 
 __global__ void invert_kernel(const int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                               int64_t k) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < k;
        i += (int64_t)gridDim.x * blockDim.x)
     inv[perm[i]] = (int32_t)i;
@@ -354,8 +358,8 @@ cudaError_t scatter_cols(const void* in, void* out, int64_t rows, int64_t cols,
     const int grid = (int)std::min<int64_t>((cols + 255) / 256, 4096);
     {
       TraceScope t("perm_invert", s);
-      invert_kernel<<<grid, 256, 0, s>>>(col_map, inv_tmp, cols);
-      cudaError_t e = cudaGetLastError();
+      cudaError_t e = launch_k(invert_kernel, dim3(grid), dim3(256), 0, s, col_map, inv_tmp, cols);
+      if (e == cudaSuccess) e = cudaGetLastError();
       if (e != cudaSuccess) return e;
     }
     return gather_cols(in, out, rows, cols, nullptr, inv_tmp, elem_bytes, s, name);

@@ -407,6 +407,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_wait();      // operands and outputs may belong to the previous kernel of the stream
+  pdl_trigger();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -600,8 +602,17 @@ __device__ __forceinline__ void umma_commit_pair_both(uint32_t bar) {
       "h"(mask)
       : "memory");
 }
+// Arrive on a barrier of a CTA of the cluster, ordering this thread's earlier memory writes
+// before it (cluster scope: the consumer may read them from another CTA).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+               : "memory");
+}
+// The same arrive without ordering earlier memory operations: for an accumulator handed back
+// after tcgen05.wait::ld (its TMEM reads are complete), so the epilogue's global stores need not
+// be acknowledged before the MMA may reuse the accumulator.
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_bar) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
                : "memory");
 }
 
@@ -711,8 +722,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // B_I8: the producer's arrive plus one per converter warp of both CTAs
-      mbar_init(smem_u32(full + s), B_I8 ? 1 + 2 * (kPairConvThreads / 32) : 1);
+      // B_I8: the producer's arrive plus one per converter warp of a group, in both CTAs
+      mbar_init(smem_u32(full + s), B_I8 ? 1 + 2 * (kPairConvThreads / 64) : 1);
       mbar_init(smem_u32(empty + s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -722,7 +733,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     mbar_init(smem_u32(drain), 1);
     for (int r = 0; r < RAW; ++r) {
       mbar_init(smem_u32(qfull + r), 1);
-      mbar_init(smem_u32(qempty + r), kPairConvThreads / 32);
+      mbar_init(smem_u32(qempty + r), kPairConvThreads / 64);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -738,6 +749,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
   cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  pdl_wait();      // operands and outputs may belong to the previous kernel of the stream
+  pdl_trigger();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -868,13 +881,18 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
           tc.nb * 256);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_remote(leader_tempty0 + (uint32_t)(acc * 8));
+      if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty0 + (uint32_t)(acc * 8));
     }
   } else if constexpr (B_I8) {
     // ------------------------------------------------------------ int8 -> bf16 converters
-    // Thread ct owns one 8-element unit column of the staged tile and 8 of its 64 (B_MN) or
-    // 128 (K-major) lines: 8-byte conflict-free reads, 16-byte swizzled conflict-free writes.
-    const int ct = threadIdx.x - kThreads;
+    // Two groups of two warps take alternate K blocks, so two blocks are converted at a time
+    // and each group's staging slots (it % RAW has the group's parity) double-buffer its TMA
+    // loads. Thread gt of a group owns one 8-element unit column of the staged tile and 16 of
+    // its 64 (B_MN) or 128 (K-major) lines: 8-byte conflict-free reads, 16-byte swizzled
+    // conflict-free writes.
+    const int cw = warp - kThreads / 32;
+    const int grp = cw >> 1;
+    const int gt = (cw & 1) * 32 + lane;   // 0..63
     const uint32_t leader_full0 = map_to_rank(smem_u32(full), 0);
     int it = 0;
     bool ok = true;
@@ -884,8 +902,9 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
       const int bn = tc.g * p.b_gn + tc.nb * 256 + (int)rank * 128;
       float sc[8];
-      if constexpr (B_MN) load_scales8(p.b_scale + bn + 8 * (ct & 15), sc);   // per N column
+      if constexpr (B_MN) load_scales8(p.b_scale + bn + 8 * (gt & 15), sc);   // per N column
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        if ((it & 1) != grp) continue;
         const int s = it % STAGES, r = it % RAW;
         bool got = wait_bounded(smem_u32(qfull + r), (uint32_t)(it / RAW) & 1u, ctl, kErrConvert,
                                 kWaitLimitNs);
@@ -900,18 +919,19 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         if constexpr (B_MN) {
           // staged int8 tile: 64 K lines of 128 N bytes; bf16 stage: two 64-column chunks of
           // 64 K lines x 128 B, 16-byte unit u of line k at (u ^ (k & 7))
-          const int nu = ct & 15, k0 = ct >> 4;
-          uint8_t* d0 = dst + (nu >> 3) * (64 * BK * 2) + ((((nu & 7) ^ k0) << 4));
+          const int nu = gt & 15, k0 = gt >> 4;   // lines k0 + 4 j, j = 0..15
+          uint8_t* d0 = dst + (nu >> 3) * (64 * BK * 2);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int k = k0 + 8 * i;
+          for (int j = 0; j < 16; ++j) {
+            const int k = k0 + 4 * j;
             const uint2 w = *reinterpret_cast<const uint2*>(q + k * 128 + nu * 8);
-            *reinterpret_cast<uint4*>(d0 + k * 128) = dequant8(w, sc);
+            *reinterpret_cast<uint4*>(d0 + k * 128 + (((nu & 7) ^ (k & 7)) << 4)) =
+                dequant8(w, sc);
           }
         } else {
           // staged int8 tile: 128 N lines of 64 K bytes; bf16 stage: 128 lines x 128 B,
           // 16-byte unit u of line j at (u ^ (j & 7)); the scale runs along K
-          const int u = ct & 7, j0 = ct >> 3;
+          const int u = gt & 7, j0 = gt >> 3;     // lines j0 + 8 i, i = 0..15
           const int kq = kb * BK + 8 * u;   // K is a multiple of 8: a unit is all in or all out
           if (kq < p.K) {
             load_scales8(p.b_scale + tc.g * p.b_gk + kq, sc);
@@ -919,10 +939,10 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
 #pragma unroll
             for (int e = 0; e < 8; ++e) sc[e] = 0.f;
           }
-          uint8_t* d0 = dst + ((u ^ (j0 & 7)) << 4);
+          uint8_t* d0 = dst + ((u ^ (j0 & 7)) << 4);   // j & 7 == j0 & 7 for every i
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int j = j0 + 16 * i;
+          for (int i = 0; i < 16; ++i) {
+            const int j = j0 + 8 * i;
             const uint2 w = *reinterpret_cast<const uint2*>(q + j * 64 + u * 8);
             *reinterpret_cast<uint4*>(d0 + j * 128) = dequant8(w, sc);
           }
@@ -932,7 +952,9 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(qempty + r));
-          mbar_arrive_remote(leader_full0 + (uint32_t)(s * 8));
+          // the leader's own converters order their writes at CTA scope, the peer's at cluster
+          if (leader) mbar_arrive(smem_u32(full + s));
+          else mbar_arrive_remote(leader_full0 + (uint32_t)(s * 8));
         }
       }
     }
@@ -1050,7 +1072,8 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   if (e != cudaSuccess) return e;
   const int grid = std::min(p.total_tiles, sm_count());
   TraceScope t(name, s);
-  kern<<<grid, kThreads, smem, s>>>(ta, tb, p);
+  e = launch_k(kern, dim3(grid), dim3(kThreads), smem, s, ta, tb, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -1085,16 +1108,17 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  set_pdl_attr(attr[1]);
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 1;   // the occupancy query sees the cluster shape only
   static int max_clusters = 0;
   if (!max_clusters) {
     cfg.gridDim = dim3(2 * 74, 1, 1);
@@ -1102,6 +1126,7 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
         max_clusters <= 0)
       max_clusters = sm_count() / 2;
   }
+  cfg.numAttrs = 2;
   const int clusters = std::min(p.total_tiles, max_clusters);
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   TraceScope t(name, s);

@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "poetx_device_status": (I32, [V]),
         "poetx_trace_enable": (I32, [I32]),
         "poetx_trace_read": (I64, [ctypes.c_char_p, SZ]),
+        "poetx_trace_select": (I32, [ctypes.c_char_p]),
         "poetx_status_string": (ctypes.c_char_p, [I32]),
         "poetx_last_error_message": (ctypes.c_char_p, []),
         "poetx_abi_version": (I32, []),
@@ -91,7 +92,7 @@ EXPORTED = (
     "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
     "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
     "poetx_quantize_w0", "poetx_dequantize_w0", "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
-    "poetx_trace_enable", "poetx_trace_read", "poetx_status_string",
+    "poetx_trace_enable", "poetx_trace_read", "poetx_trace_select", "poetx_status_string",
     "poetx_last_error_message", "poetx_abi_version", "poetx_testing_gemm_bf16")
 
 
@@ -291,6 +292,11 @@ def device_status(stream=None) -> None:
 
 def trace_enable(on: bool = True) -> None:
     _check(lib.poetx_trace_enable(1 if on else 0))
+
+
+def trace_select(names=None) -> None:
+    """Record only the launches named in `names` (iterable of str); None records all."""
+    _check(lib.poetx_trace_select(None if not names else ",".join(names).encode()))
 
 
 def trace_read(maxlen: int = 1 << 20):

@@ -163,3 +163,10 @@ def test_quantize_argument_checks():
     assert d(None, 0x3000, 64, 64, 0x4000, None) == 1
     assert d(0x2000, 0x3000, 64, 64, 0x4008, None) == 3
     assert d(0x2000, 0x3000, 64, 0, 0x4000, None) == 0
+
+
+def test_trace_select_is_host_only_and_accepts_lists():
+    assert poetx.lib.poetx_trace_select(b"umma_dense_W0,umma_dense_W0T") == 0
+    assert poetx.lib.poetx_trace_select(b",,x,") == 0
+    assert poetx.lib.poetx_trace_select(None) == 0
+    assert poetx.lib.poetx_trace_select(b"") == 0
