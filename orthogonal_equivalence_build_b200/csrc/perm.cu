@@ -187,6 +187,95 @@ gather_cols_pipelined(const T* __restrict__ in, T* __restrict__ out, int64_t row
   asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
+// bf16 rows two at a time, interleaved in shared memory: word c holds element c of row r (low
+// half) and of row r + 1 (high half), so one random 32-bit shared-memory read yields the output
+// element of both rows. Random 2-byte reads cost about 3.6 bank wavefronts per warp instruction
+// (random banks); pairing halves the number of such instructions per element. The pair is read
+// from global memory into registers (16-byte loads) one pair ahead, interleaved with byte
+// permutes and written to shared memory; each thread owns up to VPT fixed 16-byte output
+// vectors of each row and keeps their source indices in registers for the whole launch.
+// Needs cols % 8 == 0, cols <= 65536, 16-byte aligned rows and index array.
+template <int VPT, int NT>
+__global__ void __launch_bounds__(NT)
+gather_cols_rowpair(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restrict__ out,
+                    int64_t rows, int cols, const int32_t* __restrict__ col_map) {
+  pdl_wait();
+  pdl_trigger();
+  extern __shared__ __align__(16) uint32_t pw[];   // cols words
+  const int nvec = cols / 8;
+  const int64_t npairs = (rows + 1) / 2;
+  int64_t pr = blockIdx.x;
+  if (pr >= npairs) return;
+  uint32_t ids[VPT][4];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int v = threadIdx.x + k * blockDim.x;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) ids[k][h] = 0;
+    if (v < nvec) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int4 t = __ldg(reinterpret_cast<const int4*>(col_map + v * 8) + h);
+        ids[k][2 * h] = (uint32_t)t.x | ((uint32_t)t.y << 16);
+        ids[k][2 * h + 1] = (uint32_t)t.z | ((uint32_t)t.w << 16);
+      }
+    }
+  }
+  uint4 ra[VPT], rb[VPT];
+  auto load = [&](int64_t p) {
+    const int64_t r0 = 2 * p;
+    const bool has1 = r0 + 1 < rows;
+    const uint4* s0 = reinterpret_cast<const uint4*>(in + r0 * cols);
+    const uint4* s1 = reinterpret_cast<const uint4*>(in + (r0 + 1) * cols);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int v = threadIdx.x + k * blockDim.x;
+      if (v < nvec) {
+        ra[k] = __ldcs(s0 + v);
+        rb[k] = has1 ? __ldcs(s1 + v) : make_uint4(0, 0, 0, 0);
+      }
+    }
+  };
+  load(pr);
+  for (; pr < npairs; pr += gridDim.x) {
+    __syncthreads();   // the previous pair's reads of pw are done
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int v = threadIdx.x + k * blockDim.x;
+      if (v < nvec) {
+        const uint4 a = ra[k], b = rb[k];
+        uint4* d = reinterpret_cast<uint4*>(pw + 8 * v);
+        d[0] = make_uint4(__byte_perm(a.x, b.x, 0x5410), __byte_perm(a.x, b.x, 0x7632),
+                          __byte_perm(a.y, b.y, 0x5410), __byte_perm(a.y, b.y, 0x7632));
+        d[1] = make_uint4(__byte_perm(a.z, b.z, 0x5410), __byte_perm(a.z, b.z, 0x7632),
+                          __byte_perm(a.w, b.w, 0x5410), __byte_perm(a.w, b.w, 0x7632));
+      }
+    }
+    __syncthreads();
+    const int64_t nxt = pr + gridDim.x;
+    if (nxt < npairs) load(nxt);   // lands in registers while this pair is gathered
+    const int64_t r0 = 2 * pr;
+    const bool has1 = r0 + 1 < rows;
+    uint4* o0 = reinterpret_cast<uint4*>(out + r0 * cols);
+    uint4* o1 = reinterpret_cast<uint4*>(out + (r0 + 1) * cols);
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const int v = threadIdx.x + k * blockDim.x;
+      if (v < nvec) {
+        uint32_t x[4], y[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const uint32_t lo = pw[ids[k][h] & 0xFFFFu], hi = pw[ids[k][h] >> 16];
+          x[h] = __byte_perm(lo, hi, 0x5410);   // row r:     elements 2h, 2h + 1
+          y[h] = __byte_perm(lo, hi, 0x7632);   // row r + 1
+        }
+        __stcs(o0 + v, make_uint4(x[0], x[1], x[2], x[3]));
+        if (has1) __stcs(o1 + v, make_uint4(y[0], y[1], y[2], y[3]));
+      }
+    }
+  }
+}
+
 int num_sms() {
   static int sms = 0;
   if (!sms) {
@@ -210,6 +299,26 @@ cudaError_t launch_gather(const void* in, void* out, int64_t rows, int64_t cols,
   const size_t row_bytes = (size_t)cols * sizeof(T);
   constexpr int VEC = 16 / sizeof(T);
   const int64_t nvec = cols / VEC;
+  if (sizeof(T) == 2 && !row_map && row_bytes % 16 == 0 && cols <= 65536 && nvec <= 4 * 512 &&
+      aligned16p(in) && aligned16p(out) && aligned16p(col_map)) {
+    // token rows of a bf16 activation: row pairs interleaved in shared memory
+    const size_t smem = (size_t)cols * 4;
+    const int64_t npairs = (rows + 1) / 2;
+    TraceScope t(name ? name : "perm_gather_cols_bf16", s);
+    auto launch = [&](auto kern, int threads, int per_sm) {
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      per_sm = std::max(1, std::min(per_sm, (int)((200 * 1024) / smem)));
+      const int64_t grid = std::min<int64_t>(npairs, (int64_t)num_sms() * per_sm);
+      launch_k(kern, dim3((unsigned)grid), dim3(threads), smem, s,
+               static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows,
+               (int)cols, col_map);
+    };
+    // CTAs per SM as the registers allow (70 / 123 / 123 per thread)
+    if (nvec <= 2 * 256) launch(gather_cols_rowpair<2, 256>, 256, 3);
+    else if (nvec <= 4 * 256) launch(gather_cols_rowpair<4, 256>, 256, 2);
+    else launch(gather_cols_rowpair<4, 512>, 512, 1);
+    return cudaGetLastError();
+  }
   if (row_bytes % 16 == 0 && row_bytes <= 96 * 1024 && cols <= 65536 && nvec <= 8 * 256 &&
       aligned16p(in) && aligned16p(out) && aligned16p(col_map)) {
     // chunks of about 24 KB per buffer, two buffers per CTA

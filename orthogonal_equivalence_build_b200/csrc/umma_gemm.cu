@@ -677,8 +677,9 @@ __device__ __forceinline__ void load_scales8(const float* __restrict__ p, float 
 
 template <bool B_I8>
 struct PairCfg {
-  static constexpr int STAGES = B_I8 ? 5 : 6;
-  static constexpr int RAW = B_I8 ? 4 : 0;          // int8 staging slots
+  static constexpr int STAGES = B_I8 ? 4 : 6;
+  static constexpr int RAW = B_I8 ? 8 : 0;          // int8 staging slots
+  static constexpr int RAW_AHEAD = RAW - 2;         // int8 tiles in flight ahead of the A stream
   static constexpr int RAW_BYTES = 128 * BK;        // this CTA's 128 B rows (or columns) x 64
   static constexpr int THREADS = kThreads + (B_I8 ? kPairConvThreads : 0);
   static constexpr size_t SMEM = (size_t)STAGES * (128 * BK * 2 * 2) + (size_t)RAW * RAW_BYTES +
@@ -756,6 +757,29 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     if (lane == 0) {
       int it = 0;
       bool ok = true;
+      // int8 B: its own stream of staged tiles, RAW_AHEAD K blocks ahead of the A stream (one
+      // split, so every tile of this cluster has the same nk K blocks)
+      const int nk = (p.K + BK - 1) / BK;
+      const int my_tiles =
+          cluster_id < p.total_tiles ? (p.total_tiles - cluster_id + num_clusters - 1) / num_clusters
+                                     : 0;
+      const int total_it = B_I8 ? my_tiles * nk : 0;
+      int rit = 0;
+      constexpr int RAWD = RAW > 0 ? RAW : 1;   // (the bf16 instantiation never calls this)
+      auto issue_raw = [&](int j) -> bool {
+        const int r = j % RAWD;
+        if (!wait_bounded(smem_u32(qempty + r), ((uint32_t)(j / RAWD) & 1u) ^ 1u, ctl,
+                          kErrProducer, kWaitLimitNs))
+          return false;
+        const TileCoord tj = decode_pair_tile(p, cluster_id + (j / nk) * num_clusters);
+        const int bnj = tj.g * p.b_gn + tj.nb * 256 + (int)rank * 128, bkj = tj.g * p.b_gk;
+        const int kj = (j % nk) * BK;
+        const uint32_t qb = smem_u32(qfull + r);
+        mbar_expect_tx(qb, Cfg::RAW_BYTES);
+        if constexpr (B_MN) tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bnj, bkj + kj);
+        else tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bkj + kj, bnj);
+        return true;
+      };
       for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
         const TileCoord tc = decode_pair_tile(p, tile);
         const int kb0 = tc.split * p.kblocks_per_split;
@@ -765,17 +789,16 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if constexpr (B_I8) {
+            while (ok && rit < total_it && rit <= it + Cfg::RAW_AHEAD) {
+              ok = issue_raw(rit);
+              if (ok) ++rit;
+            }
+            if (!ok) break;
+          }
           if (!wait_bounded(smem_u32(empty + s), ph ^ 1u, ctl, kErrProducer, kWaitLimitNs)) {
             ok = false;
             break;
-          }
-          if constexpr (B_I8) {
-            const int r = it % RAW;
-            if (!wait_bounded(smem_u32(qempty + r), ((uint32_t)(it / RAW) & 1u) ^ 1u, ctl,
-                              kErrProducer, kWaitLimitNs)) {
-              ok = false;
-              break;
-            }
           }
           const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
           if (leader)
@@ -790,12 +813,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx, am + kc.ady);
           }
           if constexpr (B_I8) {
-            // int8 tile into this CTA's staging slot, completing its own local barrier
-            const int r = it % RAW;
-            const uint32_t qb = smem_u32(qfull + r);
-            mbar_expect_tx(qb, Cfg::RAW_BYTES);
-            if constexpr (B_MN) tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bn, bk + k);
-            else tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bk + k, bn);
+            // the int8 tile of this K block was issued by issue_raw
           } else if constexpr (B_MN) {
             tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx, bk + k + kc.bdy);
             tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
@@ -812,7 +830,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
                          kDrainLimitNs);
         if constexpr (B_I8)
-          for (int j = max(0, it - RAW); j < it; ++j)
+          for (int j = max(0, rit - RAW); j < rit; ++j)
             wait_bounded(smem_u32(qfull + j % RAW), (uint32_t)(j / RAW) & 1u, ctl, 0,
                          kDrainLimitNs);
       }
@@ -1197,6 +1215,7 @@ bool pair_supported(const Gemm& g) {
     Gemm h = g;
     h.b_i8 = false;
     return supported(h) && g.N % 256 == 0 && g.M >= 256 && g.groups == 1 && g.splits == 1 &&
+           g.nseg == 1 && g.epi.mode == kEpiStore &&
            !g.a_mn && !g.out_f32 && g.b_scale && g.b_ld % 16 == 0 && g.b_cols % 16 == 0 &&
            (reinterpret_cast<uintptr_t>(g.b_scale) & 15) == 0;
   }
