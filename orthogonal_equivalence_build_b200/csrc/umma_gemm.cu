@@ -558,6 +558,9 @@ struct PairParams {
   void* C;
   long long ldc, c_gs, c_split;
   const float* b_scale;   // int8 B only: one scale per column of the stored B tensor
+  int raster, band;       // tile order within a group: 0 = bands of `band` pair-rows, N inner;
+                          // 1 = bands of `band` pair-columns, N fastest inside a band
+  int hint;               // L2 policy of the loads: 0 none; 1 A kept, B streamed; 2 the reverse
   Epi epi;
   int* err;
 };
@@ -583,6 +586,35 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar)
       : "memory");
+}
+// The same load with an L2 cache policy (createpolicy): evict-last for the operand a raster
+// band reuses, evict-first for the one it streams.
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map,
+                                                      uint32_t leader_bar, int c0, int c1,
+                                                      uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar, int c0, int c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
 }
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                uint32_t idesc, uint32_t accumulate) {
@@ -623,8 +655,11 @@ __device__ __forceinline__ constexpr uint32_t instr_desc_pair() {
          ((B_MN ? 1u : 0u) << 16) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
 }
 
+// Tile order (L2 reuse): raster 0 sweeps all N tiles of a band of `band` pair-rows (the band's
+// A rows stay in L2 while B streams); raster 1 sweeps all M tiles of a band of `band`
+// pair-columns with the band's columns innermost (the band's B stays in L2 while each A row
+// tile is shared by the columns of the band at once).
 __device__ __forceinline__ TileCoord decode_pair_tile(const PairParams& p, int tile) {
-  constexpr int GROUP_M = 8;   // bands of 8 pair-rows (2048 rows)
   const int per_group = p.tiles_m * p.tiles_n;
   const int per_split = per_group * p.groups;
   TileCoord t;
@@ -632,12 +667,21 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const PairParams& p, int t
   const int r = tile - t.split * per_split;
   t.g = r / per_group;
   const int local = r - t.g * per_group;
-  const int band = local / (GROUP_M * p.tiles_n);
-  const int first_m = band * GROUP_M;
-  const int gm = min(GROUP_M, p.tiles_m - first_m);
-  const int within = local - band * GROUP_M * p.tiles_n;
-  t.mb = first_m + within % gm;
-  t.nb = within / gm;
+  if (p.raster == 0) {
+    const int band = local / (p.band * p.tiles_n);
+    const int first_m = band * p.band;
+    const int gm = min(p.band, p.tiles_m - first_m);
+    const int within = local - band * p.band * p.tiles_n;
+    t.mb = first_m + within % gm;
+    t.nb = within / gm;
+  } else {
+    const int band = local / (p.band * p.tiles_m);
+    const int first_n = band * p.band;
+    const int gn = min(p.band, p.tiles_n - first_n);
+    const int within = local - band * p.band * p.tiles_m;
+    t.nb = first_n + within % gn;
+    t.mb = within / gn;
+  }
   return t;
 }
 
@@ -757,6 +801,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     if (lane == 0) {
       int it = 0;
       bool ok = true;
+      const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
       // int8 B: its own stream of staged tiles, RAW_AHEAD K blocks ahead of the A stream (one
       // split, so every tile of this cluster has the same nk K blocks)
       const int nk = (p.K + BK - 1) / BK;
@@ -765,19 +810,36 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                                      : 0;
       const int total_it = B_I8 ? my_tiles * nk : 0;
       int rit = 0;
+      // position of the int8 stream: K block rkb of the cluster's tile rtile, whose B coordinates
+      // are decoded once per tile (this thread issues every load; it must stay cheap per block)
+      int rtile = cluster_id, rkb = 0, rbn = 0, rbk = 0;
+      auto raw_tile = [&]() {
+        if (rtile < p.total_tiles) {
+          const TileCoord tj = decode_pair_tile(p, rtile);
+          rbn = tj.g * p.b_gn + tj.nb * 256 + (int)rank * 128;
+          rbk = tj.g * p.b_gk;
+        }
+      };
+      if constexpr (B_I8) raw_tile();
       constexpr int RAWD = RAW > 0 ? RAW : 1;   // (the bf16 instantiation never calls this)
       auto issue_raw = [&](int j) -> bool {
         const int r = j % RAWD;
         if (!wait_bounded(smem_u32(qempty + r), ((uint32_t)(j / RAWD) & 1u) ^ 1u, ctl,
                           kErrProducer, kWaitLimitNs))
           return false;
-        const TileCoord tj = decode_pair_tile(p, cluster_id + (j / nk) * num_clusters);
-        const int bnj = tj.g * p.b_gn + tj.nb * 256 + (int)rank * 128, bkj = tj.g * p.b_gk;
-        const int kj = (j % nk) * BK;
+        const int kj = rkb * BK;
         const uint32_t qb = smem_u32(qfull + r);
         mbar_expect_tx(qb, Cfg::RAW_BYTES);
-        if constexpr (B_MN) tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bnj, bkj + kj);
-        else tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, bkj + kj, bnj);
+        const uint64_t pol = p.hint == 2 ? pol_keep : pol_stream;
+        if constexpr (B_MN)
+          tma_load_2d_hint(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, rbn, rbk + kj, pol);
+        else
+          tma_load_2d_hint(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, rbk + kj, rbn, pol);
+        if (++rkb == nk) {
+          rkb = 0;
+          rtile += num_clusters;
+          raw_tile();
+        }
         return true;
       };
       for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
@@ -809,15 +871,30 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, am + kc.adx, ak + k + kc.ady);
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), &tma_a, fb,
                              am + 64 + kc.adx, ak + k + kc.ady);
+          } else if (p.hint) {
+            tma_load_2d_pair_hint(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx,
+                                  am + kc.ady, p.hint == 1 ? pol_keep : pol_stream);
           } else {
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx, am + kc.ady);
           }
           if constexpr (B_I8) {
             // the int8 tile of this K block was issued by issue_raw
           } else if constexpr (B_MN) {
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx, bk + k + kc.bdy);
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
-                             bn + 64 + kc.bdx, bk + k + kc.bdy);
+            if (p.hint) {
+              const uint64_t pol = p.hint == 1 ? pol_stream : pol_keep;
+              tma_load_2d_pair_hint(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx,
+                                    bk + k + kc.bdy, pol);
+              tma_load_2d_pair_hint(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
+                                    bn + 64 + kc.bdx, bk + k + kc.bdy, pol);
+            } else {
+              tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx,
+                               bk + k + kc.bdy);
+              tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
+                               bn + 64 + kc.bdx, bk + k + kc.bdy);
+            }
+          } else if (p.hint) {
+            tma_load_2d_pair_hint(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx,
+                                  bn + kc.bdy, p.hint == 1 ? pol_stream : pol_keep);
           } else {
             tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx, bn + kc.bdy);
           }
@@ -939,12 +1016,17 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
           // 64 K lines x 128 B, 16-byte unit u of line k at (u ^ (k & 7))
           const int nu = gt & 15, k0 = gt >> 4;   // lines k0 + 4 j, j = 0..15
           uint8_t* d0 = dst + (nu >> 3) * (64 * BK * 2);
+          // every staged read before any operand write (the compiler cannot tell the two
+          // shared-memory ranges apart, so interleaving them would serialise each unit)
+          uint2 w[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            w[j] = *reinterpret_cast<const uint2*>(q + (k0 + 4 * j) * 128 + nu * 8);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int k = k0 + 4 * j;
-            const uint2 w = *reinterpret_cast<const uint2*>(q + k * 128 + nu * 8);
             *reinterpret_cast<uint4*>(d0 + k * 128 + (((nu & 7) ^ (k & 7)) << 4)) =
-                dequant8(w, sc);
+                dequant8(w[j], sc);
           }
         } else {
           // staged int8 tile: 128 N lines of 64 K bytes; bf16 stage: 128 lines x 128 B,
@@ -958,12 +1040,13 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             for (int e = 0; e < 8; ++e) sc[e] = 0.f;
           }
           uint8_t* d0 = dst + ((u ^ (j0 & 7)) << 4);   // j & 7 == j0 & 7 for every i
+          uint2 w[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int j = j0 + 8 * i;
-            const uint2 w = *reinterpret_cast<const uint2*>(q + j * 64 + u * 8);
-            *reinterpret_cast<uint4*>(d0 + j * 128) = dequant8(w, sc);
-          }
+          for (int i = 0; i < 16; ++i)
+            w[i] = *reinterpret_cast<const uint2*>(q + (j0 + 8 * i) * 64 + u * 8);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            *reinterpret_cast<uint4*>(d0 + (j0 + 8 * i) * 128) = dequant8(w[i], sc);
         }
         // make the generic-proxy stores visible to the tensor core's reads, then publish
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1120,6 +1203,21 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   fill_segments(g, p);
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
   p.b_scale = g.b_scale;
+  // dense products: wide N keeps bands of 16 pair-rows (W0' swept T / 4096 times); narrow N
+  // with a long K (dA' = dB W0'^T) sweeps M under bands of 8 pair-columns
+  p.raster = 0;
+  p.band = 8;
+  p.hint = 0;
+  if (p.groups == 1 && p.splits == 1) {
+    if (p.tiles_n <= 16 && p.tiles_m >= 32 && g.K >= 8192) {
+      p.raster = 1;   // the band's B columns are reused by every row tile: keep them in L2
+      p.band = 8;
+      p.hint = 2;
+    } else {
+      p.band = 16;    // the band's A rows are reused by every column tile: keep them in L2
+      p.hint = 1;
+    }
+  }
   p.epi = g.epi;
   p.err = device_error_word();
   auto kern = umma_gemm_pair_kernel<A_MN, B_MN, OUT_F32, B_I8>;
