@@ -292,7 +292,8 @@ def run_ours(args):
             poetx.quantize_w0(w0m, wq, scale)
             w0m = wq
         L = poetx.PoetxLinear(w0m, pr, pp, torch.from_numpy(p["q_r"]).to(dev),
-                              torch.from_numpy(p["q_p"]).to(dev), b, w0m_scale=scale)
+                              torch.from_numpy(p["q_p"]).to(dev), b, w0m_scale=scale,
+                              staged=args.xq_staged)
         d = {"lin": lin, "layer": L,
              "x_host": torch.from_numpy(a["X"]).to(dt).pin_memory(),
              "dy_host": torch.from_numpy(a["dY"]).to(dt).pin_memory()}
@@ -350,7 +351,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     # events only around the dominant kernel inside the timed region: an event between two
     # launches keeps the second from overlapping the first one's tail
-    w0_names = (("umma_dense_W0_i8", "umma_dense_W0T_i8") if args.xq
+    w0_names = (("umma_dense_W0_i8", "umma_dense_W0T_i8") if args.xq and not args.xq_staged
                 else ("umma_dense_W0", "umma_dense_W0T"))
     poetx.trace_read()
     poetx.trace_select(w0_names)
@@ -487,8 +488,10 @@ def run_ours(args):
         if nlin == 1:
             cfg.update({"m": layers[0]["lin"].m, "n": layers[0]["lin"].n})
         if args.xq:
-            cfg["w0m_storage"] = ("int8 codes + fp32 column scales, dequantised to bf16 in the "
-                                  "W0' GEMMs' shared-memory operand stages")
+            cfg["w0m_storage"] = (
+                "int8 codes + fp32 column scales, dequantised to bf16 "
+                + ("into the workspace once per W0' product (staged)" if args.xq_staged
+                   else "in the W0' GEMMs' shared-memory operand stages"))
         if wl.merge_every:
             cfg["merge_reinit"] = (f"every {wl.merge_every} steps: {merge_ms:.3f} ms for all "
                                    f"linears, amortised into ms_per_step")
@@ -534,7 +537,11 @@ def main(argv=None):
                     help="time only the first linear of a multi-linear workload")
     ap.add_argument("--xq", action="store_true",
                     help="store W0' in 8 bits (int8 + column scales) and time that layer")
+    ap.add_argument("--xq-staged", action="store_true",
+                    help="with --xq: dequantise W0' into the workspace once per product")
     args = ap.parse_args(argv)
+    if args.xq_staged:
+        args.xq = True
     if args.warmup < 3 and args.impl == "ours" and not os.environ.get("POETX_BENCH_ALLOW_SHORT"):
         args.warmup = 3
     if args.impl == "reference":

@@ -70,6 +70,11 @@ typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
  * other shapes dequantise into the workspace first). Requires dtype == POETX_BF16 and m, n
  * multiples of 16. */
 #define POETX_LAYER_W0M_I8 1
+/* With POETX_LAYER_W0M_I8: dequantise W0' into the workspace (m*n bf16) once per W0' product and
+ * run the bf16 product on it, instead of dequantising each tile inside the product. Results are
+ * bitwise the same; it needs 2*m*n more workspace bytes and is faster on this part, because
+ * the in-kernel conversion is repeated for every row tile of tokens. */
+#define POETX_LAYER_W0M_STAGED 2
 
 /* One POET-X linear. Every pointer is a device pointer owned by the caller. */
 typedef struct {
@@ -77,7 +82,7 @@ typedef struct {
   int64_t n;       /* out-features: columns of W0 */
   int64_t b;       /* block size; must divide m and n */
   int32_t dtype;   /* poetx_dtype of w0m, activations, saved_b, gradients and g_*_lp */
-  int32_t flags;   /* 0, or POETX_LAYER_W0M_I8 */
+  int32_t flags;   /* 0, POETX_LAYER_W0M_I8, or POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED */
   void* w0m;       /* [m, n] merged weight W0' (see poetx_merge_permutations); int8 codes
                       when flags has POETX_LAYER_W0M_I8 */
   int32_t* perm_r; /* [m] permutation of R */

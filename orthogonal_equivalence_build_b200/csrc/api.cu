@@ -156,9 +156,10 @@ poetx_status check_layer(const poetx_layer* L, bool need_lp) {
   if (!L) return fail(POETX_ERR_INVALID_ARG, "layer is NULL");
   if (L->dtype != POETX_F32 && L->dtype != POETX_BF16)
     return fail(POETX_ERR_DTYPE, "unknown layer dtype %d", L->dtype);
-  if (L->flags != 0 && L->flags != POETX_LAYER_W0M_I8)
+  if (L->flags != 0 && L->flags != POETX_LAYER_W0M_I8 &&
+      L->flags != (POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED))
     return fail(POETX_ERR_INVALID_ARG, "unknown layer flags %d", L->flags);
-  if (L->flags == POETX_LAYER_W0M_I8) {
+  if (L->flags & POETX_LAYER_W0M_I8) {
     if (L->dtype != POETX_BF16)
       return fail(POETX_ERR_DTYPE, "an int8 W0' needs a BF16 layer");
     if (!L->w0m_scale) return fail(POETX_ERR_INVALID_ARG, "int8 W0' without w0m_scale");
@@ -269,12 +270,14 @@ size_t merge_layout(const poetx_layer* L, void* base, MergeWs* o) {
 
 DT dt_of(int32_t d) { return d == POETX_BF16 ? DT::BF16 : DT::F32; }
 
-bool w0m_i8(const poetx_layer* L) { return L->flags == POETX_LAYER_W0M_I8; }
+bool w0m_i8(const poetx_layer* L) { return (L->flags & POETX_LAYER_W0M_I8) != 0; }
+bool w0m_staged(const poetx_layer* L) { return (L->flags & POETX_LAYER_W0M_STAGED) != 0; }
 
-// bf16 scratch for an explicit dequantisation of an int8 W0' when a product shape is not fused
+// bf16 scratch for an explicit dequantisation of an int8 W0': staged layers, and product shapes
+// the in-kernel dequantisation does not cover
 size_t xq_deq_bytes(const poetx_layer* L, int64_t T, bool fwd_product, bool bwd_product) {
   if (!w0m_i8(L)) return 0;
-  const bool need = (fwd_product && !dense_i8_fused(T, L->n)) ||
+  const bool need = w0m_staged(L) || (fwd_product && !dense_i8_fused(T, L->n)) ||
                     (bwd_product && !dense_i8_fused(T, L->m));
   return need ? (size_t)(L->m * L->n) * 2 : 0;
 }
@@ -283,6 +286,14 @@ size_t xq_deq_bytes(const poetx_layer* L, int64_t T, bool fwd_product, bool bwd_
 cudaError_t w0_product(const poetx_layer* L, const void* A, void* C, int64_t T, bool trans,
                        void* deq_ws, cudaStream_t s) {
   const int64_t N = trans ? L->m : L->n, K = trans ? L->n : L->m;
+  if (w0m_i8(L) && w0m_staged(L)) {
+    if (!deq_ws) return cudaErrorInvalidValue;
+    auto* W = static_cast<__nv_bfloat16*>(deq_ws);
+    cudaError_t e = dequantize_cols_i8(static_cast<const int8_t*>(L->w0m), L->w0m_scale, L->m,
+                                       L->n, W, s);
+    if (e != cudaSuccess) return e;
+    return gemm_dense(DT::BF16, A, W, C, T, N, K, trans, s);
+  }
   if (w0m_i8(L))
     return gemm_dense_i8(A, static_cast<const int8_t*>(L->w0m), L->w0m_scale, C, T, N, K, trans,
                          deq_ws, s);

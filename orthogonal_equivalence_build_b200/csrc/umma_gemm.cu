@@ -560,7 +560,6 @@ struct PairParams {
   const float* b_scale;   // int8 B only: one scale per column of the stored B tensor
   int raster, band;       // tile order within a group: 0 = bands of `band` pair-rows, N inner;
                           // 1 = bands of `band` pair-columns, N fastest inside a band
-  int hint;               // L2 policy of the loads: 0 none; 1 A kept, B streamed; 2 the reverse
   Epi epi;
   int* err;
 };
@@ -586,35 +585,6 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar)
       : "memory");
-}
-// The same load with an L2 cache policy (createpolicy): evict-last for the operand a raster
-// band reuses, evict-first for the one it streams.
-__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map,
-                                                      uint32_t leader_bar, int c0, int c1,
-                                                      uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(leader_bar), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map,
-                                                 uint32_t bar, int c0, int c1, uint64_t policy) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
-      : "memory");
-}
-__device__ __forceinline__ uint64_t policy_evict_last() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
-  return p;
-}
-__device__ __forceinline__ uint64_t policy_evict_first() {
-  uint64_t p;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
-  return p;
 }
 __device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                uint32_t idesc, uint32_t accumulate) {
@@ -801,7 +771,6 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     if (lane == 0) {
       int it = 0;
       bool ok = true;
-      const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
       // int8 B: its own stream of staged tiles, RAW_AHEAD K blocks ahead of the A stream (one
       // split, so every tile of this cluster has the same nk K blocks)
       const int nk = (p.K + BK - 1) / BK;
@@ -830,11 +799,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         const int kj = rkb * BK;
         const uint32_t qb = smem_u32(qfull + r);
         mbar_expect_tx(qb, Cfg::RAW_BYTES);
-        const uint64_t pol = p.hint == 2 ? pol_keep : pol_stream;
-        if constexpr (B_MN)
-          tma_load_2d_hint(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, rbn, rbk + kj, pol);
-        else
-          tma_load_2d_hint(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, rbk + kj, rbn, pol);
+        if constexpr (B_MN) tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, rbn, rbk + kj);
+        else tma_load_2d(smem_u32(sq + r * Cfg::RAW_BYTES), &tma_b, qb, rbk + kj, rbn);
         if (++rkb == nk) {
           rkb = 0;
           rtile += num_clusters;
@@ -871,30 +837,15 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, am + kc.adx, ak + k + kc.ady);
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), &tma_a, fb,
                              am + 64 + kc.adx, ak + k + kc.ady);
-          } else if (p.hint) {
-            tma_load_2d_pair_hint(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx,
-                                  am + kc.ady, p.hint == 1 ? pol_keep : pol_stream);
           } else {
             tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx, am + kc.ady);
           }
           if constexpr (B_I8) {
             // the int8 tile of this K block was issued by issue_raw
           } else if constexpr (B_MN) {
-            if (p.hint) {
-              const uint64_t pol = p.hint == 1 ? pol_stream : pol_keep;
-              tma_load_2d_pair_hint(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx,
-                                    bk + k + kc.bdy, pol);
-              tma_load_2d_pair_hint(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
-                                    bn + 64 + kc.bdx, bk + k + kc.bdy, pol);
-            } else {
-              tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx,
-                               bk + k + kc.bdy);
-              tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
-                               bn + 64 + kc.bdx, bk + k + kc.bdy);
-            }
-          } else if (p.hint) {
-            tma_load_2d_pair_hint(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx,
-                                  bn + kc.bdy, p.hint == 1 ? pol_stream : pol_keep);
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx, bk + k + kc.bdy);
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
+                             bn + 64 + kc.bdx, bk + k + kc.bdy);
           } else {
             tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx, bn + kc.bdy);
           }
@@ -1207,15 +1158,12 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   // with a long K (dA' = dB W0'^T) sweeps M under bands of 8 pair-columns
   p.raster = 0;
   p.band = 8;
-  p.hint = 0;
   if (p.groups == 1 && p.splits == 1) {
     if (p.tiles_n <= 16 && p.tiles_m >= 32 && g.K >= 8192) {
-      p.raster = 1;   // the band's B columns are reused by every row tile: keep them in L2
+      p.raster = 1;   // the band's B columns are shared by every row tile of the band
       p.band = 8;
-      p.hint = 2;
     } else {
-      p.band = 16;    // the band's A rows are reused by every column tile: keep them in L2
-      p.hint = 1;
+      p.band = 16;    // the band's A rows are shared by every column tile of the band
     }
   }
   p.epi = g.epi;

@@ -40,6 +40,7 @@ class Layer(ctypes.Structure):
 
 
 LAYER_W0M_I8 = 1
+LAYER_W0M_STAGED = 2
 
 
 def _load() -> ctypes.CDLL:
@@ -143,7 +144,7 @@ class PoetxLinear:
 
     def __init__(self, w0m: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,
                  q_r: torch.Tensor, q_p: torch.Tensor, b: int,
-                 w0m_scale: Optional[torch.Tensor] = None):
+                 w0m_scale: Optional[torch.Tensor] = None, staged: bool = False):
         m, n = w0m.shape
         dev = w0m.device
         self.b = int(b)
@@ -159,7 +160,7 @@ class PoetxLinear:
         self.g_r_lp = torch.empty(m // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
         self.g_p_lp = torch.empty(n // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
         self.desc = Layer(m=m, n=n, b=self.b, dtype=BF16 if i8 else dtype_code(w0m.dtype),
-                          flags=LAYER_W0M_I8 if i8 else 0,
+                          flags=(LAYER_W0M_I8 | (LAYER_W0M_STAGED if staged else 0)) if i8 else 0,
                           w0m=_ptr(w0m), perm_r=_ptr(perm_r), perm_p=_ptr(perm_p),
                           q_r=_ptr(q_r), q_p=_ptr(q_p), g_r=_ptr(self.g_r), g_p=_ptr(self.g_p),
                           g_r_lp=_ptr(self.g_r_lp), g_p_lp=_ptr(self.g_p_lp),

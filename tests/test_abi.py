@@ -56,7 +56,8 @@ def _fwd(L, x=0x100000, T=128, y=0x200000, ws=None, wsb=0):
     (dict(g_r_lp=None), 1),                     # bf16 layer needs the bf16 copies
     (dict(perm_r=0x20004), 3),                  # misaligned
     (dict(b=2048, m=4096, n=4096), 2),          # b too large
-    (dict(flags=2), 1),                         # unknown flag
+    (dict(flags=2), 1),                         # staged without the int8 flag
+    (dict(flags=4), 1),                         # unknown flag
     (dict(flags=1, w0m_scale=0xA0000, dtype=poetx.F32), 4),   # int8 W0' needs a bf16 layer
     (dict(flags=1, w0m_scale=0xA0004), 3),      # misaligned scales
     (dict(flags=1, w0m_scale=0xA0000, m=520, n=1040, b=8), 2),  # int8 W0' rows of 16 bytes
@@ -150,6 +151,11 @@ def test_int8_w0_workspace_only_where_the_product_is_not_fused():
         assert 4096 * 14336 * 2 <= extra < 4096 * 14336 * 2 + 4096
     assert poetx.lib.poetx_merge_reinit_workspace_bytes(ctypes.byref(L8)) == \
         poetx.lib.poetx_merge_reinit_workspace_bytes(ctypes.byref(L16))
+    # staged dequantisation always takes the bf16 copy of W0'
+    L8s = _layer(m=4096, n=14336, b=512, flags=3, w0m_scale=0xA0000)
+    for fn in (poetx.lib.poetx_fwd_workspace_bytes, poetx.lib.poetx_bwd_workspace_bytes):
+        extra = fn(ctypes.byref(L8s), 4096) - fn(ctypes.byref(L16), 4096)
+        assert 4096 * 14336 * 2 <= extra < 4096 * 14336 * 2 + 4096
 
 
 def test_quantize_argument_checks():

@@ -105,6 +105,21 @@ def test_xq_layer_bitwise_equals_bf16_layer_on_dequantised_weight(key, m, n, b, 
         assert torch.equal(a, r), name
 
 
+@pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 3584, 512, 1100),
+                                         ("llama1p3b_attn", 512, 640, 128, 300)])
+def test_staged_dequantisation_is_bitwise_the_in_kernel_one(key, m, n, b, T):
+    x = XqCase(key, m=m, n=n, b=b, tokens=T)
+    c = x.c
+    staged = poetx.PoetxLinear(x.wq, c.perm_r, c.perm_p, c.q_r, c.q_p, c.b, w0m_scale=x.scale,
+                               staged=True)
+    poetx.layer_cnp_build(staged)
+    a = x.run(x.xq)
+    s = x.run(staged)
+    torch.cuda.synchronize()
+    for name, u, v in zip(("y", "B", "dx", "dq_r", "dq_p"), a, s):
+        assert torch.equal(u, v), name
+
+
 def test_xq_backward_without_saved_b_is_identical():
     x = XqCase("llama8b_up_proj", m=1024, n=2048, b=512, tokens=600)
     a = x.run(x.xq)
