@@ -226,52 +226,49 @@ __device__ __forceinline__ TileCoord decode_tile(const Params& p, int tile) {
 // column; off0: element offset of the warp's first row in C at the tile's first column.
 constexpr int kEpiStageBytes = 8192;
 
-__device__ __forceinline__ void st4h(__nv_bfloat16* p, const float (&v)[4]) {
-  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]));
+// Elementwise step after a grouped b x b product at (g; i, j..j+7): acc = the eight sums, q = Q.
+// off = g*b*b + i*b + j (elements), bb = b*b.
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+  return make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                    pack_bf16x2(v[6], v[7]));
 }
-// hi = bf16(x), lo = bf16(x - hi): x = hi + lo to about 16 significant bits
-__device__ __forceinline__ void st4_split(__nv_bfloat16* hi, __nv_bfloat16* lo, const float (&x)[4]) {
-  float h[4], l[4];
+__device__ __forceinline__ void st8_split(__nv_bfloat16* hi, __nv_bfloat16* lo, const float (&x)[8]) {
+  float h[8], l[8];
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < 8; ++k) {
     h[k] = __bfloat162float(__float2bfloat16_rn(x[k]));
     l[k] = x[k] - h[k];
   }
-  st4h(hi, h);
-  st4h(lo, l);
+  *reinterpret_cast<uint4*>(hi) = pack8(h);
+  *reinterpret_cast<uint4*>(lo) = pack8(l);
 }
-
-__device__ __forceinline__ void unpack4h(uint2 u, float (&v)[4]) {
-  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
-  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
-  v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
-}
-
-// Elementwise step after a grouped b x b product at (g; i, j..j+3): acc = the four sums, q = Q.
-__device__ __forceinline__ void epi_apply(const Epi& e, int g, int i, int j, const float (&acc)[4],
-                                          const float (&q)[4]) {
-  const long long bb = (long long)e.b * e.b;
-  const long long off = (long long)g * bb + (long long)i * e.b + j;
+__device__ __forceinline__ void epi_apply8(const Epi& e, int g, int i, int j, long long off,
+                                           long long bb, const float (&acc)[8],
+                                           const float (&q)[8]) {
   if (e.mode == kEpiCnpS) {
-    float h[4];
+    float h[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) h[k] = (i == j + k ? 2.f : 0.f) + 2.f * q[k] + acc[k];
-    st4_split(e.o[0] + off, e.o[1] + off, acc);
-    st4_split(e.o[2] + off, e.o[3] + off, h);
+    for (int k = 0; k < 8; ++k) h[k] = (i == j + k ? 2.f : 0.f) + 2.f * q[k] + acc[k];
+    st8_split(e.o[0] + off, e.o[1] + off, acc);
+    st8_split(e.o[2] + off, e.o[3] + off, h);
   } else if (e.mode == kEpiCnpG) {
-    float v[4];
+    float v[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) v[k] = (i == j + k ? 1.f : 0.f) + 2.f * q[k] + acc[k];
+    for (int k = 0; k < 8; ++k) v[k] = (i == j + k ? 1.f : 0.f) + 2.f * q[k] + acc[k];
     const int run = g < e.nb0 ? 0 : 1;
-    const long long loc = (long long)(g - (run ? e.nb0 : 0)) * bb + (long long)i * e.b + j;
-    if (e.g[run]) *reinterpret_cast<float4*>(e.g[run] + loc) = make_float4(v[0], v[1], v[2], v[3]);
-    if (e.g_lp[run]) st4h(e.g_lp[run] + loc, v);
+    const long long loc = off - (run ? (long long)e.nb0 * bb : 0);
+    if (e.g[run]) {
+      float4* gp = reinterpret_cast<float4*>(e.g[run] + loc);
+      gp[0] = make_float4(v[0], v[1], v[2], v[3]);
+      gp[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    if (e.g_lp[run]) *reinterpret_cast<uint4*>(e.g_lp[run] + loc) = pack8(v);
   } else if (e.mode == kEpiDqS) {
-    float m[4];
+    float m[8];
 #pragma unroll
-    for (int k = 0; k < 4; ++k) m[k] = acc[k] - 2.f * q[k];
-    st4h(e.o[0] + off, acc);
-    st4h(e.o[1] + off, m);
+    for (int k = 0; k < 8; ++k) m[k] = acc[k] - 2.f * q[k];
+    *reinterpret_cast<uint4*>(e.o[0] + off) = pack8(acc);
+    *reinterpret_cast<uint4*>(e.o[1] + off) = pack8(m);
   }
 }
 
@@ -279,8 +276,7 @@ template <bool OUT_F32>
 __device__ __forceinline__ void epilogue_warp_rows(uint32_t tmem_row0, int ncols,
                                                    uint8_t* __restrict__ stage, void* C,
                                                    long long off0, long long ldc, int nlive,
-                                                   int lane, const Epi& epi, int g, int row0,
-                                                   int col0) {
+                                                   int lane) {
   constexpr int ESZ = OUT_F32 ? 4 : 2;
   constexpr int ROWB = 64 * ESZ;      // bytes of one row per 64-column chunk
   constexpr int V16 = ROWB / 16;      // 16-byte pieces per row chunk: 8 (bf16) or 16 (fp32)
@@ -312,48 +308,119 @@ __device__ __forceinline__ void epilogue_warp_rows(uint32_t tmem_row0, int ncols
       }
     }
     __syncwarp();
-    if (OUT_F32 && epi.mode != kEpiStore) {
-      // Q at this lane's 32 / RPI positions of the chunk: every load issued before any use
-      constexpr int NR = 32 / RPI;
-      const long long bb = (long long)epi.b * epi.b;
-      const long long qoff0 = (long long)g * bb + (long long)(row0 + rsub) * epi.b + col0 + c + sub * 4;
-      uint2 qh[NR], ql[NR];
 #pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        const int r = i * RPI + rsub;
-        const long long o = qoff0 + (long long)(i * RPI) * epi.b;
-        qh[i] = r < nlive ? __ldg(reinterpret_cast<const uint2*>(epi.qh + o)) : make_uint2(0, 0);
-        ql[i] = (r < nlive && epi.ql) ? __ldg(reinterpret_cast<const uint2*>(epi.ql + o))
-                                      : make_uint2(0, 0);
-      }
-#pragma unroll
-      for (int i = 0; i < NR; ++i) {
-        const int r = i * RPI + rsub;
-        if (r < nlive) {
-          const uint4 v =
-              *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
-          const float a[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z),
-                              __uint_as_float(v.w)};
-          float q[4], l[4];
-          unpack4h(qh[i], q);
-          unpack4h(ql[i], l);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) q[k] += l[k];
-          epi_apply(epi, g, row0 + r, col0 + c + sub * 4, a, q);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32 / RPI; ++i) {
-        const int r = i * RPI + rsub;
-        if (r < nlive) {
-          const uint4 v =
-              *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
-          *reinterpret_cast<uint4*>(Cb + (off0 + (long long)r * ldc + c) * ESZ + sub * 16) = v;
-        }
+    for (int i = 0; i < 32 / RPI; ++i) {
+      const int r = i * RPI + rsub;
+      if (r < nlive) {
+        const uint4 v =
+            *reinterpret_cast<const uint4*>(stage + r * ROWB + ((sub ^ (r & (V16 - 1))) * 16));
+        *reinterpret_cast<uint4*>(Cb + (off0 + (long long)r * ldc + c) * ESZ + sub * 16) = v;
       }
     }
     __syncwarp();
+  }
+}
+
+// bf16 epilogue through the tensor-memory accelerator: each 32-row x 64-column chunk of a warp is
+// packed into the 128-byte-swizzled layout of one half of the warp's 8 KB stage and written by
+// one bulk tensor store (rows beyond the tensor are clipped by the copy). The two halves
+// alternate, so a chunk is packed while the previous chunk's store still reads its half.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {   // at most N groups still reading shared
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {    // every group's writes complete
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void epilogue_tma_bf16(uint32_t tmem_row0, int ncols,
+                                                  uint8_t* __restrict__ stage,
+                                                  const CUtensorMap* map, int x0, int y0,
+                                                  int lane, int& chunk) {
+#pragma unroll 1
+  for (int c = 0; c < ncols; c += 64, ++chunk) {
+    uint8_t* half = stage + (chunk & 1) * 4096;
+    if (lane == 0) bulk_wait_read<1>();   // the store that last read this half is done reading
+    __syncwarp();
+    uint32_t r0[32], r1[32];
+    tmem_ld32(tmem_row0 + (uint32_t)c, r0);
+    tmem_ld32(tmem_row0 + (uint32_t)(c + 32), r1);
+    uint8_t* myrow = half + lane * 128;
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+      const uint32_t* src = v < 4 ? &r0[8 * v] : &r1[8 * (v - 4)];
+      *reinterpret_cast<uint4*>(myrow + ((v ^ (lane & 7)) * 16)) = make_uint4(
+          pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+          pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+          pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+          pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the copy
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(map, smem_u32(half), x0 + c, y0);
+      bulk_commit();
+    }
+  }
+}
+
+// Fused elementwise epilogue of a grouped b x b product (epilogue modes): lane = one accumulator
+// row, 32 columns per TMEM load. The Q values of a chunk (16-byte loads of the hi and lo parts)
+// are requested one chunk ahead; the caller requests chunk 0 (fused_q_load) before it waits for
+// the accumulator, so those loads overlap the main loop.
+struct FusedQ {
+  uint4 h[4], l[4];
+};
+__device__ __forceinline__ void fused_q_load(const Epi& e, long long roff, int c, bool live,
+                                             FusedQ& q) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    q.h[v] = live ? __ldg(reinterpret_cast<const uint4*>(e.qh + roff + c) + v) : make_uint4(0, 0, 0, 0);
+    q.l[v] = (live && e.ql) ? __ldg(reinterpret_cast<const uint4*>(e.ql + roff + c) + v)
+                            : make_uint4(0, 0, 0, 0);
+  }
+}
+__device__ __forceinline__ long long fused_row_offset(const Epi& e, int g, int row, int col0) {
+  return (long long)g * e.b * e.b + (long long)row * e.b + col0;
+}
+__device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols, const Epi& e, int g,
+                                               int row0, int col0, int nlive, int lane,
+                                               FusedQ& q) {
+  const long long bb = (long long)e.b * e.b;
+  const long long roff = fused_row_offset(e, g, row0 + lane, col0);
+  const bool live = lane < nlive;
+#pragma unroll 1
+  for (int cc = 0; cc < ncols; cc += 32) {
+    uint32_t r[32];
+    tmem_ld32(tmem_row0 + (uint32_t)cc, r);
+    if (live) {
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {   // eight columns cc + 8v .. cc + 8v + 7
+        float a[8], qq[8];
+        const uint32_t hw[4] = {q.h[v].x, q.h[v].y, q.h[v].z, q.h[v].w};
+        const uint32_t lw[4] = {q.l[v].x, q.l[v].y, q.l[v].z, q.l[v].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[k]);
+          const __nv_bfloat162 l2 = *reinterpret_cast<const __nv_bfloat162*>(&lw[k]);
+          qq[2 * k] = __low2float(h2) + __low2float(l2);
+          qq[2 * k + 1] = __high2float(h2) + __high2float(l2);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(r[8 * v + k]);
+        epi_apply8(e, g, row0 + lane, col0 + cc + 8 * v, roff + cc + 8 * v, bb, a, qq);
+      }
+    }
+    if (cc + 32 < ncols) fused_q_load(e, roff, cc + 32, live, q);
   }
 }
 
@@ -511,16 +578,22 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
       const TileCoord tc = decode_tile(p, tile);
       const int acc = tcount & 1;
       const uint32_t use = (uint32_t)(tcount >> 1);
-      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
-      tc_fence_after();
       const int row0 = tc.mb * BM + quarter * 32;   // first row of this warp
       const int nlive = max(0, min(32, p.M - row0));
+      const bool fused = OUT_F32 && p.epi.mode != kEpiStore;
+      FusedQ q0;
+      if (fused)
+        fused_q_load(p.epi, fused_row_offset(p.epi, tc.g, row0 + lane, tc.nb * BN), 0, lane < nlive, q0);
+      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
+      tc_fence_after();
       const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
                              (long long)row0 * p.ldc + (long long)tc.nb * BN;
-      epilogue_warp_rows<OUT_F32>(
-          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN), BN,
-          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane, p.epi, tc.g, row0,
-          tc.nb * BN);
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      if (fused)
+        epilogue_fused(trow, BN, p.epi, tc.g, row0, tc.nb * BN, nlive, lane, q0);
+      else
+        epilogue_warp_rows<OUT_F32>(trow, BN, sepi + (warp - 2) * kEpiStageBytes, p.C, off0,
+                                    p.ldc, nlive, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(tempty + acc));
@@ -689,22 +762,28 @@ __device__ __forceinline__ void load_scales8(const float* __restrict__ p, float 
   sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
 }
 
-template <bool B_I8>
+// EPI_W epilogue warps (4, or 8 = two per TMEM lane quarter, each taking half of the tile's
+// columns). Eight measured slower for the fp32-accumulator products (block gradients, the CNP /
+// dq blocks: 0.31 -> 0.33 ms and 83 -> 97 us), so every variant uses four.
+template <bool B_I8, bool OUT_F32>
 struct PairCfg {
+  static constexpr int EPI_W = 4;                   // epilogue warps
   static constexpr int STAGES = B_I8 ? 4 : 6;
   static constexpr int RAW = B_I8 ? 8 : 0;          // int8 staging slots
-  static constexpr int RAW_AHEAD = RAW - 2;         // int8 tiles in flight ahead of the A stream
+  static constexpr int RAW_AHEAD = RAW > 2 ? RAW - 2 : 0;  // int8 tiles in flight ahead of A
   static constexpr int RAW_BYTES = 128 * BK;        // this CTA's 128 B rows (or columns) x 64
-  static constexpr int THREADS = kThreads + (B_I8 ? kPairConvThreads : 0);
+  static constexpr int THREADS = 64 + 32 * EPI_W + (B_I8 ? kPairConvThreads : 0);
   static constexpr size_t SMEM = (size_t)STAGES * (128 * BK * 2 * 2) + (size_t)RAW * RAW_BYTES +
-                                 4 * kEpiStageBytes + 1024 + 256;
+                                 EPI_W * kEpiStageBytes + 1024 + 256;
 };
 
 template <bool A_MN, bool B_MN, bool OUT_F32, bool B_I8>
-__global__ void __launch_bounds__(PairCfg<B_I8>::THREADS, 1)
+__global__ void __launch_bounds__((PairCfg<B_I8, OUT_F32>::THREADS), 1)
 umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
-                      const __grid_constant__ CUtensorMap tma_b, const PairParams p) {
-  using Cfg = PairCfg<B_I8>;
+                      const __grid_constant__ CUtensorMap tma_b,
+                      const __grid_constant__ CUtensorMap tma_c, const PairParams p) {
+  using Cfg = PairCfg<B_I8, OUT_F32>;
+  constexpr int EPI_W = Cfg::EPI_W;
   constexpr int STAGES = Cfg::STAGES;
   constexpr int RAW = Cfg::RAW;
   constexpr int A_BYTES = 128 * BK * 2;  // this CTA's 128 rows of A, 16 KB
@@ -717,12 +796,12 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
   uint8_t* sa = smem;
   uint8_t* sb = smem + STAGES * A_BYTES;
   uint8_t* sq = sb + STAGES * B_BYTES;     // int8 staging (B_I8)
-  uint8_t* sepi = sq + RAW * Cfg::RAW_BYTES;   // 4 epilogue warps x 8 KB
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + 4 * kEpiStageBytes);
+  uint8_t* sepi = sq + RAW * Cfg::RAW_BYTES;   // EPI_W epilogue warps x 8 KB
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + EPI_W * kEpiStageBytes);
   uint64_t* full = bars;                   // used in the leader only
   uint64_t* empty = bars + STAGES;
   uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + 2;            // used in the leader only (8 arrivals)
+  uint64_t* tempty = tfull + 2;            // used in the leader only (2 * EPI_W arrivals)
   uint64_t* drain = tempty + 2;
   uint64_t* qfull = drain + 1;             // int8 staging slot loaded (local)
   uint64_t* qempty = qfull + RAW;          // int8 staging slot read by the converters (local)
@@ -743,7 +822,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(tfull + a), 1);
-      mbar_init(smem_u32(tempty + a), 8);
+      mbar_init(smem_u32(tempty + a), 2 * EPI_W);
     }
     mbar_init(smem_u32(drain), 1);
     for (int r = 0; r < RAW; ++r) {
@@ -907,27 +986,48 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       wait_bounded(smem_u32(drain), 0, ctl, ok ? kErrMma : 0, ok ? kWaitLimitNs : kDrainLimitNs);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 2 + EPI_W) {
+    // TMEM lanes 32 * (warp % 4) .. + 31; with eight warps, warps 6.. take the second half of
+    // the columns
     const int quarter = warp & 3;
+    constexpr int COLS = ACC_COLS / (EPI_W / 4);
+    const int cbase = ((warp - 2) / 4) * COLS;
     const uint32_t leader_tempty0 = map_to_rank(smem_u32(tempty), 0);
-    int tcount = 0;
+    int tcount = 0, chunk = 0;
     for (int tile = cluster_id; tile < p.total_tiles; tile += num_clusters, ++tcount) {
       const TileCoord tc = decode_pair_tile(p, tile);
       const int acc = tcount & 1;
       const uint32_t use = (uint32_t)(tcount >> 1);
-      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
-      tc_fence_after();
       const int row0 = tc.mb * 256 + (int)rank * 128 + quarter * 32;
       const int nlive = max(0, min(32, p.M - row0));
+      const bool fused = OUT_F32 && p.epi.mode != kEpiStore;
+      FusedQ q0;
+      const int col0 = tc.nb * 256 + cbase;
+      if (fused)
+        fused_q_load(p.epi, fused_row_offset(p.epi, tc.g, row0 + lane, col0), 0, lane < nlive,
+                     q0);
+      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
+      tc_fence_after();
       const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
-                             (long long)row0 * p.ldc + (long long)tc.nb * 256;
-      epilogue_warp_rows<OUT_F32>(
-          tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * ACC_COLS), ACC_COLS,
-          sepi + (warp - 2) * kEpiStageBytes, p.C, off0, p.ldc, nlive, lane, p.epi, tc.g, row0,
-          tc.nb * 256);
+                             (long long)row0 * p.ldc + (long long)col0;
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
+                            (uint32_t)(acc * ACC_COLS + cbase);
+      if (fused)
+        epilogue_fused(trow, COLS, p.epi, tc.g, row0, col0, nlive, lane, q0);
+      else if constexpr (!OUT_F32)
+        epilogue_tma_bf16(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, &tma_c,
+                          (int)(((long long)tc.g * p.c_gs) % p.ldc) + col0,
+                          (int)(((long long)tc.g * p.c_gs) / p.ldc) + row0, lane, chunk);
+      else
+        epilogue_warp_rows<OUT_F32>(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, p.C, off0,
+                                    p.ldc, nlive, lane);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty0 + (uint32_t)(acc * 8));
+    }
+    if constexpr (!OUT_F32) {
+      if (lane == 0) bulk_wait_all();   // every store written before the CTA leaves
+      __syncwarp();
     }
   } else if constexpr (B_I8) {
     // ------------------------------------------------------------ int8 -> bf16 converters
@@ -936,7 +1036,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     // loads. Thread gt of a group owns one 8-element unit column of the staged tile and 16 of
     // its 64 (B_MN) or 128 (K-major) lines: 8-byte conflict-free reads, 16-byte swizzled
     // conflict-free writes.
-    const int cw = warp - kThreads / 32;
+    const int cw = warp - (2 + EPI_W);
     const int grp = cw >> 1;
     const int gt = (cw & 1) * 32 + lane;   // 0..63
     const uint32_t leader_full0 = map_to_rank(smem_u32(full), 0);
@@ -952,6 +1052,17 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         if ((it & 1) != grp) continue;
         const int s = it % STAGES, r = it % RAW;
+        if constexpr (!B_MN) {
+          // scales along K for this block, requested before the waits so that their latency
+          // overlaps them (K is a multiple of 8: a unit of 8 is all inside or all outside)
+          const int kq = kb * BK + 8 * (gt & 7);
+          if (kq < p.K) {
+            load_scales8(p.b_scale + tc.g * p.b_gk + kq, sc);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sc[e] = 0.f;
+          }
+        }
         bool got = wait_bounded(smem_u32(qfull + r), (uint32_t)(it / RAW) & 1u, ctl, kErrConvert,
                                 kWaitLimitNs);
         got = got && wait_bounded(smem_u32(empty + s), ((uint32_t)(it / STAGES) & 1u) ^ 1u, ctl,
@@ -983,13 +1094,6 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
           // staged int8 tile: 128 N lines of 64 K bytes; bf16 stage: 128 lines x 128 B,
           // 16-byte unit u of line j at (u ^ (j & 7)); the scale runs along K
           const int u = gt & 7, j0 = gt >> 3;     // lines j0 + 8 i, i = 0..15
-          const int kq = kb * BK + 8 * u;   // K is a multiple of 8: a unit is all in or all out
-          if (kq < p.K) {
-            load_scales8(p.b_scale + tc.g * p.b_gk + kq, sc);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) sc[e] = 0.f;
-          }
           uint8_t* d0 = dst + ((u ^ (j0 & 7)) << 4);   // j & 7 == j0 & 7 for every i
           uint2 w[16];
 #pragma unroll
@@ -1131,7 +1235,7 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
 
 template <bool A_MN, bool B_MN, bool OUT_F32, bool B_I8>
 cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
-  using Cfg = PairCfg<B_I8>;
+  using Cfg = PairCfg<B_I8, OUT_F32>;
   constexpr size_t smem = Cfg::SMEM;
   CUtensorMap ta, tb;
   if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : 128)) return cudaErrorInvalidValue;
@@ -1141,6 +1245,15 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
       return cudaErrorInvalidValue;
   } else {
     if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
+  }
+  // bf16 output through TMA stores: C as a 2-D [M][ldc] tensor, 64 x 32 boxes, 128-byte swizzle
+  CUtensorMap tc = ta;   // fp32 outputs keep the thread stores; the map is then unused
+  if constexpr (!OUT_F32) {
+    // a group offset c_gs is a column offset (< ldc) or whole rows (a multiple of ldc)
+    if (g.c_gs % g.ldc != 0 && g.c_gs >= g.ldc) return cudaErrorNotSupported;
+    const int64_t extent = (g.groups - 1) * g.c_gs + g.M * g.ldc;
+    const int64_t rows = (extent + g.ldc - 1) / g.ldc;
+    if (!make_map(&tc, g.C, rows, g.ldc, g.ldc, 32)) return cudaErrorInvalidValue;
   }
   PairParams p;
   p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = (int)g.groups;
@@ -1194,7 +1307,7 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   const int clusters = std::min(p.total_tiles, max_clusters);
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   TraceScope t(name, s);
-  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
