@@ -1,10 +1,17 @@
 // bf16 x bf16 -> fp32 GEMM on the 5th-generation tensor cores (tcgen05 / TMEM / TMA), sm_100a.
 //
-// One kernel serves every bf16 contraction of the layer: the W0' products (dense), the
+// Two kernels serve every bf16 contraction of the layer: the W0' products (dense), the
 // batch-wise block-diagonal products A_j G_j ("POET-X" blog §第三斧: each b x b block is one
-// batch element) and the per-block gradients dG_j = A_j^T B_j (contraction over tokens, split-K).
+// batch element), the per-block gradients dG_j = A_j^T B_j (contraction over tokens, split-K)
+// and the b x b products of the Cayley-Neumann blocks and their gradient:
+//   umma_gemm_kernel       one CTA per 128 x BN tile (used where the pair tiling does not fit);
+//   umma_gemm_pair_kernel  two-CTA clusters on 256 x 256 tiles (tcgen05.mma.cta_group::2), the
+//                          main path; variants: int8 B dequantised in shared memory (8-bit
+//                          W0'), fused elementwise epilogues (CNP / dq), bf16 outputs through TMA
+//                          bulk tensor stores, K segments, band rasters.
 //
-// Structure (persistent, warp-specialised, 192 threads, one CTA per SM):
+// Structure (persistent, warp-specialised, 192 threads (320 with the int8 converters), one CTA
+// per SM):
 //   warp 0      TMA producer: streams 128 x 64 A and BN x 64 B tiles into a STAGES-deep ring of
 //               128-byte-swizzled shared-memory stages (mbarrier complete_tx).
 //   warp 1      owns the TMEM allocation (2 x BN fp32 columns: two accumulators) and one lane
