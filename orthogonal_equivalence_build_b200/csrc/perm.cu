@@ -134,8 +134,11 @@ gather_cols_pipelined(const T* __restrict__ in, T* __restrict__ out, int64_t row
 #pragma unroll
       for (int h = 0; h < VEC / 4; ++h) {
         const int4 t = __ldg(reinterpret_cast<const int4*>(col_map + v * VEC) + h);
-        ids[k][2 * h] = (uint32_t)t.x | ((uint32_t)t.y << 16);
-        ids[k][2 * h + 1] = (uint32_t)t.z | ((uint32_t)t.w << 16);
+        // clamped into the row: a map that is not a permutation gives wrong columns, never an
+        // access outside the staged row
+        const uint32_t cm = (uint32_t)cols - 1u;
+        ids[k][2 * h] = min((uint32_t)t.x, cm) | (min((uint32_t)t.y, cm) << 16);
+        ids[k][2 * h + 1] = min((uint32_t)t.z, cm) | (min((uint32_t)t.w, cm) << 16);
       }
     }
   }
@@ -188,14 +191,19 @@ gather_cols_pipelined(const T* __restrict__ in, T* __restrict__ out, int64_t row
 }
 
 // bf16 rows two at a time, interleaved in shared memory: word c holds element c of row r (low
-// half) and of row r + 1 (high half), so one random 32-bit shared-memory read yields the output
-// element of both rows. Random 2-byte reads cost about 3.6 bank wavefronts per warp instruction
-// (random banks); pairing halves the number of such instructions per element. The pair is read
-// from global memory into registers (16-byte loads) one pair ahead, interleaved with byte
-// permutes and written to shared memory; each thread owns up to VPT fixed 16-byte output
-// vectors of each row and keeps their source indices in registers for the whole launch.
-// Needs cols % 8 == 0, cols <= 65536, 16-byte aligned rows and index array.
-template <int VPT, int NT>
+// half) and of row r + 1 (high half), so one random 32-bit shared-memory access moves the
+// element of both rows. Random 2-byte accesses cost about 3.6 bank wavefronts per warp
+// instruction (random banks); pairing halves the number of such instructions per element. The
+// pair is read from global memory into registers (16-byte loads) one pair ahead. Each thread
+// owns up to VPT fixed 16-byte vectors of each row and keeps their column indices in registers
+// for the whole launch.
+//   gather  (SCATTER = false): out[r, c] = in[r, col_map[c]]. The pair is written to shared
+//           memory in order; output vector v reads its eight source words at random.
+//   scatter (SCATTER = true):  out[r, col_map[c]] = in[r, c]. Input vector v writes its eight
+//           words at random positions; the output is read back in order. No inverse map needed.
+// Needs cols % 8 == 0, cols <= 65536, 16-byte aligned rows and index array; for the scatter,
+// col_map must be a permutation (an output column no input maps to is left unwritten).
+template <int VPT, int NT, bool SCATTER>
 __global__ void __launch_bounds__(NT)
 gather_cols_rowpair(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restrict__ out,
                     int64_t rows, int cols, const int32_t* __restrict__ col_map) {
@@ -215,9 +223,11 @@ gather_cols_rowpair(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restr
     if (v < nvec) {
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
+        // clamped into the row (as in gather_cols_pipelined)
         const int4 t = __ldg(reinterpret_cast<const int4*>(col_map + v * 8) + h);
-        ids[k][2 * h] = (uint32_t)t.x | ((uint32_t)t.y << 16);
-        ids[k][2 * h + 1] = (uint32_t)t.z | ((uint32_t)t.w << 16);
+        const uint32_t cm = (uint32_t)cols - 1u;
+        ids[k][2 * h] = min((uint32_t)t.x, cm) | (min((uint32_t)t.y, cm) << 16);
+        ids[k][2 * h + 1] = min((uint32_t)t.z, cm) | (min((uint32_t)t.w, cm) << 16);
       }
     }
   }
@@ -244,11 +254,22 @@ gather_cols_rowpair(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restr
       const int v = threadIdx.x + k * blockDim.x;
       if (v < nvec) {
         const uint4 a = ra[k], b = rb[k];
-        uint4* d = reinterpret_cast<uint4*>(pw + 8 * v);
-        d[0] = make_uint4(__byte_perm(a.x, b.x, 0x5410), __byte_perm(a.x, b.x, 0x7632),
-                          __byte_perm(a.y, b.y, 0x5410), __byte_perm(a.y, b.y, 0x7632));
-        d[1] = make_uint4(__byte_perm(a.z, b.z, 0x5410), __byte_perm(a.z, b.z, 0x7632),
-                          __byte_perm(a.w, b.w, 0x5410), __byte_perm(a.w, b.w, 0x7632));
+        // word e = element e of row r (low half) | element e of row r + 1 (high half)
+        const uint32_t w[8] = {__byte_perm(a.x, b.x, 0x5410), __byte_perm(a.x, b.x, 0x7632),
+                               __byte_perm(a.y, b.y, 0x5410), __byte_perm(a.y, b.y, 0x7632),
+                               __byte_perm(a.z, b.z, 0x5410), __byte_perm(a.z, b.z, 0x7632),
+                               __byte_perm(a.w, b.w, 0x5410), __byte_perm(a.w, b.w, 0x7632)};
+        if constexpr (SCATTER) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            pw[ids[k][h] & 0xFFFFu] = w[2 * h];
+            pw[ids[k][h] >> 16] = w[2 * h + 1];
+          }
+        } else {
+          uint4* d = reinterpret_cast<uint4*>(pw + 8 * v);
+          d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
     }
     __syncthreads();
@@ -263,11 +284,22 @@ gather_cols_rowpair(const __nv_bfloat16* __restrict__ in, __nv_bfloat16* __restr
       const int v = threadIdx.x + k * blockDim.x;
       if (v < nvec) {
         uint32_t x[4], y[4];
+        if constexpr (SCATTER) {
+          const uint4* d = reinterpret_cast<const uint4*>(pw + 8 * v);
+          const uint4 d0 = d[0], d1 = d[1];
+          const uint32_t w[8] = {d0.x, d0.y, d0.z, d0.w, d1.x, d1.y, d1.z, d1.w};
 #pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          const uint32_t lo = pw[ids[k][h] & 0xFFFFu], hi = pw[ids[k][h] >> 16];
-          x[h] = __byte_perm(lo, hi, 0x5410);   // row r:     elements 2h, 2h + 1
-          y[h] = __byte_perm(lo, hi, 0x7632);   // row r + 1
+          for (int h = 0; h < 4; ++h) {
+            x[h] = __byte_perm(w[2 * h], w[2 * h + 1], 0x5410);
+            y[h] = __byte_perm(w[2 * h], w[2 * h + 1], 0x7632);
+          }
+        } else {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const uint32_t lo = pw[ids[k][h] & 0xFFFFu], hi = pw[ids[k][h] >> 16];
+            x[h] = __byte_perm(lo, hi, 0x5410);   // row r:     elements 2h, 2h + 1
+            y[h] = __byte_perm(lo, hi, 0x7632);   // row r + 1
+          }
         }
         __stcs(o0 + v, make_uint4(x[0], x[1], x[2], x[3]));
         if (has1) __stcs(o1 + v, make_uint4(y[0], y[1], y[2], y[3]));
@@ -291,6 +323,33 @@ constexpr size_t kMaxRowSmem = 200 * 1024;
 
 bool aligned16p(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
+// token rows of a bf16 activation: row pairs interleaved in shared memory
+bool rowpair_ok(const void* in, const void* out, int64_t cols, const int32_t* col_map) {
+  return cols % 8 == 0 && cols <= 65536 && cols / 8 <= 4 * 512 && aligned16p(in) &&
+         aligned16p(out) && aligned16p(col_map);
+}
+
+template <bool SCATTER>
+cudaError_t launch_rowpair(const void* in, void* out, int64_t rows, int64_t cols,
+                           const int32_t* col_map, cudaStream_t s) {
+  if (rows == 0 || cols == 0) return cudaSuccess;
+  const size_t smem = (size_t)cols * 4;
+  const int64_t npairs = (rows + 1) / 2, nvec = cols / 8;
+  auto launch = [&](auto kern, int threads, int per_sm) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    per_sm = std::max(1, std::min(per_sm, (int)((200 * 1024) / smem)));
+    const int64_t grid = std::min<int64_t>(npairs, (int64_t)num_sms() * per_sm);
+    launch_k(kern, dim3((unsigned)grid), dim3(threads), smem, s,
+             static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows,
+             (int)cols, col_map);
+  };
+  // CTAs per SM as the registers allow
+  if (nvec <= 2 * 256) launch(gather_cols_rowpair<2, 256, SCATTER>, 256, 3);
+  else if (nvec <= 4 * 256) launch(gather_cols_rowpair<4, 256, SCATTER>, 256, 2);
+  else launch(gather_cols_rowpair<4, 512, SCATTER>, 512, 1);
+  return cudaGetLastError();
+}
+
 template <typename T>
 cudaError_t launch_gather(const void* in, void* out, int64_t rows, int64_t cols,
                           const int32_t* row_map, const int32_t* col_map, cudaStream_t s,
@@ -299,25 +358,9 @@ cudaError_t launch_gather(const void* in, void* out, int64_t rows, int64_t cols,
   const size_t row_bytes = (size_t)cols * sizeof(T);
   constexpr int VEC = 16 / sizeof(T);
   const int64_t nvec = cols / VEC;
-  if (sizeof(T) == 2 && !row_map && row_bytes % 16 == 0 && cols <= 65536 && nvec <= 4 * 512 &&
-      aligned16p(in) && aligned16p(out) && aligned16p(col_map)) {
-    // token rows of a bf16 activation: row pairs interleaved in shared memory
-    const size_t smem = (size_t)cols * 4;
-    const int64_t npairs = (rows + 1) / 2;
+  if (sizeof(T) == 2 && !row_map && rowpair_ok(in, out, cols, col_map)) {
     TraceScope t(name ? name : "perm_gather_cols_bf16", s);
-    auto launch = [&](auto kern, int threads, int per_sm) {
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      per_sm = std::max(1, std::min(per_sm, (int)((200 * 1024) / smem)));
-      const int64_t grid = std::min<int64_t>(npairs, (int64_t)num_sms() * per_sm);
-      launch_k(kern, dim3((unsigned)grid), dim3(threads), smem, s,
-               static_cast<const __nv_bfloat16*>(in), static_cast<__nv_bfloat16*>(out), rows,
-               (int)cols, col_map);
-    };
-    // CTAs per SM as the registers allow (70 / 123 / 123 per thread)
-    if (nvec <= 2 * 256) launch(gather_cols_rowpair<2, 256>, 256, 3);
-    else if (nvec <= 4 * 256) launch(gather_cols_rowpair<4, 256>, 256, 2);
-    else launch(gather_cols_rowpair<4, 512>, 512, 1);
-    return cudaGetLastError();
+    return launch_rowpair<false>(in, out, rows, cols, col_map, s);
   }
   if (row_bytes % 16 == 0 && row_bytes <= 96 * 1024 && cols <= 65536 && nvec <= 8 * 256 &&
       aligned16p(in) && aligned16p(out) && aligned16p(col_map)) {
@@ -462,6 +505,14 @@ cudaError_t scatter_cols(const void* in, void* out, int64_t rows, int64_t cols,
                          const int32_t* col_map, int elem_bytes, int32_t* inv_tmp,
                          cudaStream_t s, const char* name) {
   if (rows == 0 || cols == 0) return cudaSuccess;
+  if (elem_bytes == 2 && rowpair_ok(in, out, cols, col_map) && cols / 8 <= 2 * 256) {
+    // rows of up to 4096 bf16 (several CTAs per SM): the row-pair scatter, no inverse map.
+    // Wider rows run one CTA per SM, where the random writes consume the very registers that
+    // the next pair's loads fill, so those loads are no longer hidden (14336 columns: 56.5 us
+    // against 38.9 us for the gather at 4096 tokens); they take the inverse and the gather.
+    TraceScope t(name ? name : "perm_scatter_cols_bf16", s);
+    return launch_rowpair<true>(in, out, rows, cols, col_map, s);
+  }
   if (inv_tmp && aligned16p(inv_tmp) && ((size_t)cols * elem_bytes) % 16 == 0) {
     // out[r, p] = in[r, inverse(col_map)[p]]: the scatter as a pipelined gather
     const int grid = (int)std::min<int64_t>((cols + 255) / 256, 4096);

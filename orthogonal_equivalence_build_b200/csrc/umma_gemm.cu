@@ -380,41 +380,61 @@ __device__ __forceinline__ void epilogue_tma_bf16(uint32_t tmem_row0, int ncols,
   }
 }
 
-// Fused elementwise epilogue of a grouped b x b product (epilogue modes): lane = one accumulator
-// row, 32 columns per TMEM load. The Q values of a chunk (16-byte loads of the hi and lo parts)
-// are requested one chunk ahead; the caller requests chunk 0 (fused_q_load) before it waits for
-// the accumulator, so those loads overlap the main loop.
+// Fused elementwise epilogue of a grouped b x b product (epilogue modes). Each 32-column chunk of
+// the warp's 32 accumulator rows comes out of TMEM one row per lane, goes through one half of the
+// warp's shared-memory stage (16-byte units of row r at unit ^ (r & 7): conflict-free both ways)
+// and is read back four lanes per row, eight consecutive columns each, so that every Q load and
+// output store of a warp covers 8 rows x 64 (bf16) or 128 (fp32) contiguous bytes. Lane l takes
+// rows 8i + l/4 (i = 0..3) and columns 8 (l % 4) .. + 7 of the chunk. The Q values of a chunk
+// (16-byte loads of the hi and lo parts) are requested one chunk ahead; the caller requests
+// chunk 0 (fused_q_load) before it waits for the accumulator, so those loads overlap the main
+// loop.
 struct FusedQ {
   uint4 h[4], l[4];
 };
-__device__ __forceinline__ void fused_q_load(const Epi& e, long long roff, int c, bool live,
-                                             FusedQ& q) {
+__device__ __forceinline__ long long fused_base(const Epi& e, int g, int row0, int col0, int lane) {
+  return (long long)g * e.b * e.b + (long long)row0 * e.b + col0 + 8 * (lane & 3);
+}
+__device__ __forceinline__ void fused_q_load(const Epi& e, long long base, int c, int nlive,
+                                             int lane, FusedQ& q) {
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
-    q.h[v] = live ? __ldg(reinterpret_cast<const uint4*>(e.qh + roff + c) + v) : make_uint4(0, 0, 0, 0);
-    q.l[v] = (live && e.ql) ? __ldg(reinterpret_cast<const uint4*>(e.ql + roff + c) + v)
+  for (int i = 0; i < 4; ++i) {
+    const int rr = 8 * i + (lane >> 2);
+    const bool live = rr < nlive;
+    const long long off = base + (long long)rr * e.b + c;
+    q.h[i] = live ? __ldg(reinterpret_cast<const uint4*>(e.qh + off)) : make_uint4(0, 0, 0, 0);
+    q.l[i] = (live && e.ql) ? __ldg(reinterpret_cast<const uint4*>(e.ql + off))
                             : make_uint4(0, 0, 0, 0);
   }
 }
-__device__ __forceinline__ long long fused_row_offset(const Epi& e, int g, int row, int col0) {
-  return (long long)g * e.b * e.b + (long long)row * e.b + col0;
-}
-__device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols, const Epi& e, int g,
+__device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols,
+                                               uint8_t* __restrict__ stage, const Epi& e, int g,
                                                int row0, int col0, int nlive, int lane,
                                                FusedQ& q) {
   const long long bb = (long long)e.b * e.b;
-  const long long roff = fused_row_offset(e, g, row0 + lane, col0);
-  const bool live = lane < nlive;
+  const long long base = fused_base(e, g, row0, col0, lane);
+  const int cg = lane & 3;
 #pragma unroll 1
-  for (int cc = 0; cc < ncols; cc += 32) {
+  for (int cc = 0, half = 0; cc < ncols; cc += 32, half ^= 1) {
     uint32_t r[32];
     tmem_ld32(tmem_row0 + (uint32_t)cc, r);
-    if (live) {
+    uint8_t* buf = stage + half * 4096;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {   // eight columns cc + 8v .. cc + 8v + 7
-        float a[8], qq[8];
-        const uint32_t hw[4] = {q.h[v].x, q.h[v].y, q.h[v].z, q.h[v].w};
-        const uint32_t lw[4] = {q.l[v].x, q.l[v].y, q.l[v].z, q.l[v].w};
+    for (int u = 0; u < 8; ++u)
+      *reinterpret_cast<uint4*>(buf + lane * 128 + ((u ^ (lane & 7)) << 4)) =
+          make_uint4(r[4 * u], r[4 * u + 1], r[4 * u + 2], r[4 * u + 3]);
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int rr = 8 * i + (lane >> 2);
+      const uint8_t* row = buf + rr * 128;
+      const float4 a0 = *reinterpret_cast<const float4*>(row + (((2 * cg) ^ (rr & 7)) << 4));
+      const float4 a1 = *reinterpret_cast<const float4*>(row + (((2 * cg + 1) ^ (rr & 7)) << 4));
+      if (rr < nlive) {
+        const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        float qq[8];
+        const uint32_t hw[4] = {q.h[i].x, q.h[i].y, q.h[i].z, q.h[i].w};
+        const uint32_t lw[4] = {q.l[i].x, q.l[i].y, q.l[i].z, q.l[i].w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const __nv_bfloat162 h2 = *reinterpret_cast<const __nv_bfloat162*>(&hw[k]);
@@ -422,13 +442,13 @@ __device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols, co
           qq[2 * k] = __low2float(h2) + __low2float(l2);
           qq[2 * k + 1] = __high2float(h2) + __high2float(l2);
         }
-#pragma unroll
-        for (int k = 0; k < 8; ++k) a[k] = __uint_as_float(r[8 * v + k]);
-        epi_apply8(e, g, row0 + lane, col0 + cc + 8 * v, roff + cc + 8 * v, bb, a, qq);
+        epi_apply8(e, g, row0 + rr, col0 + cc + 8 * cg, base + (long long)rr * e.b + cc, bb, a,
+                   qq);
       }
     }
-    if (cc + 32 < ncols) fused_q_load(e, roff, cc + 32, live, q);
+    if (cc + 32 < ncols) fused_q_load(e, base, cc + 32, nlive, lane, q);
   }
+  __syncwarp();   // every lane's reads of the stage are done before it is written again
 }
 
 template <int BN, bool A_MN, bool B_MN, bool OUT_F32, int STAGES>
@@ -590,14 +610,15 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
       const bool fused = OUT_F32 && p.epi.mode != kEpiStore;
       FusedQ q0;
       if (fused)
-        fused_q_load(p.epi, fused_row_offset(p.epi, tc.g, row0 + lane, tc.nb * BN), 0, lane < nlive, q0);
+        fused_q_load(p.epi, fused_base(p.epi, tc.g, row0, tc.nb * BN, lane), 0, nlive, lane, q0);
       if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
       tc_fence_after();
       const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
                              (long long)row0 * p.ldc + (long long)tc.nb * BN;
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       if (fused)
-        epilogue_fused(trow, BN, p.epi, tc.g, row0, tc.nb * BN, nlive, lane, q0);
+        epilogue_fused(trow, BN, sepi + (warp - 2) * kEpiStageBytes, p.epi, tc.g, row0,
+                       tc.nb * BN, nlive, lane, q0);
       else
         epilogue_warp_rows<OUT_F32>(trow, BN, sepi + (warp - 2) * kEpiStageBytes, p.C, off0,
                                     p.ldc, nlive, lane);
@@ -1010,9 +1031,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       const bool fused = OUT_F32 && p.epi.mode != kEpiStore;
       FusedQ q0;
       const int col0 = tc.nb * 256 + cbase;
-      if (fused)
-        fused_q_load(p.epi, fused_row_offset(p.epi, tc.g, row0 + lane, col0), 0, lane < nlive,
-                     q0);
+      if (fused) fused_q_load(p.epi, fused_base(p.epi, tc.g, row0, col0, lane), 0, nlive, lane, q0);
       if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
       tc_fence_after();
       const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
@@ -1020,7 +1039,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                             (uint32_t)(acc * ACC_COLS + cbase);
       if (fused)
-        epilogue_fused(trow, COLS, p.epi, tc.g, row0, col0, nlive, lane, q0);
+        epilogue_fused(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, p.epi, tc.g, row0, col0,
+                       nlive, lane, q0);
       else if constexpr (!OUT_F32)
         epilogue_tma_bf16(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, &tma_c,
                           (int)(((long long)tc.g * p.c_gs) % p.ldc) + col0,

@@ -75,7 +75,8 @@ def test_validate_permutation():
                                        ("llama1p3b_attn", 512, 128, 333),
                                        ("llama1p3b_attn", 1024, 256, 130),
                                        ("llama1p3b_attn", 1024, 256, 777),
-                                       ("llama8b_up_proj", 1024, 512, 1100)])
+                                       ("llama8b_up_proj", 1024, 512, 1100),
+                                       ("llama8b_up_proj", 14336, 512, 97)])
 def test_identity_layer_is_bit_exact(key, m, b, T):
     """q = 0 and W0 = I: G = I exactly and every product is by 1.0 or 0.0, so Y == X and
     dX == dY bit for bit; this pins the gathers, scatters and operand layouts."""
@@ -87,8 +88,13 @@ def test_identity_layer_is_bit_exact(key, m, b, T):
     assert torch.equal(dx, c.dy)
 
 
-@pytest.mark.parametrize("key,m,b,T", [("tiny_fp32", 256, 64, 77), ("llama1p3b_attn", 512, 128, 260)])
+@pytest.mark.parametrize("key,m,b,T", [("tiny_fp32", 256, 64, 77), ("llama1p3b_attn", 512, 128, 260),
+                                       ("llama8b_up_proj", 8192, 512, 129)])
 def test_permutation_weight_is_bit_exact(key, m, b, T):
+    """W0 a permutation matrix with q = 0: Y is X with its columns moved, bit for bit. With the
+    identity cases above, bf16 rows of 512 to 14336 columns take every row-pair gather and
+    scatter configuration (256 threads x 2 vectors, 256 x 4, 512 x 4), odd token counts
+    included."""
     rng = np.random.default_rng(5)
     s = rng.permutation(m)
     w0 = np.zeros((m, m), dtype=np.float32)
