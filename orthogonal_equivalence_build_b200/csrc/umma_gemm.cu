@@ -766,28 +766,51 @@ constexpr int kPairConvThreads = 128;
 // float(q) for a signed byte q without a conversion instruction: q + 128 = byte ^ 0x80 placed in
 // the low mantissa bits of 2^23 (0x4B000000) is the float 2^23 + 128 + q; subtracting 2^23 + 128
 // is exact. Then the fp32 product with the column scale (round to nearest), as in the reference
-// definition bf16(fp32(q) * s).
-__device__ __forceinline__ float byte_to_float(uint32_t flipped_word, int byte) {
-  return __uint_as_float(__byte_perm(flipped_word, 0x4B000000u, 0x7540u | (uint32_t)byte)) -
-         8388736.0f;
+// definition bf16(fp32(q) * s). The subtraction and the product run on packed pairs
+// (add / mul .rn.f32x2: the IEEE fp32 operation on each lane, half the instructions).
+__device__ __forceinline__ uint64_t f32x2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(lo), "r"(hi));
+  return d;
 }
-__device__ __forceinline__ uint4 dequant8(uint2 w, const float (&sc)[8]) {
-  const uint32_t x0 = w.x ^ 0x80808080u, x1 = w.y ^ 0x80808080u;
-  float f[8];
+__device__ __forceinline__ uint64_t f32x2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint32_t f32x2_to_bf16x2(uint64_t v) {
+  uint32_t lo, hi;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(lo), "=r"(hi) : "l"(v));
+  return pack_bf16x2(__uint_as_float(lo), __uint_as_float(hi));
+}
+__device__ __forceinline__ uint32_t biased_byte(uint32_t flipped_word, int byte) {
+  return __byte_perm(flipped_word, 0x4B000000u, 0x7540u | (uint32_t)byte);   // 2^23 + 128 + q
+}
+// sc2[p]: the scales of elements 2p and 2p + 1, packed
+__device__ __forceinline__ uint4 dequant8(uint2 w, const uint64_t (&sc2)[4]) {
+  const uint32_t x[2] = {w.x ^ 0x80808080u, w.y ^ 0x80808080u};
+  const uint64_t bias = f32x2_pack(__float_as_uint(-8388736.0f), __float_as_uint(-8388736.0f));
+  uint32_t o[4];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[i] = __fmul_rn(byte_to_float(x0, i), sc[i]);
-    f[4 + i] = __fmul_rn(byte_to_float(x1, i), sc[4 + i]);
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t xw = x[p >> 1];
+    const int b0 = 2 * (p & 1);
+    const uint64_t q2 = f32x2_add(f32x2_pack(biased_byte(xw, b0), biased_byte(xw, b0 + 1)), bias);
+    o[p] = f32x2_to_bf16x2(f32x2_mul(q2, sc2[p]));
   }
-  return make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
-                    pack_bf16x2(f[6], f[7]));
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
-__device__ __forceinline__ void load_scales8(const float* __restrict__ p, float (&sc)[8]) {
-  const float4 a = __ldg(reinterpret_cast<const float4*>(p));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
-  sc[0] = a.x; sc[1] = a.y; sc[2] = a.z; sc[3] = a.w;
-  sc[4] = b.x; sc[5] = b.y; sc[6] = b.z; sc[7] = b.w;
+__device__ __forceinline__ void load_scales8(const float* __restrict__ p, uint64_t (&sc2)[4]) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+  sc2[0] = f32x2_pack(a.x, a.y); sc2[1] = f32x2_pack(a.z, a.w);
+  sc2[2] = f32x2_pack(b.x, b.y); sc2[3] = f32x2_pack(b.z, b.w);
 }
 
 // EPI_W epilogue warps (4, or 8 = two per TMEM lane quarter, each taking half of the tile's
@@ -1074,7 +1097,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       const int kb0 = tc.split * p.kblocks_per_split;
       const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
       const int bn = tc.g * p.b_gn + tc.nb * 256 + (int)rank * 128;
-      float sc[8];
+      uint64_t sc[4];
       if constexpr (B_MN) load_scales8(p.b_scale + bn + 8 * (gt & 15), sc);   // per N column
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         if ((it & 1) != grp) continue;
@@ -1087,7 +1110,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             load_scales8(p.b_scale + tc.g * p.b_gk + kq, sc);
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sc[e] = 0.f;
+            for (int e = 0; e < 4; ++e) sc[e] = 0ull;   // +0.0f pairs
           }
         }
         bool got = wait_bounded(smem_u32(qfull + r), (uint32_t)(it / RAW) & 1u, ctl, kErrConvert,
