@@ -76,10 +76,13 @@ def test_validate_permutation():
                                        ("llama1p3b_attn", 1024, 256, 130),
                                        ("llama1p3b_attn", 1024, 256, 777),
                                        ("llama8b_up_proj", 1024, 512, 1100),
-                                       ("llama8b_up_proj", 14336, 512, 97)])
+                                       ("llama8b_up_proj", 14336, 512, 97),
+                                       ("llama1p3b_attn", 2048, 256, 8191),
+                                       ("llama8b_up_proj", 4096, 512, 4099)])
 def test_identity_layer_is_bit_exact(key, m, b, T):
     """q = 0 and W0 = I: G = I exactly and every product is by 1.0 or 0.0, so Y == X and
-    dX == dY bit for bit; this pins the gathers, scatters and operand layouts."""
+    dX == dY bit for bit; this pins the gathers, scatters and operand layouts. The last two
+    cases run tens of row tiles per block product, with a ragged last row tile."""
     c = LayerCase(key, m=m, n=m, b=b, tokens=T, q_zero=True, w0=np.eye(m, dtype=np.float32))
     y, bsave = c.forward()
     dx, dq_r, dq_p = c.backward(bsave)
@@ -139,6 +142,7 @@ def test_fp32_layer_shapes(m, n, b, T):
     ("llama1p3b_attn", 512, 512, 128, 1),
     ("llama8b_up_proj", 1024, 2048, 512, 1000),
     ("llama1p3b_attn", 768, 512, 256, 2049),
+    ("llama8b_up_proj", 1024, 2048, 512, 2305),
 ])
 def test_bf16_layer_parity(key, m, n, b, T):
     _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), TOL_BF16)
