@@ -298,11 +298,36 @@ void three_pass(umma::Gemm& g, int64_t nb, int64_t b) {
   g.b_dy[0] = 0; g.b_dy[1] = nb * b; g.b_dy[2] = 0;
 }
 
+// These launches hold a few tens of b x b products (one wave or two), so their time is that of
+// the busiest SM: waves x (tile area + a fixed cost per tile), minimised over 256 x 256 CTA-pair
+// tiles (half the operand traffic per MMA) and 128 x 256 / 128 / 64 single-CTA tiles, ties to
+// the larger tile. The fixed cost is a 128 x 128 tile's worth for plain stores and a quarter of
+// that for the fused epilogues, whose per-element work spreads over more SMs with smaller
+// tiles (measured at b = 256 over 16 blocks and b = 512 over 20; b = 512 over 36 blocks keeps
+// the pairs).
 cudaError_t run_block_gemm(const umma::Gemm& g, cudaStream_t s) {
   if (!umma::supported(g)) return cudaErrorNotSupported;
-  // CTA pairs (256 x 256 tiles, half the operand traffic per MMA) for b a multiple of 256
-  if (umma::pair_supported(g)) return umma::gemm_pair(g, s);
-  return umma::gemm(g, s);
+  const int64_t sms = umma::sm_count();
+  const int64_t fixed = g.epi.mode == umma::kEpiStore ? 128 * 128 : 128 * 32;
+  int64_t best = -1;
+  int best_bn = 0;   // 0: CTA pairs
+  if (umma::pair_supported(g)) {
+    const int64_t tiles = g.groups * ((g.M + 255) / 256) * (g.N / 256);
+    best = (tiles + sms / 2 - 1) / (sms / 2) * (128 * 256 + fixed);
+  }
+  for (int bn : {256, 128, 64}) {
+    if (g.N % bn) continue;
+    const int64_t tiles = g.groups * ((g.M + 127) / 128) * (g.N / bn);
+    const int64_t cost = (tiles + sms - 1) / sms * (128 * bn + fixed);
+    if (best < 0 || cost < best) {
+      best = cost;
+      best_bn = bn;
+    }
+  }
+  if (best_bn == 0) return umma::gemm_pair(g, s);
+  umma::Gemm h = g;
+  h.bn = best_bn;
+  return umma::gemm(h, s);
 }
 
 #define POETX_TRY(x)                  \

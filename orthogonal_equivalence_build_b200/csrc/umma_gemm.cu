@@ -1225,16 +1225,6 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, i
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-int sm_count() {
-  static int n = 0;
-  if (!n) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
-  }
-  return n;
-}
 
 template <typename P>
 void fill_segments(const Gemm& g, P& p) {
@@ -1378,6 +1368,17 @@ cudaError_t dispatch_majors(const Gemm& g, cudaStream_t s) {
 
 }  // namespace
 
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
 int effective_splits(int64_t K, int64_t splits) {
   const int64_t kblocks = (K + BK - 1) / BK;
   const int64_t s = std::max<int64_t>(1, std::min<int64_t>(splits, kblocks));
@@ -1452,8 +1453,10 @@ cudaError_t gemm_pair(const Gemm& g, cudaStream_t s) {
 }
 
 cudaError_t gemm(const Gemm& g, cudaStream_t s) {
-  if (g.N % 256 == 0) return dispatch_majors<256>(g, s);
-  if (g.N % 128 == 0) return dispatch_majors<128>(g, s);
+  if (g.bn != 0 && g.bn != 64 && g.bn != 128 && g.bn != 256) return cudaErrorInvalidValue;
+  const int cap = g.bn ? g.bn : 256;
+  if (g.N % 256 == 0 && cap >= 256) return dispatch_majors<256>(g, s);
+  if (g.N % 128 == 0 && cap >= 128) return dispatch_majors<128>(g, s);
   return dispatch_majors<64>(g, s);
 }
 

@@ -54,6 +54,7 @@ struct Gemm {
   Epi epi;
   void* C = nullptr; bool out_f32 = false; int64_t ldc = 0, c_gs = 0, c_split = 0;
   const char* name = nullptr;
+  int bn = 0;   // single-CTA tile width (64, 128 or 256; N must be a multiple); 0: the widest
 };
 
 bool supported(const Gemm& g);
@@ -65,7 +66,9 @@ cudaError_t gemm_pair(const Gemm& g, cudaStream_t s);
 // Number of K ranges the kernel actually uses for `splits` requested ranges over K
 // (ranges of whole 64-wide K blocks, none empty).
 int effective_splits(int64_t K, int64_t splits);
+// The single-CTA kernel (128 x bn tiles).
 cudaError_t gemm(const Gemm& g, cudaStream_t s);
+int sm_count();
 
 }  // namespace umma
 }  // namespace poetx
