@@ -223,7 +223,8 @@ struct BwdWs {
   void* B;               // recomputed forward product when the caller did not keep it
   float* dG;             // [m/b + n/b][b][b]: the R blocks, then the P blocks
   void* chain;
-  void *part_r, *part_p;  // split-K partial sums of dG_R, dG_P
+  void *part_r, *part_p;  // split-K partial sums of dG_R, dG_P (separate launches)
+  void* part_rp;          // split-K partial sums of the one launch over both (same region)
   int32_t* inv;
   void* Wd;               // dequantised W0' (int8 layers whose product shapes are not fused)
 };
@@ -240,8 +241,13 @@ size_t bwd_layout(const poetx_layer* L, int64_t T, void* base, BwdWs* o) {
   w.dG = static_cast<float*>(a.take((size_t)((L->m + L->n) * L->b) * sizeof(float)));
   const DT t = L->dtype == POETX_BF16 ? DT::BF16 : DT::F32;
   w.chain = a.take(gemm_dq_ws_bytes(t, L->m / L->b + L->n / L->b, L->b));
-  w.part_r = a.take(block_grad_ws_bytes(t, L->m, L->b, T));
-  w.part_p = a.take(block_grad_ws_bytes(t, L->n, L->b, T));
+  const size_t pr = block_grad_ws_bytes(t, L->m, L->b, T);
+  const size_t pp = block_grad_ws_bytes(t, L->n, L->b, T);
+  const size_t prp = block_grad2_ws_bytes(t, L->m, L->n, L->b, T);
+  uint8_t* parts = static_cast<uint8_t*>(a.take(std::max(prp, pr + pp)));
+  w.part_r = parts;
+  w.part_p = parts ? parts + pr : nullptr;
+  w.part_rp = parts;
   w.inv = static_cast<int32_t*>(a.take(L->m * 4));
   const size_t wd = xq_deq_bytes(L, T, true, true);
   w.Wd = wd ? a.take(wd) : nullptr;
@@ -508,7 +514,9 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   float* dG_r = w.dG;
   float* dG_p = w.dG + (m / b) * b * b;
   int sp_r = 1, sp_p = 1;
-  if (dq_p)
+  // with both dq wanted, dG_R and dG_P run as one launch once dA' exists (bf16, b % 256 == 0)
+  const bool one_dg = dq_r && dq_p && t == DT::BF16 && b % 256 == 0 && T > 0;
+  if (dq_p && !one_dg)
     CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, dG_p, T, n, b, w.part_p, &sp_p, s), "bwd dG_P");
   CHECK_CUDA(w0_product(L, w.dB, w.dA1, T, true, w.Wd, s), "bwd W0'^T GEMM");
   if (dx) {
@@ -516,22 +524,44 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
     CHECK_CUDA(scatter_cols(w.dA, dx, T, m, L->perm_r, e, w.inv, s, "perm_bwd_scatter_dX"),
                "bwd scatter dX");
   }
+  bool merged = false;
+  int sp_rp = 1;
   if (dq_r) {
     CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_gather_X"), "bwd gather X");
-    CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, dG_r, T, m, b, w.part_r, &sp_r, s), "bwd dG_R");
+    if (one_dg) {
+      const cudaError_t ce = gemm_block_grad2(t, w.A, w.dA1, m, saved_b, w.dC, n, w.dG, T, b,
+                                              w.part_rp, &sp_rp, s);
+      if (ce == cudaSuccess) merged = true;
+      else if (ce != cudaErrorNotSupported) CHECK_CUDA(ce, "bwd dG_R + dG_P");
+      else CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, dG_p, T, n, b, w.part_p, &sp_p, s),
+                      "bwd dG_P");
+    }
+    if (!merged)
+      CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, dG_r, T, m, b, w.part_r, &sp_r, s), "bwd dG_R");
   }
   if (dq_r || dq_p) {
     // one dq chain over the R blocks and the P blocks
     BlockRuns r;
     int k = 0;
-    if (dq_r) {
-      r.q[k] = L->q_r; r.dq[k] = dq_r; r.splits[k] = sp_r; r.nb[k] = (int)(m / b);
-      r.parts[k] = sp_r > 1 ? static_cast<const float*>(w.part_r) : dG_r;
-      ++k;
-    }
-    if (dq_p) {
-      r.q[k] = L->q_p; r.dq[k] = dq_p; r.splits[k] = sp_p; r.nb[k] = (int)(n / b);
-      r.parts[k] = sp_p > 1 ? static_cast<const float*>(w.part_p) : dG_p;
+    if (merged) {
+      // partials of the one launch: [splits][m/b + n/b][b][b]
+      const float* base = static_cast<const float*>(w.part_rp);
+      const int64_t stride = (m / b + n / b) * b * b;
+      r.q[0] = L->q_r; r.dq[0] = dq_r; r.splits[0] = sp_rp; r.nb[0] = (int)(m / b);
+      r.q[1] = L->q_p; r.dq[1] = dq_p; r.splits[1] = sp_rp; r.nb[1] = (int)(n / b);
+      r.parts[0] = sp_rp > 1 ? base : dG_r;
+      r.parts[1] = sp_rp > 1 ? base + (m / b) * b * b : dG_p;
+      if (sp_rp > 1) r.split_stride[0] = r.split_stride[1] = stride;
+    } else {
+      if (dq_r) {
+        r.q[k] = L->q_r; r.dq[k] = dq_r; r.splits[k] = sp_r; r.nb[k] = (int)(m / b);
+        r.parts[k] = sp_r > 1 ? static_cast<const float*>(w.part_r) : dG_r;
+        ++k;
+      }
+      if (dq_p) {
+        r.q[k] = L->q_p; r.dq[k] = dq_p; r.splits[k] = sp_p; r.nb[k] = (int)(n / b);
+        r.parts[k] = sp_p > 1 ? static_cast<const float*>(w.part_p) : dG_p;
+      }
     }
     r.nb0 = r.nb[0];
     CHECK_CUDA(gemm_dq_from_dg_runs(t, r, b, dq_r ? dG_r : dG_p, w.chain, s), "dq chain");

@@ -166,7 +166,8 @@ dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
   // this block's partial sums within its run, [splits][nb_run][b][b]
   const float* pr = r.parts[run] + (int64_t)local * c.bb;
   const int splits = r.splits[run];
-  const int64_t split_stride = (int64_t)r.nb[run] * c.bb;
+  const int64_t split_stride =
+      r.split_stride[run] ? r.split_stride[run] : (int64_t)r.nb[run] * c.bb;
   const bool in_place = splits == 1 && pr == dG + base;  // written straight into dG
 #pragma unroll
   for (int h = 0; h < 2; ++h) {

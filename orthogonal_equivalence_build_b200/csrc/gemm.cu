@@ -186,6 +186,46 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
   return simt_gemm(g, s);
 }
 
+namespace {
+umma::Gemm block_grad2_gemm(const void* A1, const void* B1, int64_t w1, const void* A2,
+                            const void* B2, int64_t w2, int64_t rows, int64_t b, int sp) {
+  umma::Gemm g;
+  g.M = b; g.N = b; g.K = rows; g.groups = (w1 + w2) / b; g.splits = sp;
+  g.groups_1 = w1 / b;
+  g.A = A1; g.a_rows = rows; g.a_cols = w1; g.a_ld = w1; g.a_mn = true;
+  g.B = B1; g.b_rows = rows; g.b_cols = w1; g.b_ld = w1; g.b_mn = true;
+  g.A2 = A2; g.a2_rows = rows; g.a2_cols = w2; g.a2_ld = w2;
+  g.B2 = B2; g.b2_rows = rows; g.b2_cols = w2; g.b2_ld = w2;
+  g.a_gm = b; g.a_gk = 0; g.b_gn = b; g.b_gk = 0;
+  g.out_f32 = true; g.ldc = b; g.c_gs = b * b; g.c_split = (w1 + w2) * b;
+  g.name = "umma_block_grad";
+  return g;
+}
+int block_grad2_splits(int64_t w1, int64_t w2, int64_t b, int64_t rows) {
+  return umma::effective_splits(rows, grad_splits((w1 + w2) / b, b, rows));
+}
+}  // namespace
+
+size_t block_grad2_ws_bytes(DT t, int64_t w1, int64_t w2, int64_t b, int64_t rows) {
+  if (t != DT::BF16 || b % 256 != 0) return 0;
+  const int sp = block_grad2_splits(w1, w2, b, rows);
+  return sp > 1 ? (size_t)sp * (size_t)((w1 + w2) * b) * sizeof(float) : 0;
+}
+
+cudaError_t gemm_block_grad2(DT t, const void* A1, const void* B1, int64_t w1, const void* A2,
+                             const void* B2, int64_t w2, float* dG, int64_t rows, int64_t b,
+                             void* partials, int* splits_used, cudaStream_t s) {
+  *splits_used = 1;
+  if (t != DT::BF16 || rows == 0 || b % 256 != 0) return cudaErrorNotSupported;
+  const int sp = block_grad2_splits(w1, w2, b, rows);
+  if (sp > 1 && !partials) return cudaErrorNotSupported;
+  umma::Gemm g = block_grad2_gemm(A1, B1, w1, A2, B2, w2, rows, b, sp);
+  g.C = sp > 1 ? partials : dG;
+  if (!umma::pair_supported(g)) return cudaErrorNotSupported;
+  *splits_used = sp;
+  return umma::gemm_pair(g, s);
+}
+
 size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b) {
   return tc_blocks_supported(b) ? cnp_tc_ws_bytes(nb, b) : cnp_ws_bytes(nb, b);
 }

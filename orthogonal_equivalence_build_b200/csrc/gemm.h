@@ -32,6 +32,15 @@ size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows);
 cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
                             int64_t width, int64_t b, void* partials, int* splits_used,
                             cudaStream_t s);
+// The same contraction for two runs of blocks in one launch (bf16, CTA pairs, b % 256 == 0):
+// groups 0 .. w1/b - 1 from (A1, B1) [rows, w1], then w2/b groups from (A2, B2) [rows, w2];
+// dG [(w1 + w2)/b][b][b]. One launch over all blocks fills the waves with fewer splits. With
+// more than one range the partials go to `partials` ([splits][(w1 + w2)/b][b][b],
+// block_grad2_ws_bytes bytes). Returns cudaErrorNotSupported where it does not apply.
+size_t block_grad2_ws_bytes(DT t, int64_t w1, int64_t w2, int64_t b, int64_t rows);
+cudaError_t gemm_block_grad2(DT t, const void* A1, const void* B1, int64_t w1, const void* A2,
+                             const void* B2, int64_t w2, float* dG, int64_t rows, int64_t b,
+                             void* partials, int* splits_used, cudaStream_t s);
 // CNP blocks and the dq chain: tensor cores (cnp_tc.cu) when b is a multiple of 128, SIMT fp32
 // (cnp.cu) otherwise; the dq chain of fp32 layers always runs in fp32 SIMT.
 bool tc_blocks_supported(int64_t b);
@@ -47,6 +56,7 @@ struct BlockRuns {
   float* dq[2] = {nullptr, nullptr};          // packed gradients
   const float* parts[2] = {nullptr, nullptr}; // dG split partials [splits][nb][b][b]
   int splits[2] = {1, 1};
+  int64_t split_stride[2] = {0, 0};           // elements between splits (0: nb[run] * b * b)
   int nb[2] = {0, 0};
   int nb0 = 0;                                // == nb[0]
 };

@@ -659,6 +659,7 @@ struct PairParams {
   void* C;
   long long ldc, c_gs, c_split;
   const float* b_scale;   // int8 B only: one scale per column of the stored B tensor
+  int g2;                 // first group read from the second operand pair (groups: none)
   int raster, band;       // tile order within a group: 0 = bands of `band` pair-rows, N inner;
                           // 1 = bands of `band` pair-columns, N fastest inside a band
   Epi epi;
@@ -832,7 +833,9 @@ template <bool A_MN, bool B_MN, bool OUT_F32, bool B_I8>
 __global__ void __launch_bounds__((PairCfg<B_I8, OUT_F32>::THREADS), 1)
 umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b,
-                      const __grid_constant__ CUtensorMap tma_c, const PairParams p) {
+                      const __grid_constant__ CUtensorMap tma_c,
+                      const __grid_constant__ CUtensorMap tma_a2,
+                      const __grid_constant__ CUtensorMap tma_b2, const PairParams p) {
   using Cfg = PairCfg<B_I8, OUT_F32>;
   constexpr int EPI_W = Cfg::EPI_W;
   constexpr int STAGES = Cfg::STAGES;
@@ -942,8 +945,13 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         const TileCoord tc = decode_pair_tile(p, tile);
         const int kb0 = tc.split * p.kblocks_per_split;
         const int kb1 = min(kb0 + p.kblocks_per_split, (p.K + BK - 1) / BK);
-        const int am = tc.g * p.a_gm + tc.mb * 256 + (int)rank * 128, ak = tc.g * p.a_gk;
-        const int bn = tc.g * p.b_gn + tc.nb * 256 + (int)rank * 128, bk = tc.g * p.b_gk;
+        // groups from g2 on come from the second operand pair, counted from its first group
+        const bool second = tc.g >= p.g2;
+        const CUtensorMap* map_a = second ? &tma_a2 : &tma_a;
+        const CUtensorMap* map_b = second ? &tma_b2 : &tma_b;
+        const int gl = second ? tc.g - p.g2 : tc.g;
+        const int am = gl * p.a_gm + tc.mb * 256 + (int)rank * 128, ak = gl * p.a_gk;
+        const int bn = gl * p.b_gn + tc.nb * 256 + (int)rank * 128, bk = gl * p.b_gk;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -964,20 +972,20 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
           const KCoord kc = k_coord(p, kb);
           const int k = kc.k;
           if constexpr (A_MN) {
-            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, am + kc.adx, ak + k + kc.ady);
-            tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), &tma_a, fb,
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), map_a, fb, am + kc.adx, ak + k + kc.ady);
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES + 64 * BK * 2), map_a, fb,
                              am + 64 + kc.adx, ak + k + kc.ady);
           } else {
-            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, ak + k + kc.adx, am + kc.ady);
+            tma_load_2d_pair(smem_u32(sa + s * A_BYTES), map_a, fb, ak + k + kc.adx, am + kc.ady);
           }
           if constexpr (B_I8) {
             // the int8 tile of this K block was issued by issue_raw
           } else if constexpr (B_MN) {
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bn + kc.bdx, bk + k + kc.bdy);
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), &tma_b, fb,
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), map_b, fb, bn + kc.bdx, bk + k + kc.bdy);
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES + 64 * BK * 2), map_b, fb,
                              bn + 64 + kc.bdx, bk + k + kc.bdy);
           } else {
-            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), &tma_b, fb, bk + k + kc.bdx, bn + kc.bdy);
+            tma_load_2d_pair(smem_u32(sb + s * B_BYTES), map_b, fb, bk + k + kc.bdx, bn + kc.bdy);
           }
         }
       }
@@ -1289,14 +1297,25 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   // bf16 output through TMA stores: C as a 2-D [M][ldc] tensor, 64 x 32 boxes, 128-byte swizzle
   CUtensorMap tc = ta;   // fp32 outputs keep the thread stores; the map is then unused
   if constexpr (!OUT_F32) {
-    // a group offset c_gs is a column offset (< ldc) or whole rows (a multiple of ldc)
+    // a group offset c_gs is a column offset (< ldc: every group in the same M rows) or whole
+    // rows (a multiple of ldc: group g starts g * c_gs / ldc rows down). The map holds exactly
+    // the rows the product owns, so the copy clips a ragged last row tile at row M of its group.
     if (g.c_gs % g.ldc != 0 && g.c_gs >= g.ldc) return cudaErrorNotSupported;
-    const int64_t extent = (g.groups - 1) * g.c_gs + g.M * g.ldc;
-    const int64_t rows = (extent + g.ldc - 1) / g.ldc;
+    if (g.c_gs % g.ldc != 0 && (g.groups - 1) * g.c_gs + g.N > g.ldc) return cudaErrorNotSupported;
+    const int64_t rows = (g.c_gs % g.ldc == 0) ? (g.groups - 1) * (g.c_gs / g.ldc) + g.M : g.M;
     if (!make_map(&tc, g.C, rows, g.ldc, g.ldc, 32)) return cudaErrorInvalidValue;
+  }
+  // the second operand pair (groups >= groups_1), same box shapes and swizzle
+  CUtensorMap ta2 = ta, tb2 = tb;
+  if (g.A2) {
+    if constexpr (B_I8) return cudaErrorNotSupported;
+    if (!make_map(&ta2, g.A2, g.a2_rows, g.a2_cols, g.a2_ld, A_MN ? BK : 128) ||
+        !make_map(&tb2, g.B2, g.b2_rows, g.b2_cols, g.b2_ld, B_MN ? BK : 128))
+      return cudaErrorInvalidValue;
   }
   PairParams p;
   p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = (int)g.groups;
+  p.g2 = g.A2 ? (int)g.groups_1 : (int)g.groups;
   p.tiles_m = (int)((g.M + 255) / 256);
   p.tiles_n = (int)(g.N / 256);
   const int kblocks = (int)((g.K + BK - 1) / BK);
@@ -1347,7 +1366,7 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   const int clusters = std::min(p.total_tiles, max_clusters);
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   TraceScope t(name, s);
-  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, ta2, tb2, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1429,6 +1448,19 @@ bool pair_supported(const Gemm& g) {
            !g.a_mn && !g.out_f32 && g.b_scale && g.b_ld % 16 == 0 && g.b_cols % 16 == 0 &&
            (reinterpret_cast<uintptr_t>(g.b_scale) & 15) == 0;
   }
+  if (g.A2) {
+    // a second operand pair: both sets must be valid operands of the same grouped product
+    Gemm h = g;
+    h.A = g.A2; h.a_rows = g.a2_rows; h.a_cols = g.a2_cols; h.a_ld = g.a2_ld;
+    h.B = g.B2; h.b_rows = g.b2_rows; h.b_cols = g.b2_cols; h.b_ld = g.b2_ld;
+    h.A2 = nullptr; h.B2 = nullptr;
+    h.groups = g.groups - g.groups_1;
+    Gemm f = g;
+    f.A2 = nullptr; f.B2 = nullptr;
+    f.groups = g.groups_1;
+    return g.B2 && g.groups_1 > 0 && g.groups_1 < g.groups && !g.b_i8 && g.epi.mode == kEpiStore &&
+           pair_supported(f) && pair_supported(h);
+  }
   return supported(g) && g.N % 256 == 0 && g.M >= 256 && !(g.a_mn && !g.b_mn) &&
          !(g.a_mn && g.b_mn && !g.out_f32) && (g.groups == 1 || g.a_gm == 0 || g.a_gm % 256 == 0);
 }
@@ -1453,6 +1485,7 @@ cudaError_t gemm_pair(const Gemm& g, cudaStream_t s) {
 }
 
 cudaError_t gemm(const Gemm& g, cudaStream_t s) {
+  if (g.A2) return cudaErrorNotSupported;   // the second operand pair is CTA-pair only
   if (g.bn != 0 && g.bn != 64 && g.bn != 128 && g.bn != 256) return cudaErrorInvalidValue;
   const int cap = g.bn ? g.bn : 256;
   if (g.N % 256 == 0 && cap >= 256) return dispatch_majors<256>(g, s);

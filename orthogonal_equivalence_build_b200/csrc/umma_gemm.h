@@ -55,6 +55,12 @@ struct Gemm {
   void* C = nullptr; bool out_f32 = false; int64_t ldc = 0, c_gs = 0, c_split = 0;
   const char* name = nullptr;
   int bn = 0;   // single-CTA tile width (64, 128 or 256; N must be a multiple); 0: the widest
+  // CTA-pair kernel only: groups >= groups_1 read a second operand pair (A2, B2), laid out like
+  // (A, B) with its own extents; group g >= groups_1 is group g - groups_1 of that pair. The
+  // output keeps the global group index. 0: every group reads (A, B).
+  int64_t groups_1 = 0;
+  const void* A2 = nullptr; int64_t a2_rows = 0, a2_cols = 0, a2_ld = 0;
+  const void* B2 = nullptr; int64_t b2_rows = 0, b2_cols = 0, b2_ld = 0;
 };
 
 bool supported(const Gemm& g);

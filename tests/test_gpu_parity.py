@@ -220,6 +220,10 @@ def test_layer_cnp_build_matches_per_side_builds(key, m, n, b):
 @pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 700),
                                          ("tiny_fp32", 256, 512, 64, 99)])
 def test_one_sided_dq_matches_two_sided(key, m, n, b, T):
+    """dq of one side alone (its own dG launch) equals the two-sided dq (bf16, b % 256 == 0: one
+    dG launch over both sides) bit for bit. At T = 700 both take one split of the token range,
+    so the sums run in the same order; at larger T the split counts differ and the two agree
+    within rounding, which the oracle parity cases (T = 2049, 2305: several splits) check."""
     c = LayerCase(key, m=m, n=n, b=b, tokens=T)
     y, bsave = c.forward()
     dx, dq_r, dq_p = c.backward(bsave)
