@@ -324,3 +324,44 @@ def test_llama13b_layer_400_steps_with_merge_reinit():
         q_r += d_r
         q_p += d_p
     assert np.array_equal(c.q_r.cpu().numpy(), q_r)
+
+
+# ------------------------------------------------------------------ no writes outside the outputs
+@pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 700),
+                                         ("llama1p3b_attn", 1024, 1024, 256, 333),
+                                         ("llama8b_up_proj", 1024, 2048, 512, 2305)])
+def test_no_write_outside_outputs_or_workspace(key, m, n, b, T):
+    """Every output (y, saved B, dx, dq_r, dq_p) and both workspaces sit inside larger buffers whose
+    slack is filled with a canary; after the forward and the backward (saved B and rebuilt B) at a
+    ragged token count, every canary byte is intact."""
+    c = LayerCase(key, m=m, n=n, b=b, tokens=T)
+    pad = 4096   # elements of slack on each side
+
+    def boxed(numel, dtype):
+        buf = torch.full((numel + 2 * pad,), -7.0, dtype=dtype, device="cuda")
+        return buf, buf[pad:pad + numel]
+
+    def ws_boxed(nbytes):
+        buf = torch.full((nbytes + 2 * pad * 8,), 0xA5, dtype=torch.uint8, device="cuda")
+        return buf, buf[pad * 8:pad * 8 + nbytes]
+
+    dt = c.x.dtype
+    y_buf, y = boxed(T * n, dt)
+    b_buf, bs = boxed(T * n, dt)
+    fws_buf, fws = ws_boxed(poetx.fwd_workspace_bytes(c.layer, T))
+    poetx.linear_fwd(c.layer, c.x, y.view(T, n), bs.view(T, n), fws)
+    dx_buf, dx = boxed(T * m, dt)
+    dqr_buf, dqr = boxed(c.q_r.numel(), torch.float32)
+    dqp_buf, dqp = boxed(c.q_p.numel(), torch.float32)
+    bws_buf, bws = ws_boxed(poetx.bwd_workspace_bytes(c.layer, T))
+    for saved in (bs.view(T, n), None):
+        poetx.linear_bwd(c.layer, c.x, c.dy, saved, dx.view(T, m), dqr.view_as(c.q_r),
+                         dqp.view_as(c.q_p), bws)
+    torch.cuda.synchronize()
+    for name, buf, fill in (("y", y_buf, -7.0), ("saved_b", b_buf, -7.0), ("dx", dx_buf, -7.0),
+                            ("dq_r", dqr_buf, -7.0), ("dq_p", dqp_buf, -7.0)):
+        for side in (buf[:pad], buf[-pad:]):
+            assert bool((side == fill).all()), name
+    for name, buf in (("fwd workspace", fws_buf), ("bwd workspace", bws_buf)):
+        for side in (buf[:pad * 8], buf[-pad * 8:]):
+            assert bool((side == 0xA5).all()), name
