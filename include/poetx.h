@@ -85,8 +85,11 @@ typedef struct {
   int32_t flags;   /* 0, POETX_LAYER_W0M_I8, or POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED */
   void* w0m;       /* [m, n] merged weight W0' (see poetx_merge_permutations); int8 codes
                       when flags has POETX_LAYER_W0M_I8 */
-  int32_t* perm_r; /* [m] permutation of R */
-  int32_t* perm_p; /* [n] permutation of P */
+  int32_t* perm_r; /* [m] permutation of R: each of 0..m-1 exactly once */
+  int32_t* perm_p; /* [n] permutation of P: each of 0..n-1 exactly once. Not checked on the
+                      hot path (poetx_validate_permutation checks one): an index outside the
+                      range is undefined behaviour and can make a kernel access memory out of
+                      bounds. */
   float* q_r;      /* [m/b, b(b-1)/2] packed skew parameters of R */
   float* q_p;      /* [n/b, b(b-1)/2] packed skew parameters of P */
   float* g_r;      /* [m/b, b, b] fp32 CNP blocks of R (written by poetx_cnp_build) */
