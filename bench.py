@@ -3,8 +3,9 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload KEY] [--tokens T]
                     [--impl ours|reference] [--xq | --xq-staged] [--first-linear-only]
 
-One step is the whole hot path over one batch: poetx_cnp_build for R and P, poetx_linear_fwd,
-poetx_linear_bwd (dx, dq_r, dq_p), for every linear of the workload.  Inputs are synthetic
+One step is the whole hot path over one batch, for every linear of the workload: poetx_cnp_build
+for R and P (where the workload's step includes it), poetx_linear_fwd, poetx_linear_bwd (dx, dq_r,
+dq_p), and merge_reinit amortised over its period where the workload has one.  Inputs are synthetic
 (seeded, poetx_workloads) and resident in HBM before the timed region.  --xq stores W0' in 8 bits
 (int8 codes + column scales, dequantised inside the W0' products); --xq-staged dequantises it
 into the workspace once per product instead.  For N > 1 (torchrun, one rank per GPU) every rank runs the step
