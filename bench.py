@@ -186,20 +186,23 @@ class ClockSampler:
 _SAMPLE_CACHE = {}
 
 
-def oracle_step_sample(wl, T_sample: int):
+def oracle_step_sample(wl, T_sample: int, nlin: int = 1):
     """One float64 oracle step (CNP of R and P, forward, backward with dq) of the workload's
-    first linear on T_sample tokens.  Returns (seconds, tokens)."""
+    first nlin linears on T_sample tokens.  Returns (seconds, tokens)."""
     import oracle as O
-    key = (wl.key, T_sample)
+    key = (wl.key, T_sample, nlin)
     if key not in _SAMPLE_CACHE:
-        p = W.layer_params(wl)
-        a = W.layer_acts(wl, tokens=T_sample)
-        _SAMPLE_CACHE[key] = (p, a, O.merge_permutations(p["W0"], p["perm_r"], p["perm_p"]))
-    p, a, W0m = _SAMPLE_CACHE[key]
+        items = []
+        for li in range(nlin):
+            p = W.layer_params(wl, li)
+            a = W.layer_acts(wl, li, tokens=T_sample)
+            items.append((p, a, O.merge_permutations(p["W0"], p["perm_r"], p["perm_p"])))
+        _SAMPLE_CACHE[key] = items
     t0 = time.perf_counter()
-    G_r, G_p = O.cnp(p["q_r"], wl.b), O.cnp(p["q_p"], wl.b)
-    O.linear_bwd(a["X"], a["dY"], W0m, p["perm_r"], p["perm_p"], G_r, G_p, p["q_r"], p["q_p"],
-                 wl.b)
+    for p, a, W0m in _SAMPLE_CACHE[key]:
+        G_r, G_p = O.cnp(p["q_r"], wl.b), O.cnp(p["q_p"], wl.b)
+        O.linear_bwd(a["X"], a["dY"], W0m, p["perm_r"], p["perm_p"], G_r, G_p, p["q_r"],
+                     p["q_p"], wl.b)
     return time.perf_counter() - t0, T_sample
 
 
@@ -214,12 +217,43 @@ def blas_threads():
     return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, T_sample):
-    dt, tok = oracle_step_sample(wl, T_sample)
+def sample_text(wl, T_sample, nlin):
+    what = f"the {wl.key} layer" if nlin == 1 else f"the {nlin} linears of {wl.key}"
+    return (f"one float64 oracle step (CNP + fwd + bwd with dq) of {what} on {T_sample} of its "
+            f"{wl.tokens} tokens" + (" (merge_reinit not sampled)" if wl.merge_every else ""))
+
+
+def cpu_baseline(wl, T_sample, nlin=1):
+    dt, tok = oracle_step_sample(wl, T_sample, nlin)
     return {"value": tok / dt, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"one float64 oracle step (CNP + fwd + bwd with dq) of the {wl.key} layer "
-                      f"on {T_sample} of its {wl.tokens} tokens: {dt:.2f} s",
-            "seconds": dt}
+            "sample": f"{sample_text(wl, T_sample, nlin)}: {dt:.2f} s", "seconds": dt}
+
+
+def workload_config(wl, args, world):
+    """The `config` object of the JSON line, the same for both arms: the workload as run (its
+    linears, block size, tokens, parallelism, what one step holds, how L2 is kept cold)."""
+    T = args.tokens or wl.tokens
+    esz = 2 if wl.dtype == "bf16" else 4
+    lins = wl.linears if args.all_linears else wl.linears[:1]
+    in_bytes = sum(T * (lin.m + lin.n) * esz for lin in lins)
+    cfg = {"workload": wl.key, "linears": [f"{lin.name} {lin.m}x{lin.n}" for lin in lins],
+           "b": wl.b, "tokens_per_gpu": T, "global_batch_tokens": T * world,
+           "parallelism": f"dp{world}",
+           "step": ("cnp_build(R,P) + " if wl.cnp_in_step else "")
+           + "linear_fwd + linear_bwd(dx, dq) per linear"
+           + (" + NCCL all-reduce of dq" if world > 1 else ""),
+           "l2": (f"inputs larger than L2: X + dY = {in_bytes / 2**20:.0f} MiB per step"
+                  if in_bytes > L2_BYTES else "L2 flushed (2x126 MiB write) between steps")}
+    if len(lins) == 1:
+        cfg.update({"m": lins[0].m, "n": lins[0].n})
+    if args.xq:
+        cfg["w0m_storage"] = (
+            "int8 codes + fp32 column scales, dequantised to bf16 "
+            + ("into the workspace once per W0' product (staged)" if args.xq_staged
+               else "in the W0' GEMMs' shared-memory operand stages"))
+    if wl.merge_every:
+        cfg["merge_reinit"] = f"every {wl.merge_every} steps, amortised into ms_per_step"
+    return cfg
 
 
 def run_reference(args):
@@ -227,11 +261,11 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = W.WORKLOADS[args.workload]
-    lin = wl.linears[0]
+    nlin = len(wl.linears) if args.all_linears else 1
     T_sample = args.ref_tokens
     times = []
     for i in range(args.warmup + args.steps):
-        dt, _ = oracle_step_sample(wl, T_sample)
+        dt, _ = oracle_step_sample(wl, T_sample, nlin)
         if i >= args.warmup:
             times.append(dt)
     sec = statistics.mean(times)
@@ -241,11 +275,10 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.key, "m": lin.m, "n": lin.n, "b": wl.b,
-                   "tokens_per_step": T_sample, "parallelism": "none (host cores)"},
+        "config": workload_config(wl, args, world),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle",
-                         "sample": f"float64 oracle step on {T_sample} of {wl.tokens} tokens"},
+                         "sample": sample_text(wl, T_sample, nlin)},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
@@ -482,26 +515,9 @@ def run_ours(args):
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(wl, args.ref_tokens)
+            cpu = cpu_baseline(wl, args.ref_tokens, nlin)
             cpu.pop("seconds", None)
-        shapes = [f"{d['lin'].name} {d['lin'].m}x{d['lin'].n}" for d in layers]
-        cfg = {"workload": wl.key, "linears": shapes, "b": b, "tokens_per_gpu": T,
-               "global_batch_tokens": T * world, "parallelism": f"dp{world}",
-               "step": ("cnp_build(R,P) + " if wl.cnp_in_step else "")
-               + "linear_fwd + linear_bwd(dx, dq) per linear"
-               + (" + NCCL all-reduce of dq" if world > 1 else ""),
-               "l2": (f"inputs larger than L2: X + dY = {in_bytes / 2**20:.0f} MiB per step"
-                      if flush is None else "L2 flushed (2x126 MiB write) between steps")}
-        if nlin == 1:
-            cfg.update({"m": layers[0]["lin"].m, "n": layers[0]["lin"].n})
-        if args.xq:
-            cfg["w0m_storage"] = (
-                "int8 codes + fp32 column scales, dequantised to bf16 "
-                + ("into the workspace once per W0' product (staged)" if args.xq_staged
-                   else "in the W0' GEMMs' shared-memory operand stages"))
-        if wl.merge_every:
-            cfg["merge_reinit"] = (f"every {wl.merge_every} steps: {merge_ms:.3f} ms for all "
-                                   f"linears, amortised into ms_per_step")
+        cfg = workload_config(wl, args, world)
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -513,6 +529,7 @@ def run_ours(args):
                               "flops": F, "bytes": Bb, "peaks": peak_src},
             "roofline": roofline,
             "cpu_baseline": cpu,
+            **({"merge_reinit_ms": merge_ms} if wl.merge_every else {}),
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clocks,
