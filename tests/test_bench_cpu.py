@@ -1,0 +1,44 @@
+"""The benchmark's JSON contract, checked on CPU through its reference arm (the float64 oracle on
+the host cores): one line with the required keys, the same `config` object the GPU arm prints for
+the workload, and an end-to-end record that moves no bytes."""
+import json
+import os
+import subprocess
+import sys
+import types
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _run(*extra):
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "0", "--ref-tokens", "8", *extra],
+                         capture_output=True, text=True, timeout=300, check=True)
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out.stdout
+    return json.loads(lines[0])
+
+
+def test_reference_line_has_the_contract_keys():
+    d = _run()
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1
+    assert "8 of its 16384 tokens" in cb["sample"]
+    e2e = d["e2e"]
+    assert e2e["value"] == d["value"] and e2e["unit"] == d["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_reference_config_is_the_gpu_arms_config():
+    sys.path.insert(0, ROOT)
+    import bench
+    import poetx_workloads as W
+    for key in ("llama8b_up_proj", "llama13b_layers"):
+        d = _run("--workload", key)
+        args = types.SimpleNamespace(tokens=None, all_linears=True, xq=False, xq_staged=False)
+        assert d["config"] == bench.workload_config(W.WORKLOADS[key], args, 1), key
