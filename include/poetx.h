@@ -141,8 +141,12 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t
  *   Limit: b must need at most POETX_CNP_NOALLOC_SCRATCH_BYTES of scratch for ONE block
  *   (12*b*b bytes, in slices rounded up to 256 bytes): b <= 836; larger b returns
  *   POETX_ERR_SHAPE with a message.
- *   The first call on each device looks up the buffer's device address (cudaGetSymbolAddress)
- *   with that device current; make that first call before any stream capture.
+ *   Set-up: the first call on each device looks up the buffer's device address
+ *   (cudaGetSymbolAddress) with that device current. With lazy module loading (the CUDA
+ *   default) that lookup is also where the driver loads the library's module holding the
+ *   buffer and commits its device memory. So make the first call on each device before the
+ *   stretch of the program that must not allocate, and before any stream capture. A call with
+ *   nblocks = 0 does exactly this set-up (and its checks) and launches nothing.
  *   All calls on a device share the one buffer and it keeps the last call's contents (nothing in
  *   it needs to start at zero: every byte read is written earlier in the same call). Calls whose
  *   work overlaps on the GPU (e.g. on two streams without ordering) race on the buffer: order
@@ -246,7 +250,10 @@ poetx_status poetx_device_status(void* stream);
 /* Tracing: when enabled, every kernel the library launches is bracketed by CUDA events on its
  * stream. poetx_trace_read() synchronises those events and writes one line per launch,
  * "<kernel name> <milliseconds>\n", into buf (truncated to len), then clears the record.
- * Returns the number of launches recorded. */
+ * Returns the number of launches recorded. The same names label NVTX ranges for profilers.
+ * A bf16 contraction whose shape the tensor-core tiling does not cover (a block size b that is
+ * not a multiple of 64, or b < 64) runs on the fp32-accumulating SIMT kernel and is recorded as
+ * "simt_gemm_bf16_fallback"; fp32 layers' products are "simt_gemm_f32". */
 poetx_status poetx_trace_enable(int32_t on);
 int64_t poetx_trace_read(char* buf, size_t len);
 /* Record only launches whose name is one of `names` (comma-separated, exact match); NULL or ""

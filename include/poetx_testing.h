@@ -14,7 +14,18 @@
  *   partial products to C + s * M * ldc (c_f32 must be 1); the caller adds them. A count that
  *   would leave a range empty (e.g. 5 ranges over 16 blocks) is rejected with INVALID_ARG.
  *   variant 0 runs the single-CTA kernel (128 x BN tiles); variant 1 runs the CTA-pair kernel
- *   (tcgen05.mma.cta_group::2 on a 2-CTA cluster, 256 x 256 tiles; N % 256 == 0, M >= 256).
+ *   (tcgen05.mma.cta_group::2 on a 2-CTA cluster, 256 x 256 tiles; N % 256 == 0, M >= 256);
+ *   variants 2 and 3 run the dense CTA-pair kernel on 256 x 512 tiles (A K-major, bf16 C,
+ *   splits = 1, N % 512 == 0, M >= 256), with (2) or without (3) the two MMAs of a K step
+ *   sharing A through the tensor core's collector buffer.
+ *   epi_wait_ns > 0 limits the epilogue warps' wait for a finished accumulator to that many
+ *   nanoseconds (0: the kernels' default of 4 s). It exists to exercise the bounded-wait error
+ *   path: with a limit shorter than the main loop the wait runs out, the epilogue writes a
+ *   nonzero code into the device error word (poetx_device_status then returns
+ *   POETX_ERR_TIMEOUT and clears it), skips its stores and leaves; the producer and MMA roles
+ *   finish or drain their copies and MMAs, TMEM is freed and the kernel returns. C is then
+ *   unspecified. Use a product of at most two tiles per CTA (cluster) for a clean drain:
+ *   the MMA role then never waits for an accumulator the epilogue would have handed back.
  * Returns POETX_ERR_UNSUPPORTED when the chosen kernel's tiling does not cover the shape
  * (N % 64 != 0, K-major extents < 64, misaligned pointers or strides); it never falls back.
  * Asynchronous on `stream`.
@@ -29,7 +40,8 @@ extern "C" {
 poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, int64_t a_cols, int32_t a_mn,
                                      const void* B, int64_t b_rows, int64_t b_cols, int32_t b_mn,
                                      int64_t M, int64_t N, int64_t K, void* C, int32_t c_f32,
-                                     int64_t ldc, int32_t splits, int32_t variant, void* stream);
+                                     int64_t ldc, int32_t splits, int32_t variant,
+                                     uint64_t epi_wait_ns, void* stream);
 
 #ifdef __cplusplus
 }

@@ -64,12 +64,11 @@ extern "C" poetx_status poetx_cnp_build_noalloc(const float* q, int64_t nblocks,
               (long long)b, per_block, (size_t)POETX_CNP_NOALLOC_SCRATCH_BYTES);
     return POETX_ERR_SHAPE;
   }
-  if (nblocks == 0) return POETX_OK;
-  if (!q) {
+  if (nblocks > 0 && !q) {
     set_error("cnp_build_noalloc: q is NULL");
     return POETX_ERR_INVALID_ARG;
   }
-  if (!g && !g_lp) {
+  if (nblocks > 0 && !g && !g_lp) {
     set_error("cnp_build_noalloc: both outputs are NULL");
     return POETX_ERR_INVALID_ARG;
   }
@@ -92,12 +91,15 @@ extern "C" poetx_status poetx_cnp_build_noalloc(const float* q, int64_t nblocks,
     set_error("cnp_build_noalloc: device %d is not sm_100", dev);
     return POETX_ERR_UNSUPPORTED;
   }
+  // per-device set-up (first call on the device): the scratch buffer's device address. Under
+  // lazy module loading this is where the module that holds the buffer gets loaded.
   void* scratch = nullptr;
   cudaError_t e = scratch_address(&scratch);
   if (e != cudaSuccess) {
     set_error("cnp_build_noalloc: cudaGetSymbolAddress: %s", cudaGetErrorString(e));
     return POETX_ERR_CUDA;
   }
+  if (nblocks == 0) return POETX_OK;   // set-up only
   // largest chunk of blocks whose scratch fits the buffer
   int64_t chunk = (int64_t)(POETX_CNP_NOALLOC_SCRATCH_BYTES / per_block);
   while (chunk > 1 && gemm_cnp_ws_bytes(chunk, b) > (size_t)POETX_CNP_NOALLOC_SCRATCH_BYTES) --chunk;

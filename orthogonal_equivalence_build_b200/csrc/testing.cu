@@ -7,7 +7,7 @@ extern "C" poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, i
                                                 int64_t b_cols, int32_t b_mn, int64_t M,
                                                 int64_t N, int64_t K, void* C, int32_t c_f32,
                                                 int64_t ldc, int32_t splits, int32_t variant,
-                                                void* stream) {
+                                                uint64_t epi_wait_ns, void* stream) {
   using namespace poetx;
   if (!A || !B || !C || M <= 0 || N <= 0 || K <= 0 || splits < 1) {
     set_error("testing_gemm: bad arguments");
@@ -28,14 +28,18 @@ extern "C" poetx_status poetx_testing_gemm_bf16(const void* A, int64_t a_rows, i
   g.B = B; g.b_rows = b_rows; g.b_cols = b_cols; g.b_ld = b_cols; g.b_mn = b_mn != 0;
   g.C = C; g.out_f32 = c_f32 != 0; g.ldc = ldc; g.c_split = M * ldc;
   g.name = "umma_testing_gemm";
+  g.epi_wait_ns = epi_wait_ns;
   const bool pair = variant == 1;
+  const bool wide = variant == 2 || variant == 3;
+  g.wide_collect = variant == 2;
   if (!umma::supported(g) || (g.a_mn && g.b_mn && !g.out_f32) || (g.a_mn && !g.b_mn) ||
-      (pair && !umma::pair_supported(g)) || variant < 0 || variant > 1) {
+      (pair && !umma::pair_supported(g)) || (wide && !umma::wide_supported(g)) || variant < 0 ||
+      variant > 3) {
     set_error("testing_gemm: shape/layout not covered by the tensor-core kernel");
     return POETX_ERR_UNSUPPORTED;
   }
-  cudaError_t e = pair ? umma::gemm_pair(g, static_cast<cudaStream_t>(stream))
-                       : umma::gemm(g, static_cast<cudaStream_t>(stream));
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = wide ? umma::gemm_wide(g, s) : pair ? umma::gemm_pair(g, s) : umma::gemm(g, s);
   if (e != cudaSuccess) {
     set_error("testing_gemm: %s", cudaGetErrorString(e));
     return POETX_ERR_CUDA;

@@ -55,6 +55,7 @@ struct Params {
   long long ldc, c_gs, c_split;
   Epi epi;
   int* err;
+  unsigned long long epi_wait_ns;   // limit of the epilogue's accumulator wait
 };
 
 // TMA coordinate shifts of K block kb: k restarts at 0 in every segment.
@@ -97,6 +98,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// Non-blocking test of a phase (never suspends the thread, unlike try_wait).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
 // The same test with cluster-scope acquire: for barriers that other CTAs of the cluster
 // release into (their arrivals order their own shared-memory writes before this thread's reads).
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
@@ -121,17 +134,18 @@ struct Ctl {
   int* err;
 };
 
-// Wait for `parity` on `bar`; false if the CTA is aborting or the wait expired.
+// Wait for `parity` on `bar`; false if the CTA is aborting (unless stop_on_abort is false) or
+// the wait expired.
 template <bool CLUSTER = false>
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, Ctl c, int code,
-                                          uint64_t limit_ns) {
+                                          uint64_t limit_ns, bool stop_on_abort = true) {
   auto test = [&] { return CLUSTER ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
   if (test()) return true;
   const uint64_t t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (test()) return true;
     if ((it & 31) == 0) {
-      if (*c.abort) return false;
+      if (stop_on_abort && *c.abort) return false;
       if (global_ns() - t0 > limit_ns) {
         *c.abort = 1;
         if (code) atomicCAS(c.err, 0, code);
@@ -611,7 +625,8 @@ umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constan
       FusedQ q0;
       if (fused)
         fused_q_load(p.epi, fused_base(p.epi, tc.g, row0, tc.nb * BN, lane), 0, nlive, lane, q0);
-      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
+      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, p.epi_wait_ns))
+        break;
       tc_fence_after();
       const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
                              (long long)row0 * p.ldc + (long long)tc.nb * BN;
@@ -664,6 +679,7 @@ struct PairParams {
                           // 1 = bands of `band` pair-columns, N fastest inside a band
   Epi epi;
   int* err;
+  unsigned long long epi_wait_ns;   // limit of the epilogue's accumulator wait
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -927,7 +943,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       auto issue_raw = [&](int j) -> bool {
         const int r = j % RAWD;
         if (!wait_bounded(smem_u32(qempty + r), ((uint32_t)(j / RAWD) & 1u) ^ 1u, ctl,
-                          kErrProducer, kWaitLimitNs))
+                          kErrProducer, kWaitLimitNs, /*stop_on_abort=*/false))
           return false;
         const int kj = rkb * BK;
         const uint32_t qb = smem_u32(qfull + r);
@@ -962,7 +978,12 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             }
             if (!ok) break;
           }
-          if (!wait_bounded(smem_u32(empty + s), ph ^ 1u, ctl, kErrProducer, kWaitLimitNs)) {
+          // The two producers stop only when this wait runs out, not on the CTA's abort flag:
+          // both are released by the same multicast commits, so both then have issued the
+          // same loads, every one of which the leader armed and drains below. (Stopping on
+          // the flag could leave the peer's last load unarmed and still in flight at exit.)
+          if (!wait_bounded(smem_u32(empty + s), ph ^ 1u, ctl, kErrProducer, kWaitLimitNs,
+                            /*stop_on_abort=*/false)) {
             ok = false;
             break;
           }
@@ -1063,7 +1084,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       FusedQ q0;
       const int col0 = tc.nb * 256 + cbase;
       if (fused) fused_q_load(p.epi, fused_base(p.epi, tc.g, row0, col0, lane), 0, nlive, lane, q0);
-      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, kWaitLimitNs)) break;
+      if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, p.epi_wait_ns))
+        break;
       tc_fence_after();
       const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
                              (long long)row0 * p.ldc + (long long)col0;
@@ -1121,10 +1143,11 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
             for (int e = 0; e < 4; ++e) sc[e] = 0ull;   // +0.0f pairs
           }
         }
+        // like the producer, the converters stop only when a wait runs out (see there)
         bool got = wait_bounded(smem_u32(qfull + r), (uint32_t)(it / RAW) & 1u, ctl, kErrConvert,
-                                kWaitLimitNs);
+                                kWaitLimitNs, /*stop_on_abort=*/false);
         got = got && wait_bounded(smem_u32(empty + s), ((uint32_t)(it / STAGES) & 1u) ^ 1u, ctl,
-                                  kErrConvert, kWaitLimitNs);
+                                  kErrConvert, kWaitLimitNs, /*stop_on_abort=*/false);
         if (!__all_sync(0xffffffffu, got)) {
           ok = false;
           break;
@@ -1177,6 +1200,281 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
 
   tc_fence_before();
   cluster_sync_all();   // no remote arrive or copy may target a CTA that has left
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ wide CTA-pair kernel
+// The dense W0' products (B = A' W0', dA' = dB W0'^T) on 256 x 512 pair tiles: per 64-deep K
+// block each CTA loads 128 rows of A and 2 x 128 rows (N) of B, and the leader issues, for each
+// 16-deep K step, two 256 x 256 x 16 pair MMAs that share the A operand (the first may keep A in
+// the tensor core's collector buffer for the second). Per CTA and K block that is 48 KB of
+// operands for 128 x 512 outputs, against 32 KB for 128 x 256 on the 256 x 256 tiles: a quarter
+// less shared-memory traffic (TMA writes plus MMA operand reads) per MMA cycle, which is what
+// those tiles spend a fifth of their cycles waiting on.
+//   The accumulator is all 512 TMEM columns, as two 256-column halves with their own
+// "drained" barriers: the epilogue hands half 0 back first, and the MMA issuer starts the next
+// tile on half 0 alone, holding each stage until half 1 is back, then issues the held half-1
+// MMAs in K order and releases those stages. So the epilogue still overlaps the next main loop.
+//   Everything else (TMA on both CTAs completing the leader's full barrier, commits multicast to
+// both CTAs, bounded waits, bf16 epilogue through TMA stores, programmatic launch) is as in the
+// 256 x 256 kernel. A is K-major; B is K-major or N-major; one dense product (no groups, no
+// split K); bf16 output.
+struct WideCfg {
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = 128 * BK * 2;   // 16 KB
+  static constexpr int B_BYTES = 256 * BK * 2;   // 32 KB: N half 0 rows, then N half 1 rows
+  static constexpr int EPI_W = 4;
+  static constexpr int THREADS = 64 + 32 * EPI_W;
+  static constexpr size_t SMEM =
+      (size_t)STAGES * (A_BYTES + B_BYTES) + EPI_W * kEpiStageBytes + 1024 + 256;
+};
+
+// collector usage of the A operand: 0 = none, 1 = fill (keep A for the next MMA), 2 = last use
+template <int COLL>
+__device__ __forceinline__ void umma_bf16_pair_coll(uint32_t d_tmem, uint64_t a_desc,
+                                                    uint64_t b_desc, uint32_t idesc,
+                                                    uint32_t accumulate) {
+  if constexpr (COLL == 1) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16.collector::a::fill [%0], %1, %2, %3, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else if constexpr (COLL == 2) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16.collector::a::lastuse [%0], %1, %2, %3, p;\n\t}" ::"r"(
+            d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    umma_bf16_pair(d_tmem, a_desc, b_desc, idesc, accumulate);
+  }
+}
+
+template <bool B_MN>
+__device__ __forceinline__ uint64_t wide_b_desc(uint32_t b0, int half, int kk) {
+  const uint32_t base = b0 + (uint32_t)half * (128 * BK * 2);
+  return B_MN ? smem_desc(base + kk * 2048, 64 * BK * 2, 1024) : smem_desc(base + kk * 32, 16, 1024);
+}
+
+template <bool B_MN, bool COLLECT>
+__global__ void __launch_bounds__(WideCfg::THREADS, 1)
+umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
+                      const __grid_constant__ CUtensorMap tma_b,
+                      const __grid_constant__ CUtensorMap tma_c, const PairParams p) {
+  constexpr int STAGES = WideCfg::STAGES;
+  constexpr int A_BYTES = WideCfg::A_BYTES;
+  constexpr int B_BYTES = WideCfg::B_BYTES;
+  constexpr int EPI_W = WideCfg::EPI_W;
+  constexpr uint32_t TMEM_COLS = 512;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sa = smem;
+  uint8_t* sb = smem + STAGES * A_BYTES;
+  uint8_t* sepi = sb + STAGES * B_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + EPI_W * kEpiStageBytes);
+  uint64_t* full = bars;                   // leader only
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;     // one accumulator
+  uint64_t* tempty = tfull + 1;            // [2]: half 0, half 1 drained (leader only)
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const Ctl ctl{abort_flag, p.err};
+  const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
+  const int nk = (p.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    mbar_init(smem_u32(tfull), 1);
+    for (int h = 0; h < 2; ++h) mbar_init(smem_u32(tempty + h), 2 * EPI_W);
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0;
+      bool ok = true;
+      for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
+        const TileCoord tc = decode_pair_tile(p, tile);
+        const int am = tc.mb * 256 + (int)rank * 128;
+        const int bn = tc.nb * 512 + (int)rank * 128;   // N half h: rows bn + 256 h
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          // stops only when the wait runs out (see the 256 x 256 kernel's producer)
+          if (!wait_bounded(smem_u32(empty + s), ph ^ 1u, ctl, kErrProducer, kWaitLimitNs,
+                            /*stop_on_abort=*/false)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
+          if (leader) mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + B_BYTES));
+          const int k = kb * BK;
+          tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, k, am);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t dst = smem_u32(sb + s * B_BYTES + h * (128 * BK * 2));
+            if constexpr (B_MN) {
+              tma_load_2d_pair(dst, &tma_b, fb, bn + 256 * h, k);
+              tma_load_2d_pair(dst + 64 * BK * 2, &tma_b, fb, bn + 256 * h + 64, k);
+            } else {
+              tma_load_2d_pair(dst, &tma_b, fb, k, bn + 256 * h);
+            }
+          }
+        }
+      }
+      if (!ok && leader)
+        for (int j = max(0, it - STAGES); j < it; ++j)
+          wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
+                       kDrainLimitNs);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = instr_desc_pair<false, B_MN>();
+      int it = 0, tcount = 0;
+      bool ok = true;
+      // MMAs of one stage (iteration j, K block kb): halves h0..h1-1
+      auto issue = [&](int j, int kb, int h0, int h1) {
+        const int s = j % STAGES;
+        const uint32_t a0 = smem_u32(sa + s * A_BYTES), b0 = smem_u32(sb + s * B_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = smem_desc(a0 + kk * 32, 16, 1024);
+          const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+          if (h0 == 0 && h1 == 2 && COLLECT) {
+            umma_bf16_pair_coll<1>(tmem_base, ad, wide_b_desc<B_MN>(b0, 0, kk), idesc, acc);
+            umma_bf16_pair_coll<2>(tmem_base + 256, ad, wide_b_desc<B_MN>(b0, 1, kk), idesc, acc);
+          } else {
+            for (int h = h0; h < h1; ++h)
+              umma_bf16_pair(tmem_base + 256 * h, ad, wide_b_desc<B_MN>(b0, h, kk), idesc, acc);
+          }
+        }
+      };
+      for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
+        const uint32_t par = ((uint32_t)tcount & 1u) ^ 1u;   // previous tile's drain
+        if (!wait_bounded(smem_u32(tempty), par, ctl, kErrMma, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bool h1_free = false;
+        const int first = it;   // iteration of this tile's K block 0
+        int held = 0;           // K blocks 0..held-1 have their half-0 MMAs only
+        auto release_held = [&]() {
+          for (int kb = 0; kb < held; ++kb) {
+            issue(first + kb, kb, 1, 2);
+            umma_commit_pair_both(smem_u32(empty + (first + kb) % STAGES));
+          }
+          held = 0;
+        };
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          if (!wait_bounded<false>(smem_u32(full + s), (uint32_t)(it / STAGES) & 1u, ctl, kErrMma,
+                                   kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (!h1_free && mbar_test_wait(smem_u32(tempty + 1), par)) {
+            h1_free = true;
+            tc_fence_after();
+            release_held();
+          }
+          if (h1_free) {
+            issue(it, kb, 0, 2);
+            umma_commit_pair_both(smem_u32(empty + s));
+          } else {
+            issue(it, kb, 0, 1);
+            if (++held == STAGES) {
+              // every stage is held: wait for half 1 of the previous tile
+              if (!wait_bounded(smem_u32(tempty + 1), par, ctl, kErrMma, kWaitLimitNs)) {
+                ok = false;
+                break;
+              }
+              h1_free = true;
+              tc_fence_after();
+              release_held();
+            }
+          }
+        }
+        if (!ok) break;
+        if (!h1_free) {   // K shorter than the ring
+          if (!wait_bounded(smem_u32(tempty + 1), par, ctl, kErrMma, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          release_held();
+        }
+        umma_commit_pair_both(smem_u32(tfull));
+      }
+      umma_commit_pair_both(smem_u32(drain));
+      wait_bounded(smem_u32(drain), 0, ctl, ok ? kErrMma : 0, ok ? kWaitLimitNs : kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;
+    const uint32_t leader_tempty0 = map_to_rank(smem_u32(tempty), 0);
+    int tcount = 0, chunk = 0;
+    for (int tile = cluster_id; tile < p.total_tiles; tile += num_clusters, ++tcount) {
+      const TileCoord tc = decode_pair_tile(p, tile);
+      const int row0 = tc.mb * 256 + (int)rank * 128 + quarter * 32;
+      if (!wait_bounded(smem_u32(tfull), (uint32_t)tcount & 1u, ctl, kErrEpilogue, p.epi_wait_ns))
+        break;
+      tc_fence_after();
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        epilogue_tma_bf16(trow + (uint32_t)(256 * h), 256, sepi + (warp - 2) * kEpiStageBytes,
+                          &tma_c, tc.nb * 512 + 256 * h, row0, lane, chunk);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty0 + (uint32_t)(h * 8));
+      }
+    }
+    if (lane == 0) bulk_wait_all();
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
@@ -1271,6 +1569,7 @@ cudaError_t launch_t(const Gemm& g, cudaStream_t s, const char* name) {
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
   p.epi = g.epi;
   p.err = device_error_word();
+  p.epi_wait_ns = g.epi_wait_ns ? g.epi_wait_ns : kWaitLimitNs;
   auto kern = umma_gemm_kernel<BN, A_MN, B_MN, OUT_F32, STAGES>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1340,6 +1639,7 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   }
   p.epi = g.epi;
   p.err = device_error_word();
+  p.epi_wait_ns = g.epi_wait_ns ? g.epi_wait_ns : kWaitLimitNs;
   auto kern = umma_gemm_pair_kernel<A_MN, B_MN, OUT_F32, B_I8>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -1367,6 +1667,62 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   TraceScope t(name, s);
   e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, ta2, tb2, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <bool B_MN, bool COLLECT>
+cudaError_t launch_wide_t(const Gemm& g, cudaStream_t s, const char* name) {
+  constexpr size_t smem = WideCfg::SMEM;
+  CUtensorMap ta, tb, tc;
+  if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
+  if (!make_map(&tc, g.C, g.M, g.ldc, g.ldc, 32)) return cudaErrorInvalidValue;
+  PairParams p{};
+  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = 1; p.splits = 1; p.g2 = 1;
+  p.tiles_m = (int)((g.M + 255) / 256);
+  p.tiles_n = (int)(g.N / 512);
+  p.kblocks_per_split = (int)((g.K + BK - 1) / BK);
+  p.total_tiles = p.tiles_m * p.tiles_n;
+  p.nseg = 1; p.kb_per_seg = p.kblocks_per_split;
+  p.C = g.C; p.ldc = g.ldc;
+  // as for the 256 x 256 tiles: narrow N with a long K sweeps M under bands of pair-columns
+  // (the band's W0' columns stay in L2), otherwise bands of 16 pair-rows sweep N
+  p.raster = 0;
+  p.band = 16;
+  if (p.tiles_n <= 8 && p.tiles_m >= 32 && g.K >= 8192) {
+    p.raster = 1;
+    p.band = 8;
+  }
+  p.err = device_error_word();
+  p.epi_wait_ns = g.epi_wait_ns ? g.epi_wait_ns : kWaitLimitNs;
+  auto kern = umma_gemm_wide_kernel<B_MN, COLLECT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  set_pdl_attr(attr[1]);
+  cfg.blockDim = dim3(WideCfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;
+  if (!max_clusters) {
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess ||
+        max_clusters <= 0)
+      max_clusters = sm_count() / 2;
+  }
+  cfg.numAttrs = 2;
+  const int clusters = std::min(p.total_tiles, max_clusters);
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  TraceScope t(name, s);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1482,6 +1838,21 @@ cudaError_t gemm_pair(const Gemm& g, cudaStream_t s) {
   POETX_UP(false, true, true)
 #undef POETX_UP
   return cudaErrorNotSupported;
+}
+
+bool wide_supported(const Gemm& g) {
+  return supported(g) && !g.a_mn && !g.out_f32 && !g.b_i8 && !g.A2 && g.groups == 1 &&
+         g.splits == 1 && g.nseg == 1 && g.epi.mode == kEpiStore && g.N % 512 == 0 &&
+         g.M >= 256;
+}
+
+cudaError_t gemm_wide(const Gemm& g, cudaStream_t s) {
+  if (!wide_supported(g)) return cudaErrorNotSupported;
+  const char* name = g.name ? g.name : "umma_gemm_wide";
+  if (g.b_mn) return g.wide_collect ? launch_wide_t<true, true>(g, s, name)
+                                    : launch_wide_t<true, false>(g, s, name);
+  return g.wide_collect ? launch_wide_t<false, true>(g, s, name)
+                        : launch_wide_t<false, false>(g, s, name);
 }
 
 cudaError_t gemm(const Gemm& g, cudaStream_t s) {

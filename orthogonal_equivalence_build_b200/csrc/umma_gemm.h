@@ -61,6 +61,11 @@ struct Gemm {
   int64_t groups_1 = 0;
   const void* A2 = nullptr; int64_t a2_rows = 0, a2_cols = 0, a2_ld = 0;
   const void* B2 = nullptr; int64_t b2_rows = 0, b2_cols = 0, b2_ld = 0;
+  // Limit of the epilogue warps' wait for a finished accumulator, in ns (0: the kernels'
+  // default of a few seconds). Only the kernel-level test hook sets it, to make the wait run out.
+  unsigned long long epi_wait_ns = 0;
+  // 256 x 512 kernel only: the two MMAs of a K step share A through the collector buffer
+  bool wide_collect = true;
 };
 
 bool supported(const Gemm& g);
@@ -68,6 +73,10 @@ bool supported(const Gemm& g);
 // N % 256 == 0 and M >= 256.
 bool pair_supported(const Gemm& g);
 cudaError_t gemm_pair(const Gemm& g, cudaStream_t s);
+// Dense products (one group, no split K, A K-major, bf16 out) on 256 x 512 pair tiles with one
+// 512-column accumulator in two halves; needs N % 512 == 0 and M >= 256.
+bool wide_supported(const Gemm& g);
+cudaError_t gemm_wide(const Gemm& g, cudaStream_t s);
 
 // Number of K ranges the kernel actually uses for `splits` requested ranges over K
 // (ranges of whole 64-wide K blocks, none empty).

@@ -76,7 +76,7 @@ def _load() -> ctypes.CDLL:
         "poetx_last_error_message": (ctypes.c_char_p, []),
         "poetx_abi_version": (I32, []),
         "poetx_testing_gemm_bf16": (I32, [V, I64, I64, I32, V, I64, I64, I32, I64, I64, I64, V,
-                                          I32, I64, I32, I32, V]),
+                                          I32, I64, I32, I32, U64, V]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -312,13 +312,14 @@ def trace_read(maxlen: int = 1 << 20):
 
 def testing_gemm_bf16(a: torch.Tensor, a_mn: bool, b: torch.Tensor, b_mn: bool, M: int, N: int,
                       K: int, c: torch.Tensor, splits: int = 1, variant: int = 0,
-                      stream=None) -> None:
+                      epi_wait_ns: int = 0, stream=None) -> None:
     """Kernel-level hook (include/poetx_testing.h): C = A B on the tcgen05 kernel
-    (variant 0: single CTA, 1: CTA pair)."""
+    (variant 0: single CTA, 1: CTA pair); epi_wait_ns > 0 bounds the epilogue's accumulator
+    wait (a test of the timeout path)."""
     _check(lib.poetx_testing_gemm_bf16(_ptr(a), a.shape[0], a.shape[1], int(a_mn), _ptr(b),
                                        b.shape[0], b.shape[1], int(b_mn), M, N, K, _ptr(c),
                                        int(c.dtype == torch.float32), c.shape[-1], splits,
-                                       variant, _stream(stream)))
+                                       variant, int(epi_wait_ns), _stream(stream)))
 
 
 def abi_version() -> int:

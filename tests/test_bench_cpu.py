@@ -42,3 +42,19 @@ def test_reference_config_is_the_gpu_arms_config():
         d = _run("--workload", key)
         args = types.SimpleNamespace(tokens=None, all_linears=True, xq=False, xq_staged=False)
         assert d["config"] == bench.workload_config(W.WORKLOADS[key], args, 1), key
+
+
+def test_cpu_baseline_reports_one_thread_blas_and_merge_extrapolation():
+    """The oracle baseline carries the BLAS library, a 1-thread figure of the same sample and,
+    for a workload with a merge period, the step plus one merge_reinit spread over the period,
+    labelled as an extrapolation."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import poetx_workloads as W
+    wl = W.WORKLOADS["tiny_fp32"]   # merge_reinit every step
+    cb = bench.cpu_baseline(wl, 16, 1)
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["blas"]
+    assert cb["one_thread"]["value"] > 0 and "1 BLAS thread" in cb["one_thread"]["sample"]
+    ex = cb["extrapolated_with_merge"]
+    assert ex["merge_reinit_s"] > 0 and "extrapolated" in ex["label"]
+    assert 0 < ex["value"] < cb["value"]

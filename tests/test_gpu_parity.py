@@ -110,10 +110,12 @@ def test_permutation_weight_is_bit_exact(key, m, b, T):
 
 
 # ------------------------------------------------------------------ layer parity
-def _check_layer(c: LayerCase, tol: float, rows=None):
+def _check_layer(c: LayerCase, tol: float, xmem: bool = False):
+    """Y, dX, dq_r, dq_p of the library against the oracle on the same inputs. xmem: the
+    backward runs without the saved B (memory-saving mode: B is rebuilt inside the call)."""
     h = c.host()
     y, bsave = c.forward()
-    dx, dq_r, dq_p = c.backward(bsave)
+    dx, dq_r, dq_p = c.backward(None if xmem else bsave)
     torch.cuda.synchronize()
     G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
     ref = O.linear_bwd(h["X"], h["dY"], h["W0m"], h["perm_r"], h["perm_p"], G_r, G_p,
@@ -123,6 +125,14 @@ def _check_layer(c: LayerCase, tol: float, rows=None):
     for k, e in errs.items():
         assert e <= tol, (k, errs)
     return errs
+
+
+def tile_rows(T: int, seed: int, tile: int = 128) -> np.ndarray:
+    """One random token row in every `tile`-row band of the T rows, plus the last row: every
+    row tile of the products (and the ragged last band) is represented."""
+    rng = np.random.default_rng(seed)
+    rows = [t0 + int(rng.integers(0, min(tile, T - t0))) for t0 in range(0, T, tile)]
+    return np.unique(np.array(rows + [T - 1]))
 
 
 def test_fp32_layer_full_tiny_workload():
@@ -146,6 +156,18 @@ def test_fp32_layer_shapes(m, n, b, T):
 ])
 def test_bf16_layer_parity(key, m, n, b, T):
     _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), TOL_BF16)
+
+
+@pytest.mark.parametrize("key,m,n,b,T,tol", [
+    ("llama8b_up_proj", 1024, 2048, 512, 2305, TOL_BF16),
+    ("llama1p3b_attn", 1024, 1024, 256, 333, TOL_BF16),
+    ("llama1p3b_attn", 512, 768, 128, 129, TOL_BF16),
+    ("tiny_fp32", 512, 768, 64, 100, TOL_F32),
+])
+def test_memory_saving_backward_matches_oracle(key, m, n, b, T, tol):
+    """POET-Xmem: the backward without the saved B (rebuilt inside the call) against the
+    oracle's exact gradient, not only against the saved-B backward."""
+    _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), tol, xmem=True)
 
 
 # ------------------------------------------------------------------ merge-then-reinitialize
@@ -173,11 +195,12 @@ def test_merge_reinit_matches_oracle(key, m, n, b, tol):
 # ------------------------------------------------------------------ full-size sampled checks
 @pytest.mark.parametrize("key", ["llama1p3b_attn", "llama8b_up_proj"])
 def test_full_size_sampled(key):
-    """Full workload sizes: sampled token rows of Y and dX against the oracle row by row, and
-    dq against the oracle restricted to the sampled rows (dY is zero elsewhere)."""
+    """Full workload sizes: one token row in every 128-row tile (and the last row) of Y and dX
+    against the oracle row by row, and dq against the oracle restricted to those rows (dY is
+    zero elsewhere)."""
     c = LayerCase(key)
     h = c.host()
-    rows = np.sort(np.random.default_rng(0).choice(c.T, 12, replace=False))
+    rows = tile_rows(c.T, 0)
     G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
     y, bsave = c.forward()
     dx, _, _ = c.backward(bsave)
@@ -196,6 +219,48 @@ def test_full_size_sampled(key):
                        h["q_p"], c.b)
     assert rel_err(dq_r, ref["dq_r"]) <= TOL_BF16
     assert rel_err(dq_p, ref["dq_p"]) <= TOL_BF16
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("key", ["llama1p3b_attn", "llama8b_up_proj"])
+def test_full_size_dense_every_row_and_dq(key):
+    """Full workload size with dense dY: every row of Y and dX, and dq_r / dq_p, against the
+    oracle, for the saved-B backward and for the memory-saving one (saved_b = None). The
+    oracle streams the tokens in chunks: Y and dX of a token depend on that token only, and
+    dG = sum over tokens of A_t^T dA'_t (B_t^T dC_t) is additive over chunks, so the chunks'
+    dG are summed and dq is the CNP chain rule of the sum (dq is linear in dG)."""
+    c = LayerCase(key)
+    h = c.host()
+    G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
+    y, bsave = c.forward()
+    dx, dq_r, dq_p = c.backward(bsave)
+    dx_m, dq_r_m, dq_p_m = c.backward(None)
+    torch.cuda.synchronize()
+    num = {k: 0.0 for k in ("y", "dx", "dx_xmem")}
+    den = {k: 0.0 for k in ("y", "dx")}
+    dG_r = dG_p = 0.0
+    chunk = 4096
+    for t0 in range(0, c.T, chunk):
+        sl = slice(t0, min(c.T, t0 + chunk))
+        ref = O.linear_bwd(h["X"][sl], h["dY"][sl], h["W0m"], h["perm_r"], h["perm_p"], G_r,
+                           G_p, h["q_r"], h["q_p"], c.b)
+        dG_r = dG_r + ref["dG_r"]
+        dG_p = dG_p + ref["dG_p"]
+        # (error name, reference name, device rows, oracle rows)
+        for name, rname, gpu, want in (("y", "y", y[sl], ref["Y"]), ("dx", "dx", dx[sl], ref["dX"]),
+                                       ("dx_xmem", "dx", dx_m[sl], ref["dX"])):
+            g = gpu.double().cpu().numpy()
+            num[name] = max(num[name], float(np.max(np.abs(g - want))))
+            den[rname] = max(den[rname], float(np.max(np.abs(want))))
+        del ref
+    errs = {"y": num["y"] / den["y"], "dx": num["dx"] / den["dx"],
+            "dx_xmem": num["dx_xmem"] / den["dx"]}
+    dq_r_ref = O.dq_from_dG(dG_r, h["q_r"], c.b)
+    dq_p_ref = O.dq_from_dG(dG_p, h["q_p"], c.b)
+    errs.update({"dq_r": rel_err(dq_r, dq_r_ref), "dq_p": rel_err(dq_p, dq_p_ref),
+                 "dq_r_xmem": rel_err(dq_r_m, dq_r_ref), "dq_p_xmem": rel_err(dq_p_m, dq_p_ref)})
+    for k, e in errs.items():
+        assert e <= TOL_BF16, (k, errs)
 
 
 # ------------------------------------------------------------------ layer-level CNP and one-sided dq
@@ -257,7 +322,7 @@ def test_backward_without_saved_b_is_identical(key, m, n, b, T):
 def test_full_size_sampled_other_linears(key, layer):
     c = LayerCase(key, layer)
     h = c.host()
-    rows = np.sort(np.random.default_rng(layer).choice(c.T, 8, replace=False))
+    rows = tile_rows(c.T, layer)
     G_r, G_p = O.cnp(h["q_r"], c.b), O.cnp(h["q_p"], c.b)
     y, bsave = c.forward()
     dy_sparse = torch.zeros_like(c.dy)

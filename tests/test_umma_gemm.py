@@ -98,3 +98,70 @@ def test_umma_pair_gemm_split_k_and_identity():
         poetx.testing_gemm_bf16(A, False, eye, b_mn, 384, 256, 256, out, variant=1)
         torch.cuda.synchronize()
         assert torch.equal(out, A)
+
+
+# ------------------------------------------------------------------ bounded waits
+@pytest.mark.parametrize("variant,M,N", [(0, 128, 256), (1, 256, 256), (2, 256, 512)])
+def test_bounded_wait_runs_out_reports_timeout_and_recovers(variant, M, N):
+    """The error path of the bounded waits, made to run out without any fault: one output tile
+    (one CTA, or one CTA pair) with K = 131072, whose main loop runs for a fraction of a
+    millisecond, and the epilogue's wait for the finished accumulator limited to 1 us. The wait
+    expires; the epilogue records its code in the device error word and leaves, the producer
+    and the MMA issuer finish their copies and MMAs (one tile: neither waits for an accumulator
+    the epilogue would hand back), TMEM is freed and the kernel returns. poetx_device_status
+    then reports POETX_ERR_TIMEOUT once and clears the word, and the next product on the same
+    context is correct."""
+    poetx.device_status()
+    K = 131072
+    g = torch.Generator(device="cpu").manual_seed(variant)
+    a = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    b = torch.randn(N, K, generator=g).to(torch.bfloat16).cuda()   # K-major B
+    c = torch.zeros(M, N, device="cuda", dtype=torch.bfloat16)
+    poetx.testing_gemm_bf16(a, False, b, False, M, N, K, c, variant=variant, epi_wait_ns=1000)
+    torch.cuda.synchronize()    # the kernel returned
+    with pytest.raises(poetx.PoetxError) as e:
+        poetx.device_status()
+    assert e.value.status == 9 and "259" in str(e.value), str(e.value)   # 0x103: epilogue wait
+    poetx.device_status()       # cleared
+    # a normal product afterwards: same kernel, default wait limit
+    Ks = 1024
+    a2, b2, ref = _operands(M, N, Ks, False, False, seed=11 + variant)
+    f32 = variant != 2   # the 256 x 512 kernel writes bf16 only
+    c2 = torch.empty(M, N, device="cuda", dtype=torch.float32 if f32 else torch.bfloat16)
+    poetx.testing_gemm_bf16(a2, False, b2, False, M, N, Ks, c2, variant=variant)
+    torch.cuda.synchronize()
+    poetx.device_status()
+    err = (c2.float().cpu() - ref).abs().max().item() / ref.abs().max().item()
+    assert err < (2e-6 * Ks ** 0.5 if f32 else 6e-3), err
+
+
+# ------------------------------------------------------------------ 256 x 512 pair tiles
+@pytest.mark.parametrize("variant", [2, 3])
+@pytest.mark.parametrize("b_mn", [False, True])
+@pytest.mark.parametrize("M,N,K", [(256, 512, 64), (300, 1024, 192), (1000, 512, 1024),
+                                   (4096, 5120, 128), (4000, 5120, 2048)])
+def test_umma_wide_gemm_matches_fp32_matmul_and_pair_kernel(variant, b_mn, M, N, K):
+    """The dense kernel on 256 x 512 pair tiles (with and without the shared A collector)
+    against an fp32 matmul, and bit for bit against the 256 x 256 pair kernel: both issue the
+    same 256 x 256 x 16 MMAs in the same K order per output element. The 4096 / 4000-row cases
+    give each cluster several tiles, so the accumulator halves are handed back and reused while
+    the next tile starts; K = 128 is shorter than the stage ring; M = 300, 1000, 4000 are ragged."""
+    a, b, ref = _operands(M, N, K, False, b_mn, seed=M + N + K + variant)
+    c = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    poetx.testing_gemm_bf16(a, False, b, b_mn, M, N, K, c, variant=variant)
+    c1 = torch.empty(M, N, device="cuda", dtype=torch.bfloat16)
+    poetx.testing_gemm_bf16(a, False, b, b_mn, M, N, K, c1, variant=1)
+    torch.cuda.synchronize()
+    poetx.device_status()
+    err = (c.float().cpu() - ref).abs().max().item() / ref.abs().max().item()
+    assert err < 6e-3, err
+    assert torch.equal(c, c1)
+
+
+def test_umma_wide_rejects_narrow_n():
+    a = torch.zeros(256, 64, dtype=torch.bfloat16, device="cuda")
+    b = torch.zeros(768, 64, dtype=torch.bfloat16, device="cuda")
+    c = torch.zeros(256, 768, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(poetx.PoetxError) as e:
+        poetx.testing_gemm_bf16(a, False, b, False, 256, 768, 64, c, variant=2)
+    assert e.value.status == 7
