@@ -107,6 +107,30 @@ def sum_over_ranks_(flat, group=None):
     return flat
 
 
+class DqReducer:
+    """Data-parallel sum of the packed dq gradients, one asynchronous all-reduce per linear,
+    issued as soon as that linear's backward is enqueued: the collective then runs on the
+    communicator's own stream while the next linear's kernels run, and finish() makes the
+    caller's stream (NCCL) or the caller (gloo) wait for all of them before the step ends. Every
+    rank issues the same collectives in the same order: linear 0, 1, ...  With one rank it does
+    nothing."""
+
+    def __init__(self, group=None):
+        self.group = group
+        self.works = []
+
+    def add(self, flat):
+        import torch.distributed as dist
+        if dist.is_initialized() and dist.get_world_size(self.group) > 1:
+            self.works.append(dist.all_reduce(flat, op=dist.ReduceOp.SUM, group=self.group,
+                                              async_op=True))
+
+    def finish(self):
+        for w in self.works:
+            w.wait()
+        self.works.clear()
+
+
 def max_over_ranks(value: float, device=None, group=None) -> float:
     """The job's time is the slowest rank's."""
     import torch
@@ -383,47 +407,39 @@ def run_ours(args):
         d["y"] = torch.empty(T, lin.n, dtype=dt, device=dev)
         d["bsave"] = torch.empty(T, lin.n, dtype=dt, device=dev)
         d["dx"] = torch.empty(T, lin.m, dtype=dt, device=dev)
-        d["dq_r"] = torch.empty_like(L.q_r)
-        d["dq_p"] = torch.empty_like(L.q_p)
+        # dq_r and dq_p are views of one packed buffer: one all-reduce per linear (N > 1)
+        d["dq"] = torch.empty(L.q_r.numel() + L.q_p.numel(), device=dev)
+        d["dq_r"] = d["dq"][:L.q_r.numel()].view_as(L.q_r)
+        d["dq_p"] = d["dq"][L.q_r.numel():].view_as(L.q_p)
         layers.append(d)
         poetx.layer_cnp_build(L)
     ws = torch.empty(max(max(poetx.fwd_workspace_bytes(d["layer"], T),
                              poetx.bwd_workspace_bytes(d["layer"], T),
                              poetx.layer_cnp_workspace_bytes(d["layer"])) for d in layers),
                      dtype=torch.uint8, device=dev)
-    ndq = sum(d["dq_r"].numel() + d["dq_p"].numel() for d in layers)
-    flat_dq = torch.empty(ndq, device=dev) if world > 1 else None
+    reducer = DqReducer()
     stream = torch.cuda.current_stream(dev)
     in_bytes = sum((d["x"].numel() + d["dy"].numel()) * esz for d in layers)
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if in_bytes <= L2_BYTES else None
 
     def step(xs=None, dys=None, outs=None):
-        """One step over every linear; outs[i] = (y, dx, dq_r, dq_p) of linear i (default:
-        the layer's own result buffers)."""
+        """One step over every linear; outs[i] = (y, dx, dq) of linear i, dq the packed
+        [dq_r, dq_p] (default: the layer's own result buffers). With N > 1 each linear's dq is
+        summed over the ranks by an all-reduce issued right after its backward, overlapping
+        the next linear's kernels."""
         for i, d in enumerate(layers):
             L = d["layer"]
             xin = d["x"] if xs is None else xs[i]
             dyin = d["dy"] if dys is None else dys[i]
-            y, dx, dq_r, dq_p = ((d["y"], d["dx"], d["dq_r"], d["dq_p"]) if outs is None
-                                 else outs[i])
+            y, dx, dq = (d["y"], d["dx"], d["dq"]) if outs is None else outs[i]
+            nr = L.q_r.numel()
             if wl.cnp_in_step:
                 poetx.layer_cnp_build(L, ws)
             poetx.linear_fwd(L, xin, y, d["bsave"], ws)
-            poetx.linear_bwd(L, xin, dyin, d["bsave"], dx, dq_r, dq_p, ws)
-        if world > 1:
-            o = 0
-            for i, d in enumerate(layers):
-                dqs = (d["dq_r"], d["dq_p"]) if outs is None else outs[i][2:]
-                for t in dqs:
-                    flat_dq[o:o + t.numel()].copy_(t.view(-1))
-                    o += t.numel()
-            sum_over_ranks_(flat_dq)
-            o = 0
-            for i, d in enumerate(layers):
-                dqs = (d["dq_r"], d["dq_p"]) if outs is None else outs[i][2:]
-                for t in dqs:
-                    t.view(-1).copy_(flat_dq[o:o + t.numel()])
-                    o += t.numel()
+            poetx.linear_bwd(L, xin, dyin, d["bsave"], dx, dq[:nr].view_as(L.q_r),
+                             dq[nr:].view_as(L.q_p), ws)
+            reducer.add(dq)
+        reducer.finish()
 
     def barrier():
         if world > 1:
@@ -531,14 +547,13 @@ def run_ours(args):
     # after the last step's results are in host memory.
     out_host = [(torch.empty(T, d["lin"].n, dtype=dt).pin_memory(),
                  torch.empty(T, d["lin"].m, dtype=dt).pin_memory(),
-                 torch.empty(d["dq_r"].shape, dtype=torch.float32).pin_memory(),
-                 torch.empty(d["dq_p"].shape, dtype=torch.float32).pin_memory())
+                 torch.empty(d["dq"].shape, dtype=torch.float32).pin_memory())
                 for d in layers]
     bufs = [([torch.empty_like(d["x"]) for d in layers], [torch.empty_like(d["dy"]) for d in layers])
             for _ in range(2)]
-    outs = [[(d["y"], d["dx"], d["dq_r"], d["dq_p"]) if k == 0 else
-             (torch.empty_like(d["y"]), torch.empty_like(d["dx"]), torch.empty_like(d["dq_r"]),
-              torch.empty_like(d["dq_p"])) for d in layers] for k in range(2)]
+    outs = [[(d["y"], d["dx"], d["dq"]) if k == 0 else
+             (torch.empty_like(d["y"]), torch.empty_like(d["dx"]), torch.empty_like(d["dq"]))
+             for d in layers] for k in range(2)]
     h2d_stream = torch.cuda.Stream(dev)
     d2h_stream = torch.cuda.Stream(dev)
     copied = [torch.cuda.Event() for _ in range(2)]

@@ -37,12 +37,30 @@ cudaError_t run(const umma::Gemm& g, cudaStream_t s) {
   return umma::gemm(g, s);
 }
 
+// The dense W0' products: 256 x 512 pair tiles where N allows (every workload's m and n are
+// multiples of 512), else as above.
+cudaError_t run_dense(const umma::Gemm& g, cudaStream_t s) {
+  if (umma::wide_supported(g)) return umma::gemm_wide(g, s);
+  return run(g, s);
+}
+
+}  // namespace
+
+namespace {
+// The per-block gradients run on 256 x 512 pair tiles where b is a multiple of 512 (one tile per
+// 256 rows of a block), on 256 x 256 pair tiles where b % 256 == 0, else on single-CTA tiles.
+bool dg_wide(int64_t b) { return b % 512 == 0; }
+// CTAs that one split of one block occupies
+int64_t dg_ctas_per_block(int64_t b) {
+  if (dg_wide(b)) return (b / 256) * (b / 512) * 2;
+  return ((b + 127) / 128) * std::max<int64_t>(1, b / 256);
+}
 }  // namespace
 
 int grad_splits(int64_t nb, int64_t b, int64_t rows) {
   // Split the contraction over tokens so the (group, tile, split) work units fill whole waves of
   // the persistent grid (all units cost the same); each split keeps >= 512 token rows.
-  const int64_t tiles = nb * ((b + 127) / 128) * std::max<int64_t>(1, b / 256);
+  const int64_t tiles = nb * dg_ctas_per_block(b);
   const int64_t waves_unit = sms();
   const int64_t max_s = std::max<int64_t>(1, std::min<int64_t>(16, rows / 512));
   int best = 1;
@@ -114,7 +132,7 @@ cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, i
     else { g.b_rows = K; g.b_cols = N; g.b_ld = N; g.b_mn = true; }
     g.C = C; g.ldc = N;
     g.name = w_trans ? "umma_dense_W0T" : "umma_dense_W0";
-    if (umma::supported(g)) return run(g, s);
+    if (umma::supported(g)) return run_dense(g, s);
   }
   SimtGemm g{};
   g.M = M; g.N = N; g.K = K; g.batch = 1;
@@ -174,6 +192,7 @@ cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64
     g.name = "umma_block_grad";
     if (b % 128 == 0 && umma::supported(g) && (sp == 1 || partials)) {
       *splits_used = sp;
+      if (dg_wide(b) && umma::wide_supported(g)) return umma::gemm_wide(g, s);
       return run(g, s);
     }
   }
@@ -221,6 +240,10 @@ cudaError_t gemm_block_grad2(DT t, const void* A1, const void* B1, int64_t w1, c
   if (sp > 1 && !partials) return cudaErrorNotSupported;
   umma::Gemm g = block_grad2_gemm(A1, B1, w1, A2, B2, w2, rows, b, sp);
   g.C = sp > 1 ? partials : dG;
+  if (dg_wide(b) && umma::wide_supported(g)) {
+    *splits_used = sp;
+    return umma::gemm_wide(g, s);
+  }
   if (!umma::pair_supported(g)) return cudaErrorNotSupported;
   *splits_used = sp;
   return umma::gemm_pair(g, s);

@@ -1222,8 +1222,9 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
 // MMAs in K order and releases those stages. So the epilogue still overlaps the next main loop.
 //   Everything else (TMA on both CTAs completing the leader's full barrier, commits multicast to
 // both CTAs, bounded waits, bf16 epilogue through TMA stores, programmatic launch) is as in the
-// 256 x 256 kernel. A is K-major; B is K-major or N-major; one dense product (no groups, no
-// split K); bf16 output.
+// 256 x 256 kernel. Operand layouts, groups (per-group coordinate offsets, a second operand
+// pair), split K and fp32 outputs are those of the 256 x 256 kernel: the b = 512 blocks take one
+// 512-wide tile per block and row tile, the per-block gradients one per block and M half.
 struct WideCfg {
   static constexpr int STAGES = 4;
   static constexpr int A_BYTES = 128 * BK * 2;   // 16 KB
@@ -1266,11 +1267,18 @@ __device__ __forceinline__ uint64_t wide_b_desc(uint32_t b0, int half, int kk) {
   return B_MN ? smem_desc(base + kk * 2048, 64 * BK * 2, 1024) : smem_desc(base + kk * 32, 16, 1024);
 }
 
-template <bool B_MN, bool COLLECT>
+template <bool A_MN>
+__device__ __forceinline__ uint64_t wide_a_desc(uint32_t a0, int kk) {
+  return A_MN ? smem_desc(a0 + kk * 2048, 64 * BK * 2, 1024) : smem_desc(a0 + kk * 32, 16, 1024);
+}
+
+template <bool A_MN, bool B_MN, bool OUT_F32, bool COLLECT>
 __global__ void __launch_bounds__(WideCfg::THREADS, 1)
 umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b,
-                      const __grid_constant__ CUtensorMap tma_c, const PairParams p) {
+                      const __grid_constant__ CUtensorMap tma_c,
+                      const __grid_constant__ CUtensorMap tma_a2,
+                      const __grid_constant__ CUtensorMap tma_b2, const PairParams p) {
   constexpr int STAGES = WideCfg::STAGES;
   constexpr int A_BYTES = WideCfg::A_BYTES;
   constexpr int B_BYTES = WideCfg::B_BYTES;
@@ -1296,7 +1304,7 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
   const bool leader = rank == 0;
   const Ctl ctl{abort_flag, p.err};
   const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
-  const int nk = (p.K + BK - 1) / BK;
+  const int nk_all = (p.K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -1330,9 +1338,17 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
       bool ok = true;
       for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
         const TileCoord tc = decode_pair_tile(p, tile);
-        const int am = tc.mb * 256 + (int)rank * 128;
-        const int bn = tc.nb * 512 + (int)rank * 128;   // N half h: rows bn + 256 h
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int kb0 = tc.split * p.kblocks_per_split;
+        const int kb1 = min(kb0 + p.kblocks_per_split, nk_all);
+        // groups from g2 on come from the second operand pair, counted from its first group
+        const bool second = tc.g >= p.g2;
+        const CUtensorMap* map_a = second ? &tma_a2 : &tma_a;
+        const CUtensorMap* map_b = second ? &tma_b2 : &tma_b;
+        const int gl = second ? tc.g - p.g2 : tc.g;
+        const int am = gl * p.a_gm + tc.mb * 256 + (int)rank * 128, ak = gl * p.a_gk;
+        // N half h: rows (K-major B) or columns (N-major B) bn + 256 h
+        const int bn = gl * p.b_gn + tc.nb * 512 + (int)rank * 128, bk = gl * p.b_gk;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           // stops only when the wait runs out (see the 256 x 256 kernel's producer)
@@ -1344,15 +1360,21 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
           const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
           if (leader) mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + B_BYTES));
           const int k = kb * BK;
-          tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, k, am);
+          const uint32_t da = smem_u32(sa + s * A_BYTES);
+          if constexpr (A_MN) {
+            tma_load_2d_pair(da, map_a, fb, am, ak + k);
+            tma_load_2d_pair(da + 64 * BK * 2, map_a, fb, am + 64, ak + k);
+          } else {
+            tma_load_2d_pair(da, map_a, fb, ak + k, am);
+          }
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
             const uint32_t dst = smem_u32(sb + s * B_BYTES + h * (128 * BK * 2));
             if constexpr (B_MN) {
-              tma_load_2d_pair(dst, &tma_b, fb, bn + 256 * h, k);
-              tma_load_2d_pair(dst + 64 * BK * 2, &tma_b, fb, bn + 256 * h + 64, k);
+              tma_load_2d_pair(dst, map_b, fb, bn + 256 * h, bk + k);
+              tma_load_2d_pair(dst + 64 * BK * 2, map_b, fb, bn + 256 * h + 64, bk + k);
             } else {
-              tma_load_2d_pair(dst, &tma_b, fb, k, bn + 256 * h);
+              tma_load_2d_pair(dst, map_b, fb, bk + k, bn + 256 * h);
             }
           }
         }
@@ -1366,17 +1388,17 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader)
     if (leader && lane == 0) {
-      constexpr uint32_t idesc = instr_desc_pair<false, B_MN>();
+      constexpr uint32_t idesc = instr_desc_pair<A_MN, B_MN>();
       int it = 0, tcount = 0;
       bool ok = true;
-      // MMAs of one stage (iteration j, K block kb): halves h0..h1-1
-      auto issue = [&](int j, int kb, int h0, int h1) {
+      // MMAs of one stage (iteration j, i-th K block of the tile): halves h0..h1-1
+      auto issue = [&](int j, int i, int h0, int h1) {
         const int s = j % STAGES;
         const uint32_t a0 = smem_u32(sa + s * A_BYTES), b0 = smem_u32(sb + s * B_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
-          const uint64_t ad = smem_desc(a0 + kk * 32, 16, 1024);
-          const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+          const uint64_t ad = wide_a_desc<A_MN>(a0, kk);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
           if (h0 == 0 && h1 == 2 && COLLECT) {
             umma_bf16_pair_coll<1>(tmem_base, ad, wide_b_desc<B_MN>(b0, 0, kk), idesc, acc);
             umma_bf16_pair_coll<2>(tmem_base + 256, ad, wide_b_desc<B_MN>(b0, 1, kk), idesc, acc);
@@ -1387,6 +1409,9 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
         }
       };
       for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
+        const TileCoord tc = decode_pair_tile(p, tile);
+        const int kb0 = tc.split * p.kblocks_per_split;
+        const int nk = min(kb0 + p.kblocks_per_split, nk_all) - kb0;
         const uint32_t par = ((uint32_t)tcount & 1u) ^ 1u;   // previous tile's drain
         if (!wait_bounded(smem_u32(tempty), par, ctl, kErrMma, kWaitLimitNs)) {
           ok = false;
@@ -1394,16 +1419,16 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
         }
         tc_fence_after();
         bool h1_free = false;
-        const int first = it;   // iteration of this tile's K block 0
-        int held = 0;           // K blocks 0..held-1 have their half-0 MMAs only
+        const int first = it;   // iteration of this tile's first K block
+        int held = 0;           // the tile's K blocks 0..held-1 have their half-0 MMAs only
         auto release_held = [&]() {
-          for (int kb = 0; kb < held; ++kb) {
-            issue(first + kb, kb, 1, 2);
-            umma_commit_pair_both(smem_u32(empty + (first + kb) % STAGES));
+          for (int i = 0; i < held; ++i) {
+            issue(first + i, i, 1, 2);
+            umma_commit_pair_both(smem_u32(empty + (first + i) % STAGES));
           }
           held = 0;
         };
-        for (int kb = 0; kb < nk; ++kb, ++it) {
+        for (int i = 0; i < nk; ++i, ++it) {
           const int s = it % STAGES;
           if (!wait_bounded<false>(smem_u32(full + s), (uint32_t)(it / STAGES) & 1u, ctl, kErrMma,
                                    kWaitLimitNs)) {
@@ -1417,10 +1442,10 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
             release_held();
           }
           if (h1_free) {
-            issue(it, kb, 0, 2);
+            issue(it, i, 0, 2);
             umma_commit_pair_both(smem_u32(empty + s));
           } else {
-            issue(it, kb, 0, 1);
+            issue(it, i, 0, 1);
             if (++held == STAGES) {
               // every stage is held: wait for half 1 of the previous tile
               if (!wait_bounded(smem_u32(tempty + 1), par, ctl, kErrMma, kWaitLimitNs)) {
@@ -1460,17 +1485,30 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
         break;
       tc_fence_after();
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      // a group's output starts c_gs elements on: a column offset, or whole rows
+      const long long goff = (long long)tc.g * p.c_gs;
+      const int gx = (int)(goff % p.ldc), gy = (int)(goff / p.ldc);
+      const long long off0 = (long long)tc.split * p.c_split + goff + (long long)row0 * p.ldc +
+                             (long long)tc.nb * 512;
+      const int nlive = max(0, min(32, p.M - row0));
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        epilogue_tma_bf16(trow + (uint32_t)(256 * h), 256, sepi + (warp - 2) * kEpiStageBytes,
-                          &tma_c, tc.nb * 512 + 256 * h, row0, lane, chunk);
+        if constexpr (OUT_F32)
+          epilogue_warp_rows<true>(trow + (uint32_t)(256 * h), 256,
+                                   sepi + (warp - 2) * kEpiStageBytes, p.C, off0 + 256 * h, p.ldc,
+                                   nlive, lane);
+        else
+          epilogue_tma_bf16(trow + (uint32_t)(256 * h), 256, sepi + (warp - 2) * kEpiStageBytes,
+                            &tma_c, gx + tc.nb * 512 + 256 * h, gy + row0, lane, chunk);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty0 + (uint32_t)(h * 8));
       }
     }
-    if (lane == 0) bulk_wait_all();
-    __syncwarp();
+    if constexpr (!OUT_F32) {
+      if (lane == 0) bulk_wait_all();
+      __syncwarp();
+    }
   }
 
   tc_fence_before();
@@ -1671,32 +1709,48 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   return cudaGetLastError();
 }
 
-template <bool B_MN, bool COLLECT>
+template <bool A_MN, bool B_MN, bool OUT_F32, bool COLLECT>
 cudaError_t launch_wide_t(const Gemm& g, cudaStream_t s, const char* name) {
   constexpr size_t smem = WideCfg::SMEM;
-  CUtensorMap ta, tb, tc;
-  if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, 128)) return cudaErrorInvalidValue;
+  CUtensorMap ta, tb;
+  if (!make_map(&ta, g.A, g.a_rows, g.a_cols, g.a_ld, A_MN ? BK : 128)) return cudaErrorInvalidValue;
   if (!make_map(&tb, g.B, g.b_rows, g.b_cols, g.b_ld, B_MN ? BK : 128)) return cudaErrorInvalidValue;
-  if (!make_map(&tc, g.C, g.M, g.ldc, g.ldc, 32)) return cudaErrorInvalidValue;
+  // bf16 C as a 2-D [rows][ldc] tensor holding exactly the rows the product owns (see
+  // launch_pair_t); fp32 outputs keep the thread stores and the map is unused
+  CUtensorMap tc = ta;
+  if constexpr (!OUT_F32) {
+    const int64_t crows = (g.c_gs % g.ldc == 0) ? (g.groups - 1) * (g.c_gs / g.ldc) + g.M : g.M;
+    if (!make_map(&tc, g.C, crows, g.ldc, g.ldc, 32)) return cudaErrorInvalidValue;
+  }
+  CUtensorMap ta2 = ta, tb2 = tb;
+  if (g.A2) {
+    if (!make_map(&ta2, g.A2, g.a2_rows, g.a2_cols, g.a2_ld, A_MN ? BK : 128) ||
+        !make_map(&tb2, g.B2, g.b2_rows, g.b2_cols, g.b2_ld, B_MN ? BK : 128))
+      return cudaErrorInvalidValue;
+  }
   PairParams p{};
-  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = 1; p.splits = 1; p.g2 = 1;
+  p.M = (int)g.M; p.N = (int)g.N; p.K = (int)g.K; p.groups = (int)g.groups;
+  p.g2 = g.A2 ? (int)g.groups_1 : (int)g.groups;
   p.tiles_m = (int)((g.M + 255) / 256);
   p.tiles_n = (int)(g.N / 512);
-  p.kblocks_per_split = (int)((g.K + BK - 1) / BK);
-  p.total_tiles = p.tiles_m * p.tiles_n;
+  const int kblocks = (int)((g.K + BK - 1) / BK);
+  p.splits = effective_splits(g.K, g.splits);
+  p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
+  p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
+  p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
   p.nseg = 1; p.kb_per_seg = p.kblocks_per_split;
-  p.C = g.C; p.ldc = g.ldc;
+  p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
   // as for the 256 x 256 tiles: narrow N with a long K sweeps M under bands of pair-columns
-  // (the band's W0' columns stay in L2), otherwise bands of 16 pair-rows sweep N
+  // (the band's W0' columns stay in L2), otherwise bands of pair-rows sweep N
   p.raster = 0;
-  p.band = 16;
-  if (p.tiles_n <= 8 && p.tiles_m >= 32 && g.K >= 8192) {
+  p.band = p.groups == 1 ? 16 : 8;
+  if (p.groups == 1 && p.splits == 1 && p.tiles_n <= 8 && p.tiles_m >= 32 && g.K >= 8192) {
     p.raster = 1;
     p.band = 8;
   }
   p.err = device_error_word();
   p.epi_wait_ns = g.epi_wait_ns ? g.epi_wait_ns : kWaitLimitNs;
-  auto kern = umma_gemm_wide_kernel<B_MN, COLLECT>;
+  auto kern = umma_gemm_wide_kernel<A_MN, B_MN, OUT_F32, COLLECT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1722,7 +1776,7 @@ cudaError_t launch_wide_t(const Gemm& g, cudaStream_t s, const char* name) {
   const int clusters = std::min(p.total_tiles, max_clusters);
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   TraceScope t(name, s);
-  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, p);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, ta2, tb2, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -1841,18 +1895,46 @@ cudaError_t gemm_pair(const Gemm& g, cudaStream_t s) {
 }
 
 bool wide_supported(const Gemm& g) {
-  return supported(g) && !g.a_mn && !g.out_f32 && !g.b_i8 && !g.A2 && g.groups == 1 &&
-         g.splits == 1 && g.nseg == 1 && g.epi.mode == kEpiStore && g.N % 512 == 0 &&
-         g.M >= 256;
+  if (g.b_i8 || g.nseg != 1 || g.epi.mode != kEpiStore || g.N % 512 != 0 || g.M < 256)
+    return false;
+  if (g.A2) {
+    // a second operand pair: both sets valid operands of the same grouped product
+    Gemm h = g;
+    h.A = g.A2; h.a_rows = g.a2_rows; h.a_cols = g.a2_cols; h.a_ld = g.a2_ld;
+    h.B = g.B2; h.b_rows = g.b2_rows; h.b_cols = g.b2_cols; h.b_ld = g.b2_ld;
+    h.A2 = nullptr; h.B2 = nullptr;
+    h.groups = g.groups - g.groups_1;
+    Gemm f = g;
+    f.A2 = nullptr; f.B2 = nullptr;
+    f.groups = g.groups_1;
+    return g.B2 && g.groups_1 > 0 && g.groups_1 < g.groups && wide_supported(f) &&
+           wide_supported(h);
+  }
+  // operand layouts of the 256 x 256 kernel: A M-major only with B N-major and fp32 out
+  if (!supported(g) || (g.a_mn && !g.b_mn) || (g.a_mn && g.b_mn && !g.out_f32)) return false;
+  if (g.groups == 1) return true;
+  // groups: A's row offsets in whole pair tiles; bf16 output groups are column offsets inside
+  // one row (the output map's rows are the product's M) or whole rows
+  if (g.a_gm % 256) return false;
+  if (!g.out_f32 && g.c_gs % g.ldc != 0 &&
+      (g.c_gs >= g.ldc || (g.groups - 1) * g.c_gs + g.N > g.ldc))
+    return false;
+  return true;
 }
 
 cudaError_t gemm_wide(const Gemm& g, cudaStream_t s) {
   if (!wide_supported(g)) return cudaErrorNotSupported;
   const char* name = g.name ? g.name : "umma_gemm_wide";
-  if (g.b_mn) return g.wide_collect ? launch_wide_t<true, true>(g, s, name)
-                                    : launch_wide_t<true, false>(g, s, name);
-  return g.wide_collect ? launch_wide_t<false, true>(g, s, name)
-                        : launch_wide_t<false, false>(g, s, name);
+#define POETX_UW(AM, BMJ, F, C)                                        \
+  if (g.a_mn == AM && g.b_mn == BMJ && g.out_f32 == F && g.wide_collect == C) \
+    return launch_wide_t<AM, BMJ, F, C>(g, s, name);
+  POETX_UW(false, false, false, true)
+  POETX_UW(false, true, false, true)
+  POETX_UW(false, false, false, false)
+  POETX_UW(false, true, false, false)
+  POETX_UW(true, true, true, true)
+#undef POETX_UW
+  return cudaErrorNotSupported;
 }
 
 cudaError_t gemm(const Gemm& g, cudaStream_t s) {

@@ -73,8 +73,8 @@ bool supported(const Gemm& g);
 // N % 256 == 0 and M >= 256.
 bool pair_supported(const Gemm& g);
 cudaError_t gemm_pair(const Gemm& g, cudaStream_t s);
-// Dense products (one group, no split K, A K-major, bf16 out) on 256 x 512 pair tiles with one
-// 512-column accumulator in two halves; needs N % 512 == 0 and M >= 256.
+// Products without split K, A K-major, bf16 out (dense, or grouped as above) on 256 x 512 pair
+// tiles with one 512-column accumulator in two halves; needs N % 512 == 0 and M >= 256.
 bool wide_supported(const Gemm& g);
 cudaError_t gemm_wide(const Gemm& g, cudaStream_t s);
 

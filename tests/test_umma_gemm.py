@@ -165,3 +165,21 @@ def test_umma_wide_rejects_narrow_n():
     with pytest.raises(poetx.PoetxError) as e:
         poetx.testing_gemm_bf16(a, False, b, False, 256, 768, 64, c, variant=2)
     assert e.value.status == 7
+
+
+@pytest.mark.parametrize("splits", [1, 3])
+@pytest.mark.parametrize("M,N,K", [(512, 512, 4096), (256, 1024, 1000)])
+def test_umma_wide_gemm_m_major_fp32_split_k(splits, M, N, K):
+    """The per-block-gradient layout (A and B M/N-major, contraction over the rows, fp32 out,
+    split K into partial products) on 256 x 512 pair tiles, against an fp32 matmul and bit for
+    bit against the 256 x 256 pair kernel's partials."""
+    a, b, ref = _operands(M, N, K, True, True, seed=splits * 13 + M)
+    c = torch.full((splits, M, N), float("nan"), device="cuda")
+    poetx.testing_gemm_bf16(a, True, b, True, M, N, K, c, splits=splits, variant=2)
+    c1 = torch.full((splits, M, N), float("nan"), device="cuda")
+    poetx.testing_gemm_bf16(a, True, b, True, M, N, K, c1, splits=splits, variant=1)
+    torch.cuda.synchronize()
+    poetx.device_status()
+    total = c.sum(0).cpu()
+    assert (total - ref).abs().max().item() / ref.abs().max().item() < 1e-5
+    assert torch.equal(c, c1)
