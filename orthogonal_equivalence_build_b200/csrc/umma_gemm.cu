@@ -680,6 +680,9 @@ struct PairParams {
   Epi epi;
   int* err;
   unsigned long long epi_wait_ns;   // limit of the epilogue's accumulator wait
+  // 256 x 512 kernel: tiles from narrow_from on are half-width (256 columns): the last partial
+  // wave's tiles, each split in two, so that wave takes half as long (see launch_wide_t)
+  int narrow_from;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -1267,6 +1270,18 @@ __device__ __forceinline__ uint64_t wide_b_desc(uint32_t b0, int half, int kk) {
   return B_MN ? smem_desc(base + kk * 2048, 64 * BK * 2, 1024) : smem_desc(base + kk * 32, 16, 1024);
 }
 
+// Tile `tile` of the 256 x 512 kernel: a full-width tile (half = -1), or half `half` (0 / 1,
+// the 256-column halves) of full-width tile narrow_from + (tile - narrow_from) / 2.
+__device__ __forceinline__ TileCoord decode_wide_tile(const PairParams& p, int tile, int& half) {
+  if (tile < p.narrow_from) {
+    half = -1;
+    return decode_pair_tile(p, tile);
+  }
+  const int j = tile - p.narrow_from;
+  half = j & 1;
+  return decode_pair_tile(p, p.narrow_from + (j >> 1));
+}
+
 template <bool A_MN>
 __device__ __forceinline__ uint64_t wide_a_desc(uint32_t a0, int kk) {
   return A_MN ? smem_desc(a0 + kk * 2048, 64 * BK * 2, 1024) : smem_desc(a0 + kk * 32, 16, 1024);
@@ -1337,9 +1352,12 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
       int it = 0;
       bool ok = true;
       for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters) {
-        const TileCoord tc = decode_pair_tile(p, tile);
+        int half;
+        const TileCoord tc = decode_wide_tile(p, tile, half);
         const int kb0 = tc.split * p.kblocks_per_split;
         const int kb1 = min(kb0 + p.kblocks_per_split, nk_all);
+        // a half-width tile loads only its N half, into the stage's first B slot
+        const int h_lo = half < 0 ? 0 : half, h_n = half < 0 ? 2 : 1;
         // groups from g2 on come from the second operand pair, counted from its first group
         const bool second = tc.g >= p.g2;
         const CUtensorMap* map_a = second ? &tma_a2 : &tma_a;
@@ -1358,7 +1376,8 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
             break;
           }
           const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
-          if (leader) mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + B_BYTES));
+          if (leader)
+            mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + (B_BYTES / 2) * h_n));
           const int k = kb * BK;
           const uint32_t da = smem_u32(sa + s * A_BYTES);
           if constexpr (A_MN) {
@@ -1367,9 +1386,9 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
           } else {
             tma_load_2d_pair(da, map_a, fb, ak + k, am);
           }
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t dst = smem_u32(sb + s * B_BYTES + h * (128 * BK * 2));
+          for (int i = 0; i < h_n; ++i) {
+            const int h = h_lo + i;   // N half of the tile, loaded into slot i
+            const uint32_t dst = smem_u32(sb + s * B_BYTES + i * (128 * BK * 2));
             if constexpr (B_MN) {
               tma_load_2d_pair(dst, map_b, fb, bn + 256 * h, bk + k);
               tma_load_2d_pair(dst + 64 * BK * 2, map_b, fb, bn + 256 * h + 64, bk + k);
@@ -1409,7 +1428,8 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
         }
       };
       for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
-        const TileCoord tc = decode_pair_tile(p, tile);
+        int half;
+        const TileCoord tc = decode_wide_tile(p, tile, half);
         const int kb0 = tc.split * p.kblocks_per_split;
         const int nk = min(kb0 + p.kblocks_per_split, nk_all) - kb0;
         const uint32_t par = ((uint32_t)tcount & 1u) ^ 1u;   // previous tile's drain
@@ -1418,6 +1438,23 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
           break;
         }
         tc_fence_after();
+        if (half >= 0) {
+          // half-width tile: accumulator half 0 only, from the stage's first B slot
+          for (int i = 0; i < nk; ++i, ++it) {
+            const int s = it % STAGES;
+            if (!wait_bounded<false>(smem_u32(full + s), (uint32_t)(it / STAGES) & 1u, ctl,
+                                     kErrMma, kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue(it, i, 0, 1);
+            umma_commit_pair_both(smem_u32(empty + s));
+          }
+          if (!ok) break;
+          umma_commit_pair_both(smem_u32(tfull));
+          continue;
+        }
         bool h1_free = false;
         const int first = it;   // iteration of this tile's first K block
         int held = 0;           // the tile's K blocks 0..held-1 have their half-0 MMAs only
@@ -1479,7 +1516,8 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
     const uint32_t leader_tempty0 = map_to_rank(smem_u32(tempty), 0);
     int tcount = 0, chunk = 0;
     for (int tile = cluster_id; tile < p.total_tiles; tile += num_clusters, ++tcount) {
-      const TileCoord tc = decode_pair_tile(p, tile);
+      int half;
+      const TileCoord tc = decode_wide_tile(p, tile, half);
       const int row0 = tc.mb * 256 + (int)rank * 128 + quarter * 32;
       if (!wait_bounded(smem_u32(tfull), (uint32_t)tcount & 1u, ctl, kErrEpilogue, p.epi_wait_ns))
         break;
@@ -1491,17 +1529,22 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
       const long long off0 = (long long)tc.split * p.c_split + goff + (long long)row0 * p.ldc +
                              (long long)tc.nb * 512;
       const int nlive = max(0, min(32, p.M - row0));
+      // a half-width tile's result is in accumulator half 0; its columns start at 256 * half
+      const int nh = half < 0 ? 2 : 1, c0 = half < 0 ? 0 : 256 * half;
 #pragma unroll 1
       for (int h = 0; h < 2; ++h) {
-        if constexpr (OUT_F32)
-          epilogue_warp_rows<true>(trow + (uint32_t)(256 * h), 256,
-                                   sepi + (warp - 2) * kEpiStageBytes, p.C, off0 + 256 * h, p.ldc,
-                                   nlive, lane);
-        else
-          epilogue_tma_bf16(trow + (uint32_t)(256 * h), 256, sepi + (warp - 2) * kEpiStageBytes,
-                            &tma_c, gx + tc.nb * 512 + 256 * h, gy + row0, lane, chunk);
-        tc_fence_before();
+        if (h < nh) {
+          if constexpr (OUT_F32)
+            epilogue_warp_rows<true>(trow + (uint32_t)(256 * h), 256,
+                                     sepi + (warp - 2) * kEpiStageBytes, p.C,
+                                     off0 + c0 + 256 * h, p.ldc, nlive, lane);
+          else
+            epilogue_tma_bf16(trow + (uint32_t)(256 * h), 256, sepi + (warp - 2) * kEpiStageBytes,
+                              &tma_c, gx + tc.nb * 512 + c0 + 256 * h, gy + row0, lane, chunk);
+          tc_fence_before();
+        }
         __syncwarp();
+        // both halves are handed back for every tile (phase accounting of the MMA's waits)
         if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty0 + (uint32_t)(h * 8));
       }
     }
@@ -1659,6 +1702,7 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
   p.splits = effective_splits(g.K, g.splits);
   p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
   p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
+  p.narrow_from = p.total_tiles;
   p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
   fill_segments(g, p);
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
@@ -1737,6 +1781,7 @@ cudaError_t launch_wide_t(const Gemm& g, cudaStream_t s, const char* name) {
   p.splits = effective_splits(g.K, g.splits);
   p.kblocks_per_split = (kblocks + p.splits - 1) / p.splits;
   p.total_tiles = p.tiles_m * p.tiles_n * p.groups * p.splits;
+  p.narrow_from = p.total_tiles;
   p.a_gm = (int)g.a_gm; p.a_gk = (int)g.a_gk; p.b_gn = (int)g.b_gn; p.b_gk = (int)g.b_gk;
   p.nseg = 1; p.kb_per_seg = p.kblocks_per_split;
   p.C = g.C; p.ldc = g.ldc; p.c_gs = g.c_gs; p.c_split = g.c_split;
@@ -1773,6 +1818,13 @@ cudaError_t launch_wide_t(const Gemm& g, cudaStream_t s, const char* name) {
       max_clusters = sm_count() / 2;
   }
   cfg.numAttrs = 2;
+  // Last partial wave: when it holds at most half the clusters, its tiles are split into two
+  // half-width tiles each, so that it takes about half a tile's time instead of a whole one.
+  const int rem = p.total_tiles % max_clusters;
+  if (p.total_tiles > max_clusters && rem > 0 && 2 * rem <= max_clusters) {
+    p.narrow_from = p.total_tiles - rem;
+    p.total_tiles += rem;
+  }
   const int clusters = std::min(p.total_tiles, max_clusters);
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   TraceScope t(name, s);
