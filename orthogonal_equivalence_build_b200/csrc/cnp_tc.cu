@@ -161,7 +161,7 @@ dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
   PairCtx c;
   pair_ctx(b, c);
   int run, local;
-  load_q_tile(up, run_q(r, c.g, b, run, local), b, c);
+  const float* qb = run_q(r, c.g, b, run, local);
   const int64_t base = (int64_t)c.g * c.bb;
   // this block's partial sums within its run, [splits][nb_run][b][b]
   const float* pr = r.parts[run] + (int64_t)local * c.bb;
@@ -169,13 +169,23 @@ dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
   const int64_t split_stride =
       r.split_stride[run] ? r.split_stride[run] : (int64_t)r.nb[run] * c.bb;
   const bool in_place = splits == 1 && pr == dG + base;  // written straight into dG
+  // the first split's values of both tiles are requested before the q tile, so the two loads'
+  // latencies overlap instead of following each other across the q tile's barrier
+  float4 first[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
+    first[h] = (h == 1 && c.diag) ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                  : ld4(pr + (int64_t)i * b + j);
+  }
+  load_q_tile(up, qb, b, c);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     if (h == 1 && c.diag) break;
     const int i = (h ? c.J : c.I) * TS + c.r, j = (h ? c.I : c.J) * TS + c.c0;
     const int64_t off = (int64_t)i * b + j;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-    int sp = 0;
+    float v[4] = {first[h].x, first[h].y, first[h].z, first[h].w};
+    int sp = 1;
     for (; sp + 4 <= splits; sp += 4) {   // four loads in flight, added in split order
       float4 t[4];
 #pragma unroll

@@ -778,10 +778,16 @@ __device__ __forceinline__ TileCoord decode_pair_tile(const PairParams& p, int t
 
 // int8 B operand (8-bit weight storage, "POET-XQ"): B is stored as int8 codes with one fp32
 // scale per column of the stored tensor. The producer streams the int8 tile (8 KB per CTA and
-// stage) into a separate staging ring; four converter warps turn it into the bf16 operand
+// stage) into a separate staging ring; converter warps turn it into the bf16 operand
 // bf16(code * scale) in the 128-byte-swizzled stage the MMA reads, then arrive on the leader's
 // full barrier (which also counts the A bytes of both CTAs). The MMA and epilogue are unchanged.
-constexpr int kPairConvThreads = 128;
+// The converters form kConvGroups groups of kConvWarpsPerGroup warps that take the K blocks in
+// turn: one group converts a block in about three MMA blocks' time (its loads, the arithmetic
+// and the swizzled stores follow each other), so three groups keep up with the MMA (two paced
+// it at about 1500 cycles per 512-cycle block).
+constexpr int kConvGroups = 3;
+constexpr int kConvWarpsPerGroup = 2;
+constexpr int kPairConvThreads = 32 * kConvWarpsPerGroup * kConvGroups;
 
 // float(q) for a signed byte q without a conversion instruction: q + 128 = byte ^ 0x80 placed in
 // the low mantissa bits of 2^23 (0x4B000000) is the float 2^23 + 128 + q; subtracting 2^23 + 128
@@ -890,7 +896,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       // B_I8: the producer's arrive plus one per converter warp of a group, in both CTAs
-      mbar_init(smem_u32(full + s), B_I8 ? 1 + 2 * (kPairConvThreads / 64) : 1);
+      mbar_init(smem_u32(full + s), B_I8 ? 1 + 2 * kConvWarpsPerGroup : 1);
       mbar_init(smem_u32(empty + s), 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -900,7 +906,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     mbar_init(smem_u32(drain), 1);
     for (int r = 0; r < RAW; ++r) {
       mbar_init(smem_u32(qfull + r), 1);
-      mbar_init(smem_u32(qempty + r), kPairConvThreads / 64);
+      mbar_init(smem_u32(qempty + r), kConvWarpsPerGroup);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1114,14 +1120,15 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
     }
   } else if constexpr (B_I8) {
     // ------------------------------------------------------------ int8 -> bf16 converters
-    // Two groups of two warps take alternate K blocks, so two blocks are converted at a time
-    // and each group's staging slots (it % RAW has the group's parity) double-buffer its TMA
-    // loads. Thread gt of a group owns one 8-element unit column of the staged tile and 16 of
-    // its 64 (B_MN) or 128 (K-major) lines: 8-byte conflict-free reads, 16-byte swizzled
-    // conflict-free writes.
+    // kConvGroups groups of two warps take the K blocks in turn (block it goes to group
+    // it % kConvGroups), so that many blocks are converted at a time; the staging ring holds
+    // RAW blocks ahead. Thread gt of a group owns one 8-element unit column of the staged tile
+    // and 16 of its 64 (B_MN) or 128 (K-major) lines: 8-byte conflict-free reads, 16-byte
+    // swizzled conflict-free writes.
+    static_assert(kConvWarpsPerGroup == 2, "a group's 64 threads own the tile's unit columns");
     const int cw = warp - (2 + EPI_W);
-    const int grp = cw >> 1;
-    const int gt = (cw & 1) * 32 + lane;   // 0..63
+    const int grp = cw / kConvWarpsPerGroup;
+    const int gt = (cw % kConvWarpsPerGroup) * 32 + lane;   // 0..63
     const uint32_t leader_full0 = map_to_rank(smem_u32(full), 0);
     int it = 0;
     bool ok = true;
@@ -1133,7 +1140,7 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       uint64_t sc[4];
       if constexpr (B_MN) load_scales8(p.b_scale + bn + 8 * (gt & 15), sc);   // per N column
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        if ((it & 1) != grp) continue;
+        if (it % kConvGroups != grp) continue;
         const int s = it % STAGES, r = it % RAW;
         if constexpr (!B_MN) {
           // scales along K for this block, requested before the waits so that their latency

@@ -71,8 +71,11 @@ class XqCase:
 
 # ------------------------------------------------------------------ quantiser
 @pytest.mark.parametrize("m,n,dt", [(512, 768, torch.bfloat16), (1000, 48, torch.bfloat16),
-                                    (96, 4096, torch.float32), (4096, 1024, torch.bfloat16)])
+                                    (96, 4096, torch.float32), (4096, 1024, torch.bfloat16),
+                                    (37, 40, torch.bfloat16)])
 def test_quantize_and_dequantize_bit_exact(m, n, dt):
+    """Codes, scales and dequantised values bit for bit against the oracle; n % 16 == 0 takes
+    the 16-wide dequantisation, n = 40 the element-wise one."""
     rng = np.random.default_rng(m * 7 + n)
     w = rng.standard_normal((m, n)) * rng.uniform(0.01, 2.0, size=n)[None, :]
     w[:, 5] = 0.0                                      # an all-zero column
