@@ -84,14 +84,14 @@ def layer_flops(T, m, n, b, cnp=True):
 
 
 def layer_bytes(T, m, n, b, e=2, w_e=None):
-    """Algorithmic HBM bytes of one step: boundary tensors plus the saved B.
-    fwd reads X, W0', G and writes Y, B; bwd reads dY, X, B, W0', G and writes dX;
-    q, G, dq in fp32.  w_e: bytes per W0' element (1 for 8-bit storage, plus its column
-    scales)."""
+    """Algorithmic HBM bytes of one step: boundary tensors plus the saved activations.
+    fwd reads X, W0', G and writes Y, B and A = X[:, perm_r]; bwd reads dY, A, B, W0', G and
+    writes dX; q, G, dq in fp32.  w_e: bytes per W0' element (1 for 8-bit storage, plus its
+    column scales)."""
     gblk = (m // b + n // b) * b * b
     qn = (m // b + n // b) * b * (b - 1) // 2
     w = (e if w_e is None else w_e) * m * n + (4 * n if w_e == 1 else 0)
-    fwd = e * (T * m + T * n + T * n) + w + e * gblk
+    fwd = e * (T * m + T * n + T * n + T * m) + w + e * gblk
     bwd = e * (T * n + T * m + T * n + T * m) + w + e * gblk
     cnp = 4 * qn + 4 * gblk + 2 * gblk
     dq = 4 * qn * 2
@@ -309,6 +309,7 @@ def workload_config(wl, args, world):
            "parallelism": f"dp{world}",
            "step": ("cnp_build(R,P) + " if wl.cnp_in_step else "")
            + "linear_fwd + linear_bwd(dx, dq) per linear"
+           + ", activations B [T, n] and A = X[:, perm_r] [T, m] kept from forward to backward"
            + (" + NCCL all-reduce of dq" if world > 1 else ""),
            "l2": (f"inputs larger than L2: X + dY = {in_bytes / 2**20:.0f} MiB per step"
                   if in_bytes > L2_BYTES else "L2 flushed (2x126 MiB write) between steps")}
@@ -406,6 +407,8 @@ def run_ours(args):
         d["dy"] = d["dy_host"].to(dev)
         d["y"] = torch.empty(T, lin.n, dtype=dt, device=dev)
         d["bsave"] = torch.empty(T, lin.n, dtype=dt, device=dev)
+        # activations kept from the forward for the backward (POET-Xfast): B, and A = X[:, perm_r]
+        d["asave"] = torch.empty(T, lin.m, dtype=dt, device=dev)
         d["dx"] = torch.empty(T, lin.m, dtype=dt, device=dev)
         # dq_r and dq_p are views of one packed buffer: one all-reduce per linear (N > 1)
         d["dq"] = torch.empty(L.q_r.numel() + L.q_p.numel(), device=dev)
@@ -435,9 +438,9 @@ def run_ours(args):
             nr = L.q_r.numel()
             if wl.cnp_in_step:
                 poetx.layer_cnp_build(L, ws)
-            poetx.linear_fwd(L, xin, y, d["bsave"], ws)
+            poetx.linear_fwd(L, xin, y, d["bsave"], ws, saved_a=d["asave"])
             poetx.linear_bwd(L, xin, dyin, d["bsave"], dx, dq[:nr].view_as(L.q_r),
-                             dq[nr:].view_as(L.q_p), ws)
+                             dq[nr:].view_as(L.q_p), ws, saved_a=d["asave"])
             reducer.add(dq)
         reducer.finish()
 

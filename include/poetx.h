@@ -194,6 +194,28 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
                               void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * poetx_linear_fwd_ex / poetx_linear_bwd_ex — the same forward and backward, keeping
+ *   A = X[:, perm_r] between them ("POET-Xfast" in "POET-X: Memory-efficient LLM Training ..."
+ *   §2 Metodologia: activations are saved rather than recomputed).
+ *   saved_a [T, m] (layer dtype): the forward writes A there (instead of into its workspace);
+ *   the backward reads it wherever it needs A (the per-block gradients dG_R^j = A_j^T dA'_j and,
+ *   with saved_b NULL, the rebuild of B) instead of gathering X again, which saves one
+ *   [T, m] gather pass per backward for T*m elements of memory. saved_a may be NULL: the calls
+ *   are then poetx_linear_fwd / poetx_linear_bwd. With saved_a given, the backward does not read
+ *   x and x may be NULL. saved_a must hold the forward's A for the same x and layer state
+ *   (perm_r unchanged since: merge_reinit changes it).
+ *   Results are bit-identical to the calls without saved_a. Errors: as those calls, plus ALIGN
+ *   for a saved_a not 16-byte aligned.
+ * ------------------------------------------------------------------------------------------- */
+poetx_status poetx_linear_fwd_ex(const poetx_layer* L, const void* x, int64_t T, void* y,
+                                 void* saved_b, void* saved_a, void* workspace, size_t ws_bytes,
+                                 void* stream);
+poetx_status poetx_linear_bwd_ex(const poetx_layer* L, const void* x, const void* dy,
+                                 const void* saved_b, const void* saved_a, int64_t T, void* dx,
+                                 float* dq_r, float* dq_p, void* workspace, size_t ws_bytes,
+                                 void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * poetx_merge_permutations — W0' = Psi_R W0 Psi_P^T ("POET-X" blog §第二斧: the two permutations
  *   next to the fixed W are folded into it before the inner loop).
  *   w0 [m, n] input, w0m [m, n] output (must not overlap w0), dtype F32 or BF16. Bit-exact copy.

@@ -445,32 +445,52 @@ size_t poetx_fwd_workspace_bytes(const poetx_layer* L, int64_t T) {
   return fwd_layout(L, T, nullptr, nullptr);
 }
 
-poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, void* y,
-                              void* saved_b, void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+poetx_status linear_fwd_impl(const poetx_layer* L, const void* x, int64_t T, void* y,
+                             void* saved_b, void* saved_a, void* workspace, size_t ws_bytes,
+                             void* stream) {
   poetx_status st = check_layer(L, true);
   if (st != POETX_OK) return st;
   if (T < 0) return fail(POETX_ERR_SHAPE, "T < 0");
   if (T == 0) return POETX_OK;
   if (!x || !y) return fail(POETX_ERR_INVALID_ARG, "x or y is NULL");
-  if (!aligned16(x) || !aligned16(y) || (saved_b && !aligned16(saved_b)))
-    return fail(POETX_ERR_ALIGN, "x, y, saved_b must be 16-byte aligned");
+  if (!aligned16(x) || !aligned16(y) || (saved_b && !aligned16(saved_b)) ||
+      (saved_a && !aligned16(saved_a)))
+    return fail(POETX_ERR_ALIGN, "x, y, saved_b, saved_a must be 16-byte aligned");
   if ((st = check_ws(workspace, ws_bytes, poetx_fwd_workspace_bytes(L, T))) != POETX_OK) return st;
   if ((st = check_device()) != POETX_OK) return st;
   cudaStream_t s = as_stream(stream);
   FwdWs w;
   fwd_layout(L, T, workspace, &w);
   void* B = saved_b ? saved_b : w.B;
+  void* A = saved_a ? saved_a : w.A;   // A = X[:, perm_r], kept for the backward when given
   const int e = elem_size(L->dtype);
   const DT t = dt_of(L->dtype);
   const int64_t m = L->m, n = L->n, b = L->b;
   const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
-  CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_fwd_gather_X"), "fwd gather");
-  CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.A1, T, m, b, false, s), "fwd R blocks");
+  CHECK_CUDA(gather_cols(x, A, T, m, nullptr, L->perm_r, e, s, "perm_fwd_gather_X"), "fwd gather");
+  CHECK_CUDA(gemm_blockwise(t, A, Gr, w.A1, T, m, b, false, s), "fwd R blocks");
   CHECK_CUDA(w0_product(L, w.A1, B, T, false, w.Wd, s), "fwd W0' GEMM");
   CHECK_CUDA(gemm_blockwise(t, B, Gp, w.C, T, n, b, false, s), "fwd P blocks");
   CHECK_CUDA(scatter_cols(w.C, y, T, n, L->perm_p, e, w.inv, s, "perm_fwd_scatter_Y"), "fwd scatter");
   return POETX_OK;
+}
+}  // namespace
+
+extern "C" {
+
+poetx_status poetx_linear_fwd(const poetx_layer* L, const void* x, int64_t T, void* y,
+                              void* saved_b, void* workspace, size_t ws_bytes, void* stream) {
+  return linear_fwd_impl(L, x, T, y, saved_b, nullptr, workspace, ws_bytes, stream);
+}
+
+poetx_status poetx_linear_fwd_ex(const poetx_layer* L, const void* x, int64_t T, void* y,
+                                 void* saved_b, void* saved_a, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  return linear_fwd_impl(L, x, T, y, saved_b, saved_a, workspace, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ backward
@@ -479,16 +499,21 @@ size_t poetx_bwd_workspace_bytes(const poetx_layer* L, int64_t T) {
   return bwd_layout(L, T, nullptr, nullptr);
 }
 
-poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* dy,
-                              const void* saved_b, int64_t T, void* dx, float* dq_r, float* dq_p,
-                              void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy,
+                             const void* saved_b, const void* saved_a, int64_t T, void* dx,
+                             float* dq_r, float* dq_p, void* workspace, size_t ws_bytes,
+                             void* stream) {
   poetx_status st = check_layer(L, true);
   if (st != POETX_OK) return st;
   if (T < 0) return fail(POETX_ERR_SHAPE, "T < 0");
   if ((dq_r && !L->q_r) || (dq_p && !L->q_p))
     return fail(POETX_ERR_INVALID_ARG, "dq requested but the layer has no q");
-  if (!x || !dy) return fail(POETX_ERR_INVALID_ARG, "x or dy is NULL");
-  if (!aligned16(x) || !aligned16(dy) || (saved_b && !aligned16(saved_b)) || (dx && !aligned16(dx)) ||
+  if ((!x && !saved_a) || !dy) return fail(POETX_ERR_INVALID_ARG, "x (or saved_a) or dy is NULL");
+  if ((x && !aligned16(x)) || !aligned16(dy) || (saved_b && !aligned16(saved_b)) ||
+      (saved_a && !aligned16(saved_a)) || (dx && !aligned16(dx)) ||
       (dq_r && !aligned16(dq_r)) || (dq_p && !aligned16(dq_p)))
     return fail(POETX_ERR_ALIGN, "backward pointers must be 16-byte aligned");
   if ((st = check_ws(workspace, ws_bytes, poetx_bwd_workspace_bytes(L, T))) != POETX_OK) return st;
@@ -501,11 +526,18 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   const int64_t m = L->m, n = L->n, b = L->b;
   const void* Gr = L->dtype == POETX_BF16 ? L->g_r_lp : (const void*)L->g_r;
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
+  // A = X[:, perm_r]: the forward's saved copy, or gathered again from X (once, when first needed)
+  const void* A = saved_a;
+  bool have_a = saved_a != nullptr;
   if (!saved_b && (dq_p || dq_r)) {
     // memory-saving mode: rebuild B = (X[:, perm_r] Diag(G_R)) W0' exactly instead of keeping it
-    CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_regather_X"),
-               "bwd recompute gather");
-    CHECK_CUDA(gemm_blockwise(t, w.A, Gr, w.dA, T, m, b, false, s), "bwd recompute R blocks");
+    if (!have_a) {
+      CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_regather_X"),
+                 "bwd recompute gather");
+      A = w.A;
+      have_a = true;
+    }
+    CHECK_CUDA(gemm_blockwise(t, A, Gr, w.dA, T, m, b, false, s), "bwd recompute R blocks");
     CHECK_CUDA(w0_product(L, w.dA, w.B, T, false, w.Wd, s), "bwd recompute W0' GEMM");
     saved_b = w.B;
   }
@@ -527,9 +559,14 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
   bool merged = false;
   int sp_rp = 1;
   if (dq_r) {
-    CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_gather_X"), "bwd gather X");
+    if (!have_a) {
+      CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_gather_X"),
+                 "bwd gather X");
+      A = w.A;
+      have_a = true;
+    }
     if (one_dg) {
-      const cudaError_t ce = gemm_block_grad2(t, w.A, w.dA1, m, saved_b, w.dC, n, w.dG, T, b,
+      const cudaError_t ce = gemm_block_grad2(t, A, w.dA1, m, saved_b, w.dC, n, w.dG, T, b,
                                               w.part_rp, &sp_rp, s);
       if (ce == cudaSuccess) merged = true;
       else if (ce != cudaErrorNotSupported) CHECK_CUDA(ce, "bwd dG_R + dG_P");
@@ -537,7 +574,7 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
                       "bwd dG_P");
     }
     if (!merged)
-      CHECK_CUDA(gemm_block_grad(t, w.A, w.dA1, dG_r, T, m, b, w.part_r, &sp_r, s), "bwd dG_R");
+      CHECK_CUDA(gemm_block_grad(t, A, w.dA1, dG_r, T, m, b, w.part_r, &sp_r, s), "bwd dG_R");
   }
   if (dq_r || dq_p) {
     // one dq chain over the R blocks and the P blocks
@@ -567,6 +604,25 @@ poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* d
     CHECK_CUDA(gemm_dq_from_dg_runs(t, r, b, dq_r ? dG_r : dG_p, w.chain, s), "dq chain");
   }
   return POETX_OK;
+}
+}  // namespace
+
+extern "C" {
+
+poetx_status poetx_linear_bwd(const poetx_layer* L, const void* x, const void* dy,
+                              const void* saved_b, int64_t T, void* dx, float* dq_r, float* dq_p,
+                              void* workspace, size_t ws_bytes, void* stream) {
+  if (!x) return fail(POETX_ERR_INVALID_ARG, "x or dy is NULL");
+  return linear_bwd_impl(L, x, dy, saved_b, nullptr, T, dx, dq_r, dq_p, workspace, ws_bytes,
+                         stream);
+}
+
+poetx_status poetx_linear_bwd_ex(const poetx_layer* L, const void* x, const void* dy,
+                                 const void* saved_b, const void* saved_a, int64_t T, void* dx,
+                                 float* dq_r, float* dq_p, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  return linear_bwd_impl(L, x, dy, saved_b, saved_a, T, dx, dq_r, dq_p, workspace, ws_bytes,
+                         stream);
 }
 
 // ------------------------------------------------------------------ permutations

@@ -126,12 +126,20 @@ __device__ __forceinline__ void put_hilo4(__nv_bfloat16* __restrict__ p_hi,
   st4h(p_lo + off, l);
 }
 
+// The per-block counts of a two-product launch (see run_chain) start at zero: the first CTA
+// of the pass before it clears them (the launch waits for this grid to finish).
+__device__ __forceinline__ void zero_counts(int* deps, int ndeps) {
+  if (deps && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int i = threadIdx.x; i < ndeps; i += blockDim.x) deps[i] = 0;
+}
+
 // CNP pass 1: Q_hi, Q_lo [nb][b][b] from the packed strict upper triangles.
 __global__ void __launch_bounds__(kTileThreads)
 split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
-               __nv_bfloat16* __restrict__ Qlo) {
+               __nv_bfloat16* __restrict__ Qlo, int* __restrict__ deps, int ndeps) {
   pdl_wait();
   pdl_trigger();
+  zero_counts(deps, ndeps);
   __shared__ Tile up;
   PairCtx c;
   pair_ctx(b, c);
@@ -154,9 +162,10 @@ split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
 __global__ void __launch_bounds__(kTileThreads)
 dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
                __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ Ql,
-               __nv_bfloat16* __restrict__ dGh) {
+               __nv_bfloat16* __restrict__ dGh, int* __restrict__ deps, int ndeps) {
   pdl_wait();
   pdl_trigger();
+  zero_counts(deps, ndeps);
   __shared__ Tile up;
   PairCtx c;
   pair_ctx(b, c);
@@ -316,8 +325,9 @@ void three_pass(umma::Gemm& g, int64_t nb, int64_t b) {
 // that for the fused epilogues, whose per-element work spreads over more SMs with smaller
 // tiles (measured at b = 256 over 16 blocks and b = 512 over 20; b = 512 over 36 blocks keeps
 // the pairs).
-cudaError_t run_block_gemm(const umma::Gemm& g, cudaStream_t s) {
-  if (!umma::supported(g)) return cudaErrorNotSupported;
+// 0: CTA-pair tiles; otherwise the single-CTA tile width; -1: not covered
+int block_tile_choice(const umma::Gemm& g) {
+  if (!umma::supported(g)) return -1;
   const int64_t sms = umma::sm_count();
   const int64_t fixed = g.epi.mode == umma::kEpiStore ? 128 * 128 : 128 * 32;
   int64_t best = -1;
@@ -335,10 +345,49 @@ cudaError_t run_block_gemm(const umma::Gemm& g, cudaStream_t s) {
       best_bn = bn;
     }
   }
-  if (best_bn == 0) return umma::gemm_pair(g, s);
+  return best_bn;
+}
+
+cudaError_t run_block_gemm(const umma::Gemm& g, cudaStream_t s) {
+  const int bn = block_tile_choice(g);
+  if (bn < 0) return cudaErrorNotSupported;
+  if (bn == 0) return umma::gemm_pair(g, s);
   umma::Gemm h = g;
-  h.bn = best_bn;
+  h.bn = bn;
   return umma::gemm(h, s);
+}
+
+// Two dependent products of a chain in one launch of the CTA-pair kernel, where both would run
+// on CTA pairs alone: `second`'s groups follow `first`'s, and a tile of second-product group g
+// loads its operands only once every tile of block g % nb of the first product has stored its
+// results (deps, nb counts cleared by the pass before). The blocks pipeline through the two
+// products instead of the second launch waiting for the whole first one. Returns false (nothing
+// launched) where it does not apply.
+bool run_chain(const umma::Gemm& first, const umma::Gemm& second, int64_t nb, int* deps,
+               cudaStream_t s, cudaError_t* err) {
+  if (!deps || block_tile_choice(first) != 0 || block_tile_choice(second) != 0) return false;
+  umma::Gemm g = first;
+  g.groups = first.groups + second.groups;
+  g.groups_1 = first.groups;
+  g.A2 = second.A; g.a2_rows = second.a_rows; g.a2_cols = second.a_cols; g.a2_ld = second.a_ld;
+  g.B2 = second.B; g.b2_rows = second.b_rows; g.b2_cols = second.b_cols; g.b2_ld = second.b_ld;
+  g.epi2 = second.epi;
+  g.has_epi2 = true;
+  g.C = second.C;
+  g.c_rel2 = true;
+  g.deps = deps;
+  g.dep_blocks = (int)nb;
+  // first-product epilogue warps per block: its pair tiles x 2 CTAs x 4 warps
+  g.dep_target = (int)(((first.M + 255) / 256) * (first.N / 256) * 8);
+  if (first.a_mn != second.a_mn || first.b_mn != second.b_mn || first.out_f32 != second.out_f32 ||
+      first.nseg != second.nseg || !umma::pair_supported(g))
+    return false;
+  for (int k = 0; k < 3; ++k)
+    if (first.a_dy[k] != second.a_dy[k] || first.b_dy[k] != second.b_dy[k] ||
+        first.a_dx[k] != second.a_dx[k] || first.b_dx[k] != second.b_dx[k])
+      return false;
+  *err = umma::gemm_pair(g, s);
+  return true;
 }
 
 #define POETX_TRY(x)                  \
@@ -352,8 +401,8 @@ cudaError_t run_block_gemm(const umma::Gemm& g, cudaStream_t s) {
 bool tc_blocks_supported(int64_t b) { return b % 128 == 0 && b >= 128; }
 
 size_t cnp_tc_ws_bytes(int64_t nb, int64_t b) {
-  // [Q_hi; Q_lo], [S_hi; S_lo], [H_hi; H_lo]
-  return 3 * align_up((size_t)(2 * nb * b * b) * 2, 256);
+  // [Q_hi; Q_lo], [S_hi; S_lo], [H_hi; H_lo], per-block counts of the two-product launch
+  return 3 * align_up((size_t)(2 * nb * b * b) * 2, 256) + align_up((size_t)nb * 4, 256);
 }
 
 cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s) {
@@ -364,37 +413,42 @@ cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s
   auto* Qst = static_cast<__nv_bfloat16*>(a.take((size_t)(2 * nb * bb) * 2));
   auto* Sst = static_cast<__nv_bfloat16*>(a.take((size_t)(2 * nb * bb) * 2));
   auto* Hst = static_cast<__nv_bfloat16*>(a.take((size_t)(2 * nb * bb) * 2));
+  auto* deps = static_cast<int*>(a.take((size_t)nb * 4));
   const dim3 grid = pair_grid(nb, b);
   {
     TraceScope t("cnp_split_Q", s);
-    POETX_TRY(launch_k(split_q_kernel, grid, dim3(kTileThreads), 0, s, r, (int)b, Qst, Qst + nb * bb));
+    POETX_TRY(launch_k(split_q_kernel, grid, dim3(kTileThreads), 0, s, r, (int)b, Qst,
+                       Qst + nb * bb, deps, (int)nb));
   }
-  {
-    umma::Gemm g = block_gemm(Qst, 2 * nb * b, Qst, 2 * nb * b, nb, b, b, "umma_cnp_QQ");
-    three_pass(g, nb, b);
-    g.epi.mode = umma::kEpiCnpS;
-    g.epi.b = (int)b;
-    g.epi.qh = Qst; g.epi.ql = Qst + nb * bb;
-    g.epi.o[0] = Sst; g.epi.o[1] = Sst + nb * bb; g.epi.o[2] = Hst; g.epi.o[3] = Hst + nb * bb;
-    POETX_TRY(run_block_gemm(g, s));
-  }
-  umma::Gemm g = block_gemm(Sst, 2 * nb * b, Hst, 2 * nb * b, nb, b, b, "umma_cnp_SH");
-  three_pass(g, nb, b);
-  g.epi.mode = umma::kEpiCnpG;
-  g.epi.b = (int)b;
-  g.epi.nb0 = r.nb0;
-  g.epi.qh = Qst; g.epi.ql = Qst + nb * bb;
+  umma::Gemm qq = block_gemm(Qst, 2 * nb * b, Qst, 2 * nb * b, nb, b, b, "umma_cnp_QQ");
+  three_pass(qq, nb, b);
+  qq.epi.mode = umma::kEpiCnpS;
+  qq.epi.b = (int)b;
+  qq.epi.qh = Qst; qq.epi.ql = Qst + nb * bb;
+  qq.epi.o[0] = Sst; qq.epi.o[1] = Sst + nb * bb; qq.epi.o[2] = Hst; qq.epi.o[3] = Hst + nb * bb;
+  umma::Gemm sh = block_gemm(Sst, 2 * nb * b, Hst, 2 * nb * b, nb, b, b, "umma_cnp_SH");
+  three_pass(sh, nb, b);
+  sh.epi.mode = umma::kEpiCnpG;
+  sh.epi.b = (int)b;
+  sh.epi.nb0 = r.nb0;
+  sh.epi.qh = Qst; sh.epi.ql = Qst + nb * bb;
   for (int k = 0; k < 2; ++k) {
-    g.epi.g[k] = r.g[k];
-    g.epi.g_lp[k] = r.g_lp[k];
+    sh.epi.g[k] = r.g[k];
+    sh.epi.g_lp[k] = r.g_lp[k];
   }
-  return run_block_gemm(g, s);
+  // S = Q Q, then G = I + 2Q + S H: one launch where both run on CTA pairs
+  umma::Gemm chain = qq;
+  chain.name = "umma_cnp_QQ_SH";
+  cudaError_t ce = cudaSuccess;
+  if (run_chain(chain, sh, nb, deps, s, &ce)) return ce;
+  POETX_TRY(run_block_gemm(qq, s));
+  return run_block_gemm(sh, s);
 }
 
 size_t dq_tc_ws_bytes(int64_t nb, int64_t b) {
   const size_t h = align_up((size_t)(nb * b * b) * 2, 256);
   const size_t f = align_up((size_t)(nb * b * b) * 4, 256);
-  return 6 * h + 3 * f;
+  return 6 * h + 3 * f + align_up((size_t)nb * 4, 256);
 }
 
 cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cudaStream_t s) {
@@ -415,25 +469,33 @@ cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cu
   float* Hb = fst;
   float* T1 = fst + nb * bb;
   auto* V = static_cast<float*>(a.take(fb));
+  auto* deps = static_cast<int*>(a.take((size_t)nb * 4));
   const dim3 grid = pair_grid(nb, b);
   const int bi = (int)b;
   {
     TraceScope t("dq_prep", s);
-    POETX_TRY(launch_k(dq_prep_kernel, grid, dim3(kTileThreads), 0, s, r, bi, dG, Qh, Ql, dGh));
+    POETX_TRY(launch_k(dq_prep_kernel, grid, dim3(kTileThreads), 0, s, r, bi, dG, Qh, Ql, dGh,
+                       deps, (int)nb));
   }
+  umma::Gemm qq = block_gemm(Qh, nb * b, Qh, nb * b, nb, b, b, "umma_dq_QQ");
+  qq.epi.mode = umma::kEpiDqS;
+  qq.epi.b = bi;
+  qq.epi.qh = Qh; qq.epi.ql = Ql;
+  qq.epi.o[0] = Sh; qq.epi.o[1] = SmQ;
+  // Hbar_g = S_g dG_g (groups 0..nb-1) and T1_g = dG_g SmQ_g (groups nb..2nb-1)
+  umma::Gemm sdg = block_gemm(Sh, 2 * nb * b, dGh, 2 * nb * b, 2 * nb, b, b, "umma_dq_SdG_dGH");
+  sdg.C = fst;
   {
-    umma::Gemm g = block_gemm(Qh, nb * b, Qh, nb * b, nb, b, b, "umma_dq_QQ");
-    g.epi.mode = umma::kEpiDqS;
-    g.epi.b = bi;
-    g.epi.qh = Qh; g.epi.ql = Ql;
-    g.epi.o[0] = Sh; g.epi.o[1] = SmQ;
-    POETX_TRY(run_block_gemm(g, s));
-  }
-  {
-    // Hbar_g = S_g dG_g (groups 0..nb-1) and T1_g = dG_g SmQ_g (groups nb..2nb-1)
-    umma::Gemm g = block_gemm(Sh, 2 * nb * b, dGh, 2 * nb * b, 2 * nb, b, b, "umma_dq_SdG_dGH");
-    g.C = fst;
-    POETX_TRY(run_block_gemm(g, s));
+    // S = Q Q, then S dG and dG (S - 2Q): one launch where all run on CTA pairs
+    umma::Gemm chain = qq;
+    chain.name = "umma_dq_QQ_SdG_dGH";
+    cudaError_t ce = cudaSuccess;
+    if (run_chain(chain, sdg, nb, deps, s, &ce)) {
+      POETX_TRY(ce);
+    } else {
+      POETX_TRY(run_block_gemm(qq, s));
+      POETX_TRY(run_block_gemm(sdg, s));
+    }
   }
   {
     TraceScope t("dq_mid", s);

@@ -43,7 +43,10 @@ constexpr int kThreads = 192;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;   // 4 s
 constexpr uint64_t kDrainLimitNs = 200000000ull;   // 0.2 s per drain wait
 
-enum : int { kErrProducer = 0x101, kErrMma = 0x102, kErrEpilogue = 0x103, kErrConvert = 0x104 };
+enum : int {
+  kErrProducer = 0x101, kErrMma = 0x102, kErrEpilogue = 0x103, kErrConvert = 0x104,
+  kErrDependency = 0x105   // a second-product tile's inputs were not published in time
+};
 
 struct Params {
   int M, N, K, groups, splits;
@@ -133,6 +136,31 @@ struct Ctl {
   volatile int* abort;
   int* err;
 };
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// Wait until *cnt >= target (a count other CTAs of the same launch publish with release adds);
+// false if the wait expired (code recorded, CTA aborting).
+__device__ __noinline__ bool wait_count(const int* cnt, int target, Ctl c, int code,
+                                        uint64_t limit_ns) {
+  if (ld_acquire_gpu(cnt) >= target) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(cnt) >= target) return true;
+    if ((it & 15) == 0 && global_ns() - t0 > limit_ns) {
+      *c.abort = 1;
+      if (code) atomicCAS(c.err, 0, code);
+      return false;
+    }
+  }
+}
 
 // Wait for `parity` on `bar`; false if the CTA is aborting (unless stop_on_abort is false) or
 // the wait expired.
@@ -683,6 +711,14 @@ struct PairParams {
   // 256 x 512 kernel: tiles from narrow_from on are half-width (256 columns): the last partial
   // wave's tiles, each split in two, so that wave takes half as long (see launch_wide_t)
   int narrow_from;
+  // Two dependent products in one launch (256 x 256 kernel): groups from g2 on form the second
+  // product, with their own epilogue epi2 and, with c_rel2, output groups counted from g2. When
+  // deps is set, second-product group g waits, before its operands are loaded, until
+  // deps[(g - g2) % dep_blocks] reaches dep_target: the count of first-product epilogue warps of
+  // that group whose stores are visible (each warp adds one after its stores).
+  Epi epi2;
+  int* deps;
+  int dep_target, dep_blocks, c_rel2;
 };
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -977,6 +1013,16 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
         const int gl = second ? tc.g - p.g2 : tc.g;
         const int am = gl * p.a_gm + tc.mb * 256 + (int)rank * 128, ak = gl * p.a_gk;
         const int bn = gl * p.b_gn + tc.nb * 256 + (int)rank * 128, bk = gl * p.b_gk;
+        if (second && p.deps) {
+          // the first product's results for this group must be written before they are read;
+          // then order this thread's asynchronous-proxy (TMA) reads after them
+          if (!wait_count(p.deps + gl % p.dep_blocks, p.dep_target, ctl, kErrDependency,
+                          kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -1089,19 +1135,24 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       const uint32_t use = (uint32_t)(tcount >> 1);
       const int row0 = tc.mb * 256 + (int)rank * 128 + quarter * 32;
       const int nlive = max(0, min(32, p.M - row0));
-      const bool fused = OUT_F32 && p.epi.mode != kEpiStore;
+      // a second product's tiles use epi2 and their group index within that product
+      const bool second = tc.g >= p.g2;
+      const Epi& ep = second ? p.epi2 : p.epi;
+      const int ge = second ? tc.g - p.g2 : tc.g;
+      const int gout = (second && p.c_rel2) ? tc.g - p.g2 : tc.g;
+      const bool fused = OUT_F32 && ep.mode != kEpiStore;
       FusedQ q0;
       const int col0 = tc.nb * 256 + cbase;
-      if (fused) fused_q_load(p.epi, fused_base(p.epi, tc.g, row0, col0, lane), 0, nlive, lane, q0);
+      if (fused) fused_q_load(ep, fused_base(ep, ge, row0, col0, lane), 0, nlive, lane, q0);
       if (!wait_bounded(smem_u32(tfull + acc), use & 1u, ctl, kErrEpilogue, p.epi_wait_ns))
         break;
       tc_fence_after();
-      const long long off0 = (long long)tc.split * p.c_split + (long long)tc.g * p.c_gs +
+      const long long off0 = (long long)tc.split * p.c_split + (long long)gout * p.c_gs +
                              (long long)row0 * p.ldc + (long long)col0;
       const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) +
                             (uint32_t)(acc * ACC_COLS + cbase);
       if (fused)
-        epilogue_fused(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, p.epi, tc.g, row0, col0,
+        epilogue_fused(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, ep, ge, row0, col0,
                        nlive, lane, q0);
       else if constexpr (!OUT_F32)
         epilogue_tma_bf16(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, &tma_c,
@@ -1110,6 +1161,15 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
       else
         epilogue_warp_rows<OUT_F32>(trow, COLS, sepi + (warp - 2) * kEpiStageBytes, p.C, off0,
                                     p.ldc, nlive, lane);
+      if constexpr (OUT_F32) {
+        if (p.deps && !second) {
+          // publish this warp's part of a first-product tile: its stores (plain stores of the
+          // fused or fp32 epilogue) become visible at GPU scope before the count moves
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) red_release_gpu_add(p.deps + tc.g, 1);
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty0 + (uint32_t)(acc * 8));
@@ -1727,6 +1787,11 @@ cudaError_t launch_pair_t(const Gemm& g, cudaStream_t s, const char* name) {
     }
   }
   p.epi = g.epi;
+  p.epi2 = g.has_epi2 ? g.epi2 : g.epi;
+  p.deps = g.deps;
+  p.dep_target = g.dep_target;
+  p.dep_blocks = g.dep_blocks > 0 ? g.dep_blocks : 1;
+  p.c_rel2 = g.c_rel2 ? 1 : 0;
   p.err = device_error_word();
   p.epi_wait_ns = g.epi_wait_ns ? g.epi_wait_ns : kWaitLimitNs;
   auto kern = umma_gemm_pair_kernel<A_MN, B_MN, OUT_F32, B_I8>;
@@ -1924,11 +1989,18 @@ bool pair_supported(const Gemm& g) {
     h.B = g.B2; h.b_rows = g.b2_rows; h.b_cols = g.b2_cols; h.b_ld = g.b2_ld;
     h.A2 = nullptr; h.B2 = nullptr;
     h.groups = g.groups - g.groups_1;
+    h.has_epi2 = false; h.deps = nullptr;
+    if (g.has_epi2) h.epi = g.epi2;
     Gemm f = g;
     f.A2 = nullptr; f.B2 = nullptr;
     f.groups = g.groups_1;
-    return g.B2 && g.groups_1 > 0 && g.groups_1 < g.groups && !g.b_i8 && g.epi.mode == kEpiStore &&
-           pair_supported(f) && pair_supported(h);
+    f.has_epi2 = false; f.deps = nullptr;
+    // epilogue modes per product need fp32 accumulator outputs (the modes' own rule), and a
+    // published dependency needs the first product's stores to be plain stores (fp32 out)
+    const bool modes_ok = g.has_epi2 ? g.out_f32 : g.epi.mode == kEpiStore;
+    return g.B2 && g.groups_1 > 0 && g.groups_1 < g.groups && !g.b_i8 && modes_ok &&
+           (!g.deps || (g.out_f32 && g.dep_target > 0)) && pair_supported(f) &&
+           pair_supported(h);
   }
   return supported(g) && g.N % 256 == 0 && g.M >= 256 && !(g.a_mn && !g.b_mn) &&
          !(g.a_mn && g.b_mn && !g.out_f32) && (g.groups == 1 || g.a_gm == 0 || g.a_gm % 256 == 0);

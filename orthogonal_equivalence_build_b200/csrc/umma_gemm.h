@@ -66,6 +66,19 @@ struct Gemm {
   unsigned long long epi_wait_ns = 0;
   // 256 x 512 kernel only: the two MMAs of a K step share A through the collector buffer
   bool wide_collect = true;
+  // CTA-pair kernel, with a second operand pair: two dependent products in one launch. Groups
+  // >= groups_1 form the second product, with epilogue epi2 (has_epi2) and, with c_rel2,
+  // output groups counted from groups_1. With deps (dep_blocks ints, zero at launch, fp32
+  // outputs), second-product group g starts loading only after deps[(g - groups_1) % dep_blocks]
+  // reached dep_target, which the first product's epilogue warps of group g' = that index
+  // raise by one each after their stores (a 256 x 256 tile has 8 such warps). All clusters are
+  // resident at once and the first product's tiles come first in every cluster's order, so
+  // the waits always end (each is bounded all the same).
+  Epi epi2;
+  bool has_epi2 = false;
+  int* deps = nullptr;
+  int dep_target = 0, dep_blocks = 0;
+  bool c_rel2 = false;
 };
 
 bool supported(const Gemm& g);

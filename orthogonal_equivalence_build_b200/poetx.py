@@ -61,6 +61,8 @@ def _load() -> ctypes.CDLL:
         "poetx_linear_fwd": (I32, [LP, V, I64, V, V, V, SZ, V]),
         "poetx_bwd_workspace_bytes": (SZ, [LP, I64]),
         "poetx_linear_bwd": (I32, [LP, V, V, V, I64, V, V, V, V, SZ, V]),
+        "poetx_linear_fwd_ex": (I32, [LP, V, I64, V, V, V, V, SZ, V]),
+        "poetx_linear_bwd_ex": (I32, [LP, V, V, V, V, I64, V, V, V, V, SZ, V]),
         "poetx_merge_permutations": (I32, [V, V, V, I64, I64, I32, V, V]),
         "poetx_merge_reinit_workspace_bytes": (SZ, [LP]),
         "poetx_merge_reinit": (I32, [LP, U64, V, SZ, V]),
@@ -91,6 +93,7 @@ EXPORTED = (
     "poetx_layer_cnp_workspace_bytes", "poetx_layer_cnp_build",
     "poetx_fwd_workspace_bytes",
     "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
+    "poetx_linear_fwd_ex", "poetx_linear_bwd_ex",
     "poetx_merge_permutations", "poetx_merge_reinit_workspace_bytes", "poetx_merge_reinit",
     "poetx_quantize_w0", "poetx_dequantize_w0", "poetx_resample_permutation", "poetx_validate_permutation", "poetx_device_status",
     "poetx_trace_enable", "poetx_trace_read", "poetx_trace_select", "poetx_status_string",
@@ -219,11 +222,17 @@ def fwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:
 
 def linear_fwd(layer: PoetxLinear, x: torch.Tensor, y: torch.Tensor,
                saved_b: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
-               stream=None) -> None:
+               stream=None, saved_a: Optional[torch.Tensor] = None) -> None:
+    """poetx_linear_fwd; with saved_a [T, m] the forward also keeps A = X[:, perm_r] there
+    (poetx_linear_fwd_ex)."""
     T = x.shape[0]
     ws = _workspace(fwd_workspace_bytes(layer, T), x.device, workspace)
-    _check(lib.poetx_linear_fwd(ctypes.byref(layer.desc), _ptr(x), T, _ptr(y), _ptr(saved_b),
-                                _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+    args = (ctypes.byref(layer.desc), _ptr(x), T, _ptr(y), _ptr(saved_b))
+    tail = (_ptr(ws), 0 if ws is None else ws.numel(), _stream(stream))
+    if saved_a is None:
+        _check(lib.poetx_linear_fwd(*args, *tail))
+    else:
+        _check(lib.poetx_linear_fwd_ex(*args, _ptr(saved_a), *tail))
 
 
 def bwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:
@@ -233,12 +242,19 @@ def bwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:
 def linear_bwd(layer: PoetxLinear, x: torch.Tensor, dy: torch.Tensor, saved_b: torch.Tensor,
                dx: Optional[torch.Tensor], dq_r: Optional[torch.Tensor],
                dq_p: Optional[torch.Tensor], workspace: Optional[torch.Tensor] = None,
-               stream=None) -> None:
-    T = x.shape[0]
-    ws = _workspace(bwd_workspace_bytes(layer, T), x.device, workspace)
-    _check(lib.poetx_linear_bwd(ctypes.byref(layer.desc), _ptr(x), _ptr(dy), _ptr(saved_b), T,
-                                _ptr(dx), _ptr(dq_r), _ptr(dq_p), _ptr(ws),
-                                0 if ws is None else ws.numel(), _stream(stream)))
+               stream=None, saved_a: Optional[torch.Tensor] = None) -> None:
+    """poetx_linear_bwd; with saved_a (the forward's A) the backward reads A from it instead of
+    gathering X again (poetx_linear_bwd_ex)."""
+    T = dy.shape[0]
+    ws = _workspace(bwd_workspace_bytes(layer, T), dy.device, workspace)
+    tail = (T, _ptr(dx), _ptr(dq_r), _ptr(dq_p), _ptr(ws), 0 if ws is None else ws.numel(),
+            _stream(stream))
+    if saved_a is None:
+        _check(lib.poetx_linear_bwd(ctypes.byref(layer.desc), _ptr(x), _ptr(dy), _ptr(saved_b),
+                                    *tail))
+    else:
+        _check(lib.poetx_linear_bwd_ex(ctypes.byref(layer.desc), _ptr(x), _ptr(dy),
+                                       _ptr(saved_b), _ptr(saved_a), *tail))
 
 
 def merge_permutations(w0: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,

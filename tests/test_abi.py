@@ -176,3 +176,22 @@ def test_trace_select_is_host_only_and_accepts_lists():
     assert poetx.lib.poetx_trace_select(b",,x,") == 0
     assert poetx.lib.poetx_trace_select(None) == 0
     assert poetx.lib.poetx_trace_select(b"") == 0
+
+
+def test_saved_a_entry_points_argument_checks():
+    """poetx_linear_fwd_ex / poetx_linear_bwd_ex: x may be NULL in the backward only when
+    saved_a is given; a misaligned saved_a is rejected before any launch."""
+    L = _layer()
+    f = poetx.lib.poetx_linear_fwd_ex
+    assert f(ctypes.byref(L), 0x100000, 128, 0x200000, None, 0x300008, None, 0, None) == 3
+    assert f(ctypes.byref(L), 0x100000, 0, 0x200000, None, 0x300000, None, 0, None) == 0
+    bx = poetx.lib.poetx_linear_bwd_ex
+    need = poetx.lib.poetx_bwd_workspace_bytes(ctypes.byref(L), 128)
+    # neither x nor saved_a
+    assert bx(ctypes.byref(L), None, 0x200000, 0x300000, None, 128, None, None, None,
+              0x400000, need, None) == 1
+    assert bx(ctypes.byref(L), None, 0x200000, 0x300000, 0x500008, 128, None, None, None,
+              0x400000, need, None) == 3
+    # x NULL with saved_a: passes the argument checks (then fails on the workspace size)
+    assert bx(ctypes.byref(L), None, 0x200000, 0x300000, 0x500000, 128, None, None, None,
+              0x400000, need - 1, None) == 8

@@ -315,6 +315,31 @@ def test_backward_without_saved_b_is_identical(key, m, n, b, T):
     assert torch.equal(dx2, dx) and torch.equal(dq_r2, dq_r) and torch.equal(dq_p2, dq_p)
 
 
+@pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 700),
+                                         ("llama1p3b_attn", 512, 768, 128, 333),
+                                         ("tiny_fp32", 256, 512, 64, 99)])
+def test_saved_a_is_the_gather_and_changes_nothing(key, m, n, b, T):
+    """poetx_linear_fwd_ex keeps A = X[:, perm_r] (bit for bit); poetx_linear_bwd_ex reading it
+    (x passed as None) gives the same dX, dq as the backward that gathers X again, with the
+    saved B and with B rebuilt."""
+    c = LayerCase(key, m=m, n=n, b=b, tokens=T)
+    y, bsave = c.forward()
+    a = torch.empty_like(c.x)
+    y2 = torch.empty_like(y)
+    b2 = torch.empty_like(bsave)
+    poetx.linear_fwd(c.layer, c.x, y2, b2, saved_a=a)
+    torch.cuda.synchronize()
+    assert torch.equal(a, c.x[:, c.perm_r.long()])
+    assert torch.equal(y2, y) and torch.equal(b2, bsave)
+    for saved in (bsave, None):
+        dx, dq_r, dq_p = c.backward(saved)
+        dx2 = torch.empty_like(dx)
+        dq_r2, dq_p2 = torch.empty_like(dq_r), torch.empty_like(dq_p)
+        poetx.linear_bwd(c.layer, None, c.dy, saved, dx2, dq_r2, dq_p2, saved_a=a)
+        torch.cuda.synchronize()
+        assert torch.equal(dx2, dx) and torch.equal(dq_r2, dq_r) and torch.equal(dq_p2, dq_p)
+
+
 # ------------------------------------------------------------------ more full-size shapes
 @pytest.mark.parametrize("key,layer", [("llama8b_decoder", 1),    # k_proj 4096 x 1024
                                        ("llama8b_decoder", 6),    # down_proj 14336 x 4096
