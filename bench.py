@@ -307,8 +307,10 @@ def workload_config(wl, args, world):
     cfg = {"workload": wl.key, "linears": [f"{lin.name} {lin.m}x{lin.n}" for lin in lins],
            "b": wl.b, "tokens_per_gpu": T, "global_batch_tokens": T * world,
            "parallelism": f"dp{world}",
-           "step": ("cnp_build(R,P) + " if wl.cnp_in_step else "")
-           + "linear_fwd + linear_bwd(dx, dq) per linear"
+           "step": (("cnp_build(R,P) of all linears in one call + " if len(lins) > 1
+                     else "cnp_build(R,P) + ") if wl.cnp_in_step else "")
+           + ("linear_fwd + linear_bwd(dx, dq) per linear" if len(lins) == 1 else
+              "linear_fwd + linear_bwd_dg(dx, dG) per linear + dq of all linears in one call")
            + ", activations B [T, n] and A = X[:, perm_r] [T, m] kept from forward to backward"
            + (" + NCCL all-reduce of dq" if world > 1 else ""),
            "l2": (f"inputs larger than L2: X + dY = {in_bytes / 2**20:.0f} MiB per step"
@@ -409,6 +411,8 @@ def run_ours(args):
         d["bsave"] = torch.empty(T, lin.n, dtype=dt, device=dev)
         # activations kept from the forward for the backward (POET-Xfast): B, and A = X[:, perm_r]
         d["asave"] = torch.empty(T, lin.m, dtype=dt, device=dev)
+        if nlin > 1:   # per-block gradients, for one dq pass over every linear
+            d["dG"] = torch.empty(lin.m // b + lin.n // b, b, b, device=dev)
         d["dx"] = torch.empty(T, lin.m, dtype=dt, device=dev)
         # dq_r and dq_p are views of one packed buffer: one all-reduce per linear (N > 1)
         d["dq"] = torch.empty(L.q_r.numel() + L.q_p.numel(), device=dev)
@@ -416,9 +420,11 @@ def run_ours(args):
         d["dq_p"] = d["dq"][L.q_r.numel():].view_as(L.q_p)
         layers.append(d)
         poetx.layer_cnp_build(L)
-    ws = torch.empty(max(max(poetx.fwd_workspace_bytes(d["layer"], T),
-                             poetx.bwd_workspace_bytes(d["layer"], T),
-                             poetx.layer_cnp_workspace_bytes(d["layer"])) for d in layers),
+    all_layers = [d["layer"] for d in layers]
+    ws = torch.empty(max(max(max(poetx.fwd_workspace_bytes(d["layer"], T),
+                                 poetx.bwd_workspace_bytes(d["layer"], T)) for d in layers),
+                         poetx.layers_cnp_workspace_bytes(all_layers),
+                         poetx.layers_dq_workspace_bytes(all_layers)),
                      dtype=torch.uint8, device=dev)
     reducer = DqReducer()
     stream = torch.cuda.current_stream(dev)
@@ -427,21 +433,36 @@ def run_ours(args):
 
     def step(xs=None, dys=None, outs=None):
         """One step over every linear; outs[i] = (y, dx, dq) of linear i, dq the packed
-        [dq_r, dq_p] (default: the layer's own result buffers). With N > 1 each linear's dq is
-        summed over the ranks by an all-reduce issued right after its backward, overlapping
-        the next linear's kernels."""
+        [dq_r, dq_p] (default: the layer's own result buffers). One linear: its backward forms
+        dq. Several: each backward stops at the per-block gradients dG and one call forms every
+        linear's dq (more blocks per launch). With N > 1 each linear's dq is summed over the
+        ranks by an all-reduce issued as soon as it exists, overlapping the kernels after it."""
+        if wl.cnp_in_step:
+            # every linear's CNP blocks in one call (one layer: poetx_layer_cnp_build's work)
+            poetx.layers_cnp_build(all_layers, ws)
+        dqs = []
         for i, d in enumerate(layers):
             L = d["layer"]
             xin = d["x"] if xs is None else xs[i]
             dyin = d["dy"] if dys is None else dys[i]
             y, dx, dq = (d["y"], d["dx"], d["dq"]) if outs is None else outs[i]
+            dqs.append(dq)
             nr = L.q_r.numel()
-            if wl.cnp_in_step:
-                poetx.layer_cnp_build(L, ws)
             poetx.linear_fwd(L, xin, y, d["bsave"], ws, saved_a=d["asave"])
-            poetx.linear_bwd(L, xin, dyin, d["bsave"], dx, dq[:nr].view_as(L.q_r),
-                             dq[nr:].view_as(L.q_p), ws, saved_a=d["asave"])
-            reducer.add(dq)
+            if nlin == 1:
+                poetx.linear_bwd(L, xin, dyin, d["bsave"], dx, dq[:nr].view_as(L.q_r),
+                                 dq[nr:].view_as(L.q_p), ws, saved_a=d["asave"])
+                reducer.add(dq)
+            else:
+                poetx.linear_bwd_dg(L, xin, dyin, d["bsave"], dx, d["dG"], ws,
+                                    saved_a=d["asave"])
+        if nlin > 1:
+            poetx.layers_dq_from_dg(all_layers, [d["dG"] for d in layers],
+                                    [dq[:d["layer"].q_r.numel()] for d, dq in zip(layers, dqs)],
+                                    [dq[d["layer"].q_r.numel():] for d, dq in zip(layers, dqs)],
+                                    ws)
+            for dq in dqs:
+                reducer.add(dq)
         reducer.finish()
 
     def barrier():

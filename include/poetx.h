@@ -128,6 +128,20 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t
                                    void* stream);
 
 /* ---------------------------------------------------------------------------------------------
+ * poetx_layers_cnp_build — poetx_layer_cnp_build for a set of layers (a model's linears): every
+ *   layer's R and P blocks, up to eight layers per launch sequence. One layer's blocks fill a
+ *   b x b product launch with a wave or two of tiles; a set of layers gives the products many
+ *   waves. Same arithmetic and bit-identical results as one poetx_layer_cnp_build per layer.
+ *   layers[0 .. nlayers-1]: host array of layer descriptors, all with the same b and dtype
+ *   (else SHAPE / DTYPE), each with q_r and q_p. nlayers = 0 does nothing.
+ *   workspace >= poetx_layers_cnp_workspace_bytes(layers, nlayers) (0 for a bad layer pointer).
+ *   Errors: as poetx_layer_cnp_build for any layer, plus INVALID_ARG for nlayers < 0.
+ * ------------------------------------------------------------------------------------------- */
+size_t poetx_layers_cnp_workspace_bytes(const poetx_layer* const* layers, int32_t nlayers);
+poetx_status poetx_layers_cnp_build(const poetx_layer* const* layers, int32_t nlayers,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------------------------
  * poetx_cnp_build_noalloc — poetx_cnp_build for callers that cannot allocate device memory.
  *   The pages have no counterpart to this call; it exists for library users only. Some callers
  *   may not allocate device memory when they build the blocks (a host program that hands out all
@@ -214,6 +228,29 @@ poetx_status poetx_linear_bwd_ex(const poetx_layer* L, const void* x, const void
                                  const void* saved_b, const void* saved_a, int64_t T, void* dx,
                                  float* dq_r, float* dq_p, void* workspace, size_t ws_bytes,
                                  void* stream);
+
+/* ---------------------------------------------------------------------------------------------
+ * poetx_linear_bwd_dg — poetx_linear_bwd_ex up to the per-block gradients: the backward's
+ *   dL/dG of every block (dG_R^j = A_j^T dA'_j, dG_P^j = B_j^T dC_j, summed over tokens) goes to
+ *   dG [m/b + n/b][b][b] fp32 (the R blocks, then the P blocks) and no dq is formed. dx as in
+ *   poetx_linear_bwd (may be NULL); saved_a as in poetx_linear_bwd_ex (may be NULL).
+ * poetx_layers_dq_from_dg — dq of a set of layers from their dG, one launch sequence over every
+ *   layer's blocks (up to eight layers per sequence): the CNP chain rule of poetx_linear_bwd,
+ *   run over many more blocks at once than one layer's. For a model's linears, call
+ *   poetx_linear_bwd_dg per layer, then this once. Results equal those of poetx_linear_bwd
+ *   (the same chain on the same dG) bit for bit.
+ *   layers [nlayers] (same b and dtype, each with q_r and q_p), dG [nlayers] (as written by
+ *   poetx_linear_bwd_dg, read only), dq_r [nlayers], dq_p [nlayers] outputs (an entry may be
+ *   NULL to skip that side). workspace >= poetx_layers_dq_workspace_bytes(layers, nlayers).
+ *   Errors: as poetx_layers_cnp_build; ALIGN for a dG or dq entry not 16-byte aligned.
+ * ------------------------------------------------------------------------------------------- */
+poetx_status poetx_linear_bwd_dg(const poetx_layer* L, const void* x, const void* dy,
+                                 const void* saved_b, const void* saved_a, int64_t T, void* dx,
+                                 float* dG, void* workspace, size_t ws_bytes, void* stream);
+size_t poetx_layers_dq_workspace_bytes(const poetx_layer* const* layers, int32_t nlayers);
+poetx_status poetx_layers_dq_from_dg(const poetx_layer* const* layers, const float* const* dG,
+                                     float* const* dq_r, float* const* dq_p, int32_t nlayers,
+                                     void* workspace, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------------------------
  * poetx_merge_permutations — W0' = Psi_R W0 Psi_P^T ("POET-X" blog §第二斧: the two permutations

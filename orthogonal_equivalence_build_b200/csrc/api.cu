@@ -429,13 +429,70 @@ poetx_status poetx_layer_cnp_build(const poetx_layer* L, void* workspace, size_t
   if ((st = check_device()) != POETX_OK) return st;
   BlockRuns r;
   const bool lp = L->dtype == POETX_BF16;
-  r.q[0] = L->q_r; r.g[0] = L->g_r; r.nb[0] = r.nb0 = (int)(L->m / L->b);
+  r.q[0] = L->q_r; r.g[0] = L->g_r; r.nb[0] = (int)(L->m / L->b);
   r.q[1] = L->q_p; r.g[1] = L->g_p; r.nb[1] = (int)(L->n / L->b);
   if (lp) {
     r.g_lp[0] = static_cast<__nv_bfloat16*>(L->g_r_lp);
     r.g_lp[1] = static_cast<__nv_bfloat16*>(L->g_p_lp);
   }
   CHECK_CUDA(gemm_cnp_build_runs(r, L->b, workspace, as_stream(stream)), "layer_cnp_build");
+  return POETX_OK;
+}
+
+// Layers whose blocks one launch sequence covers (two runs each: R, then P)
+constexpr int kLayersPerBatch = kMaxRuns / 2;
+
+size_t poetx_layers_cnp_workspace_bytes(const poetx_layer* const* layers, int32_t nlayers) {
+  if (!layers || nlayers <= 0) return 0;
+  size_t need = 0;
+  for (int32_t i0 = 0; i0 < nlayers; i0 += kLayersPerBatch) {
+    int64_t nb = 0, b = 0;
+    for (int32_t i = i0; i < nlayers && i < i0 + kLayersPerBatch; ++i) {
+      const poetx_layer* L = layers[i];
+      if (!L || L->b < 2 || L->m <= 0 || L->n <= 0) return 0;
+      nb += L->m / L->b + L->n / L->b;
+      b = L->b;
+    }
+    need = std::max(need, gemm_cnp_ws_bytes(nb, b));
+  }
+  return need;
+}
+
+poetx_status poetx_layers_cnp_build(const poetx_layer* const* layers, int32_t nlayers,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  if (nlayers < 0) return fail(POETX_ERR_INVALID_ARG, "nlayers < 0");
+  if (nlayers == 0) return POETX_OK;
+  if (!layers) return fail(POETX_ERR_INVALID_ARG, "layers is NULL");
+  for (int32_t i = 0; i < nlayers; ++i) {
+    const poetx_layer* L = layers[i];
+    poetx_status st = check_layer(L, true);
+    if (st != POETX_OK) return st;
+    if (!L->q_r || !L->q_p) return fail(POETX_ERR_INVALID_ARG, "layer %d has no q", (int)i);
+    if (L->b != layers[0]->b)
+      return fail(POETX_ERR_SHAPE, "layer %d has b=%lld, layer 0 b=%lld", (int)i, (long long)L->b,
+                  (long long)layers[0]->b);
+    if (L->dtype != layers[0]->dtype)
+      return fail(POETX_ERR_DTYPE, "layer %d has another dtype than layer 0", (int)i);
+  }
+  poetx_status st = check_ws(workspace, ws_bytes, poetx_layers_cnp_workspace_bytes(layers, nlayers));
+  if (st != POETX_OK) return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  const int64_t b = layers[0]->b;
+  const bool lp = layers[0]->dtype == POETX_BF16;
+  for (int32_t i0 = 0; i0 < nlayers; i0 += kLayersPerBatch) {
+    BlockRuns r;
+    for (int32_t i = i0; i < nlayers && i < i0 + kLayersPerBatch; ++i) {
+      const poetx_layer* L = layers[i];
+      const int k = 2 * (i - i0);
+      r.q[k] = L->q_r; r.g[k] = L->g_r; r.nb[k] = (int)(L->m / b);
+      r.q[k + 1] = L->q_p; r.g[k + 1] = L->g_p; r.nb[k + 1] = (int)(L->n / b);
+      if (lp) {
+        r.g_lp[k] = static_cast<__nv_bfloat16*>(L->g_r_lp);
+        r.g_lp[k + 1] = static_cast<__nv_bfloat16*>(L->g_p_lp);
+      }
+    }
+    CHECK_CUDA(gemm_cnp_build_runs(r, b, workspace, as_stream(stream)), "layers_cnp_build");
+  }
   return POETX_OK;
 }
 
@@ -502,15 +559,21 @@ size_t poetx_bwd_workspace_bytes(const poetx_layer* L, int64_t T) {
 }  // extern "C"
 
 namespace {
+// dG_out: the per-block gradients [m/b + n/b][b][b] are written there (summed over split
+// ranges) and no dq is formed; dq_r / dq_p are then ignored.
 poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy,
                              const void* saved_b, const void* saved_a, int64_t T, void* dx,
                              float* dq_r, float* dq_p, void* workspace, size_t ws_bytes,
-                             void* stream) {
+                             void* stream, float* dG_out = nullptr) {
   poetx_status st = check_layer(L, true);
   if (st != POETX_OK) return st;
   if (T < 0) return fail(POETX_ERR_SHAPE, "T < 0");
+  if (dG_out) dq_r = dq_p = nullptr;
   if ((dq_r && !L->q_r) || (dq_p && !L->q_p))
     return fail(POETX_ERR_INVALID_ARG, "dq requested but the layer has no q");
+  if (dG_out && !aligned16(dG_out)) return fail(POETX_ERR_ALIGN, "dG not 16-byte aligned");
+  // which sides' block gradients are formed
+  const bool want_r = dq_r || dG_out, want_p = dq_p || dG_out;
   if ((!x && !saved_a) || !dy) return fail(POETX_ERR_INVALID_ARG, "x (or saved_a) or dy is NULL");
   if ((x && !aligned16(x)) || !aligned16(dy) || (saved_b && !aligned16(saved_b)) ||
       (saved_a && !aligned16(saved_a)) || (dx && !aligned16(dx)) ||
@@ -529,7 +592,7 @@ poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy
   // A = X[:, perm_r]: the forward's saved copy, or gathered again from X (once, when first needed)
   const void* A = saved_a;
   bool have_a = saved_a != nullptr;
-  if (!saved_b && (dq_p || dq_r)) {
+  if (!saved_b && (want_p || want_r)) {
     // memory-saving mode: rebuild B = (X[:, perm_r] Diag(G_R)) W0' exactly instead of keeping it
     if (!have_a) {
       CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_regather_X"),
@@ -543,12 +606,14 @@ poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy
   }
   CHECK_CUDA(gather_cols(dy, w.dC, T, n, nullptr, L->perm_p, e, s, "perm_bwd_gather_dY"), "bwd gather dY");
   CHECK_CUDA(gemm_blockwise(t, w.dC, Gp, w.dB, T, n, b, true, s), "bwd P blocks");
-  float* dG_r = w.dG;
-  float* dG_p = w.dG + (m / b) * b * b;
+  // the block gradients go straight into dG_out where a launch needs no split partials
+  float* dG_all = dG_out ? dG_out : w.dG;
+  float* dG_r = dG_all;
+  float* dG_p = dG_all + (m / b) * b * b;
   int sp_r = 1, sp_p = 1;
-  // with both dq wanted, dG_R and dG_P run as one launch once dA' exists (bf16, b % 256 == 0)
-  const bool one_dg = dq_r && dq_p && t == DT::BF16 && b % 256 == 0 && T > 0;
-  if (dq_p && !one_dg)
+  // with both sides wanted, dG_R and dG_P run as one launch once dA' exists (bf16, b % 256 == 0)
+  const bool one_dg = want_r && want_p && t == DT::BF16 && b % 256 == 0 && T > 0;
+  if (want_p && !one_dg)
     CHECK_CUDA(gemm_block_grad(t, saved_b, w.dC, dG_p, T, n, b, w.part_p, &sp_p, s), "bwd dG_P");
   CHECK_CUDA(w0_product(L, w.dB, w.dA1, T, true, w.Wd, s), "bwd W0'^T GEMM");
   if (dx) {
@@ -558,7 +623,7 @@ poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy
   }
   bool merged = false;
   int sp_rp = 1;
-  if (dq_r) {
+  if (want_r) {
     if (!have_a) {
       CHECK_CUDA(gather_cols(x, w.A, T, m, nullptr, L->perm_r, e, s, "perm_bwd_gather_X"),
                  "bwd gather X");
@@ -566,7 +631,7 @@ poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy
       have_a = true;
     }
     if (one_dg) {
-      const cudaError_t ce = gemm_block_grad2(t, A, w.dA1, m, saved_b, w.dC, n, w.dG, T, b,
+      const cudaError_t ce = gemm_block_grad2(t, A, w.dA1, m, saved_b, w.dC, n, dG_all, T, b,
                                               w.part_rp, &sp_rp, s);
       if (ce == cudaSuccess) merged = true;
       else if (ce != cudaErrorNotSupported) CHECK_CUDA(ce, "bwd dG_R + dG_P");
@@ -575,6 +640,23 @@ poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy
     }
     if (!merged)
       CHECK_CUDA(gemm_block_grad(t, A, w.dA1, dG_r, T, m, b, w.part_r, &sp_r, s), "bwd dG_R");
+  }
+  if (dG_out) {
+    // the block gradients themselves: partial sums added in split order where there are any
+    const int64_t bb = b * b;
+    if (merged) {
+      if (sp_rp > 1)
+        CHECK_CUDA(sum_partials(static_cast<const float*>(w.part_rp), dG_out,
+                                (m / b + n / b) * bb, sp_rp, s), "dG sum");
+    } else {
+      if (sp_r > 1)
+        CHECK_CUDA(sum_partials(static_cast<const float*>(w.part_r), dG_r, (m / b) * bb, sp_r, s),
+                   "dG_R sum");
+      if (sp_p > 1)
+        CHECK_CUDA(sum_partials(static_cast<const float*>(w.part_p), dG_p, (n / b) * bb, sp_p, s),
+                   "dG_P sum");
+    }
+    return POETX_OK;
   }
   if (dq_r || dq_p) {
     // one dq chain over the R blocks and the P blocks
@@ -600,7 +682,6 @@ poetx_status linear_bwd_impl(const poetx_layer* L, const void* x, const void* dy
         r.parts[k] = sp_p > 1 ? static_cast<const float*>(w.part_p) : dG_p;
       }
     }
-    r.nb0 = r.nb[0];
     CHECK_CUDA(gemm_dq_from_dg_runs(t, r, b, dq_r ? dG_r : dG_p, w.chain, s), "dq chain");
   }
   return POETX_OK;
@@ -623,6 +704,84 @@ poetx_status poetx_linear_bwd_ex(const poetx_layer* L, const void* x, const void
                                  void* stream) {
   return linear_bwd_impl(L, x, dy, saved_b, saved_a, T, dx, dq_r, dq_p, workspace, ws_bytes,
                          stream);
+}
+
+poetx_status poetx_linear_bwd_dg(const poetx_layer* L, const void* x, const void* dy,
+                                 const void* saved_b, const void* saved_a, int64_t T, void* dx,
+                                 float* dG, void* workspace, size_t ws_bytes, void* stream) {
+  if (!dG) return fail(POETX_ERR_INVALID_ARG, "dG is NULL");
+  return linear_bwd_impl(L, x, dy, saved_b, saved_a, T, dx, nullptr, nullptr, workspace,
+                         ws_bytes, stream, dG);
+}
+
+size_t poetx_layers_dq_workspace_bytes(const poetx_layer* const* layers, int32_t nlayers) {
+  if (!layers || nlayers <= 0) return 0;
+  size_t need = 0;
+  for (int32_t i0 = 0; i0 < nlayers; i0 += kLayersPerBatch) {
+    int64_t nb = 0, b = 0;
+    DT t = DT::BF16;
+    for (int32_t i = i0; i < nlayers && i < i0 + kLayersPerBatch; ++i) {
+      const poetx_layer* L = layers[i];
+      if (!L || L->b < 2 || L->m <= 0 || L->n <= 0) return 0;
+      nb += L->m / L->b + L->n / L->b;
+      b = L->b;
+      t = dt_of(L->dtype);
+    }
+    // the chain's own buffers, then the summed gradients it reads in place
+    need = std::max(need, align_up(gemm_dq_ws_bytes(t, nb, b), 256) +
+                              (size_t)(nb * b * b) * sizeof(float));
+  }
+  return need;
+}
+
+poetx_status poetx_layers_dq_from_dg(const poetx_layer* const* layers, const float* const* dG,
+                                     float* const* dq_r, float* const* dq_p, int32_t nlayers,
+                                     void* workspace, size_t ws_bytes, void* stream) {
+  if (nlayers < 0) return fail(POETX_ERR_INVALID_ARG, "nlayers < 0");
+  if (nlayers == 0) return POETX_OK;
+  if (!layers || !dG || !dq_r || !dq_p) return fail(POETX_ERR_INVALID_ARG, "NULL array");
+  for (int32_t i = 0; i < nlayers; ++i) {
+    const poetx_layer* L = layers[i];
+    poetx_status st = check_layer(L, true);
+    if (st != POETX_OK) return st;
+    if (!L->q_r || !L->q_p) return fail(POETX_ERR_INVALID_ARG, "layer %d has no q", (int)i);
+    if (L->b != layers[0]->b)
+      return fail(POETX_ERR_SHAPE, "layer %d has b=%lld, layer 0 b=%lld", (int)i, (long long)L->b,
+                  (long long)layers[0]->b);
+    if (L->dtype != layers[0]->dtype)
+      return fail(POETX_ERR_DTYPE, "layer %d has another dtype than layer 0", (int)i);
+    if (!dG[i]) return fail(POETX_ERR_INVALID_ARG, "dG of layer %d is NULL", (int)i);
+    if (!aligned16(dG[i]) || (dq_r[i] && !aligned16(dq_r[i])) || (dq_p[i] && !aligned16(dq_p[i])))
+      return fail(POETX_ERR_ALIGN, "layer %d: dG / dq not 16-byte aligned", (int)i);
+  }
+  poetx_status st = check_ws(workspace, ws_bytes, poetx_layers_dq_workspace_bytes(layers, nlayers));
+  if (st != POETX_OK) return st;
+  if ((st = check_device()) != POETX_OK) return st;
+  const int64_t b = layers[0]->b;
+  const DT t = dt_of(layers[0]->dtype);
+  for (int32_t i0 = 0; i0 < nlayers; i0 += kLayersPerBatch) {
+    BlockRuns r;
+    int64_t nb = 0;
+    for (int32_t i = i0; i < nlayers && i < i0 + kLayersPerBatch; ++i) {
+      const poetx_layer* L = layers[i];
+      const int k = 2 * (i - i0);
+      // a side whose dq is not wanted takes no blocks
+      if (dq_r[i]) {
+        r.q[k] = L->q_r; r.dq[k] = dq_r[i]; r.nb[k] = (int)(L->m / b); r.parts[k] = dG[i];
+      }
+      if (dq_p[i]) {
+        r.q[k + 1] = L->q_p; r.dq[k + 1] = dq_p[i]; r.nb[k + 1] = (int)(L->n / b);
+        r.parts[k + 1] = dG[i] + (L->m / b) * b * b;
+      }
+      nb += r.nb[k] + r.nb[k + 1];
+    }
+    if (nb == 0) continue;
+    char* base = static_cast<char*>(workspace);
+    float* scratch = reinterpret_cast<float*>(base + align_up(gemm_dq_ws_bytes(t, nb, b), 256));
+    CHECK_CUDA(gemm_dq_from_dg_runs(t, r, b, scratch, workspace, as_stream(stream)),
+               "layers_dq_from_dg");
+  }
+  return POETX_OK;
 }
 
 // ------------------------------------------------------------------ permutations

@@ -135,7 +135,7 @@ __device__ __forceinline__ void zero_counts(int* deps, int ndeps) {
 
 // CNP pass 1: Q_hi, Q_lo [nb][b][b] from the packed strict upper triangles.
 __global__ void __launch_bounds__(kTileThreads)
-split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
+split_q_kernel(const __grid_constant__ BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
                __nv_bfloat16* __restrict__ Qlo, int* __restrict__ deps, int ndeps) {
   pdl_wait();
   pdl_trigger();
@@ -160,7 +160,7 @@ split_q_kernel(const BlockRuns r, int b, __nv_bfloat16* __restrict__ Qhi,
 // dq pass 1: Qh = bf16(Q), Ql = bf16(Q - Qh); dG = sum of the split partials (fixed order),
 // dGh = bf16(dG).
 __global__ void __launch_bounds__(kTileThreads)
-dq_prep_kernel(const BlockRuns r, int b, float* __restrict__ dG,
+dq_prep_kernel(const __grid_constant__ BlockRuns r, int b, float* __restrict__ dG,
                __nv_bfloat16* __restrict__ Qh, __nv_bfloat16* __restrict__ Ql,
                __nv_bfloat16* __restrict__ dGh, int* __restrict__ deps, int ndeps) {
   pdl_wait();
@@ -262,7 +262,7 @@ dq_mid_kernel(const float* __restrict__ dG, const float* __restrict__ T1,
 
 // dq pass 4: U = V - ZQ; dq_ij = U_ij - U_ji (i < j), written packed.
 __global__ void __launch_bounds__(kTileThreads)
-dq_pack_kernel(const BlockRuns r, const float* __restrict__ V, const float* __restrict__ ZQ,
+dq_pack_kernel(const __grid_constant__ BlockRuns r, const float* __restrict__ V, const float* __restrict__ ZQ,
                int b) {
   pdl_wait();
   pdl_trigger();
@@ -406,7 +406,7 @@ size_t cnp_tc_ws_bytes(int64_t nb, int64_t b) {
 }
 
 cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s) {
-  const int64_t nb = (int64_t)r.nb[0] + r.nb[1];
+  const int64_t nb = r.total();
   if (nb == 0) return cudaSuccess;
   const int64_t bb = b * b;
   Arena a(ws, cnp_tc_ws_bytes(nb, b));
@@ -430,9 +430,11 @@ cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s
   three_pass(sh, nb, b);
   sh.epi.mode = umma::kEpiCnpG;
   sh.epi.b = (int)b;
-  sh.epi.nb0 = r.nb0;
   sh.epi.qh = Qst; sh.epi.ql = Qst + nb * bb;
-  for (int k = 0; k < 2; ++k) {
+  sh.epi.nruns = kMaxRuns;
+  for (int k = 0, end = 0; k < kMaxRuns; ++k) {
+    end += r.nb[k];
+    sh.epi.run_end[k] = end;
     sh.epi.g[k] = r.g[k];
     sh.epi.g_lp[k] = r.g_lp[k];
   }
@@ -452,7 +454,7 @@ size_t dq_tc_ws_bytes(int64_t nb, int64_t b) {
 }
 
 cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cudaStream_t s) {
-  const int64_t nb = (int64_t)r.nb[0] + r.nb[1];
+  const int64_t nb = r.total();
   if (nb == 0) return cudaSuccess;
   const int64_t bb = b * b;
   // element offsets of 256-byte-aligned slices: nb * b * b is a multiple of 128 here

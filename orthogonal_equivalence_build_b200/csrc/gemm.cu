@@ -57,6 +57,15 @@ int64_t dg_ctas_per_block(int64_t b) {
 }
 }  // namespace
 
+cudaError_t sum_partials(const float* part, float* out, int64_t count, int splits,
+                         cudaStream_t s) {
+  if (count <= 0) return cudaSuccess;
+  TraceScope tr("sum_split_partials", s);
+  sum_partials_kernel<<<(int)std::min<int64_t>((count + 255) / 256, sms() * 8), 256, 0, s>>>(
+      part, out, count, splits);
+  return cudaGetLastError();
+}
+
 int grad_splits(int64_t nb, int64_t b, int64_t rows) {
   // Split the contraction over tokens so the (group, tile, split) work units fill whole waves of
   // the persistent grid (all units cost the same); each split keeps >= 512 token rows.
@@ -257,7 +266,7 @@ cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv
                            void* ws, cudaStream_t s) {
   if (tc_blocks_supported(b)) {
     BlockRuns r;
-    r.q[0] = q; r.g[0] = g; r.g_lp[0] = g_lp; r.nb[0] = r.nb0 = (int)nb;
+    r.q[0] = q; r.g[0] = g; r.g_lp[0] = g_lp; r.nb[0] = (int)nb;
     return cnp_build_tc(r, b, ws, s);
   }
   return cnp_build(q, nb, b, g, g_lp, ws, s);
@@ -265,7 +274,7 @@ cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv
 
 cudaError_t gemm_cnp_build_runs(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s) {
   if (tc_blocks_supported(b)) return cnp_build_tc(r, b, ws, s);
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < kMaxRuns; ++k) {
     if (!r.nb[k]) continue;
     cudaError_t e = cnp_build(r.q[k], r.nb[k], b, r.g[k], r.g_lp[k], ws, s);
     if (e != cudaSuccess) return e;
@@ -282,7 +291,7 @@ cudaError_t gemm_dq_from_dg_runs(DT t, const BlockRuns& r, int64_t b, float* dG,
   if (t == DT::BF16 && tc_blocks_supported(b)) return dq_from_dg_tc(r, b, dG, ws, s);
   // fp32 layers: per run, sum split partials if any, then the fp32 SIMT chain
   float* dGk = dG;
-  for (int k = 0; k < 2; ++k) {
+  for (int k = 0; k < kMaxRuns; ++k) {
     if (!r.nb[k]) continue;
     const int64_t count = (int64_t)r.nb[k] * b * b;
     const float* src = r.parts[k];

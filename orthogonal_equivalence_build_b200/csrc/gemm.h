@@ -29,6 +29,9 @@ cudaError_t gemm_dense_i8(const void* A, const int8_t* Wq, const float* scale, v
 // bytes), dG is left untouched and *splits_used says how many ranges there are; the consumer
 // (gemm_dq_from_dg) adds them in a fixed order. With one range the result is written to dG.
 int grad_splits(int64_t nb, int64_t b, int64_t rows);
+// out[e] = sum over s < splits of part[s * count + e], in that order (fp32)
+cudaError_t sum_partials(const float* part, float* out, int64_t count, int splits,
+                         cudaStream_t s);
 size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows);
 cudaError_t gemm_block_grad(DT t, const void* A, const void* B, float* dG, int64_t rows,
                             int64_t width, int64_t b, void* partials, int* splits_used,
@@ -48,39 +51,53 @@ bool tc_blocks_supported(int64_t b);
 size_t cnp_tc_ws_bytes(int64_t nb, int64_t b);
 size_t dq_tc_ws_bytes(int64_t nb, int64_t b);
 
-// Up to two runs of b x b blocks handled by one launch sequence (the R and the P blocks of a
-// layer): launch-wide block j < nb[0] is block j of run 0, otherwise block j - nb[0] of run 1.
+// Up to kMaxRuns runs of b x b blocks handled by one launch sequence (the R and the P blocks of
+// a layer, or of several layers): launch-wide block j is block j - (nb[0] + .. + nb[k-1]) of the
+// run k it falls in. Runs with nb = 0 are empty. Kernels take it as a __grid_constant__
+// parameter (indexed in place, not copied per thread).
 struct BlockRuns {
-  const float* q[2] = {nullptr, nullptr};     // packed skew parameters of each run
-  float* g[2] = {nullptr, nullptr};           // fp32 CNP blocks (may be null)
-  __nv_bfloat16* g_lp[2] = {nullptr, nullptr};  // bf16 copies (may be null)
-  float* dq[2] = {nullptr, nullptr};          // packed gradients
-  const float* parts[2] = {nullptr, nullptr}; // dG split partials [splits][nb][b][b]
-  int splits[2] = {1, 1};
-  int64_t split_stride[2] = {0, 0};           // elements between splits (0: nb[run] * b * b)
-  int nb[2] = {0, 0};
-  int nb0 = 0;                                // == nb[0]
+  const float* q[kMaxRuns] = {};        // packed skew parameters of each run
+  float* g[kMaxRuns] = {};              // fp32 CNP blocks (may be null)
+  __nv_bfloat16* g_lp[kMaxRuns] = {};   // bf16 copies (may be null)
+  float* dq[kMaxRuns] = {};             // packed gradients
+  const float* parts[kMaxRuns] = {};    // dG split partials [splits][nb][b][b]
+  int splits[kMaxRuns];
+  int64_t split_stride[kMaxRuns] = {};  // elements between splits (0: nb[run] * b * b)
+  int nb[kMaxRuns] = {};
+  BlockRuns() {
+    for (int& x : splits) x = 1;
+  }
+  int total() const {
+    int t = 0;
+    for (int x : nb) t += x;
+    return t;
+  }
 };
 __device__ __forceinline__ int run_of(const BlockRuns& r, int g, int& local) {
-  if (g < r.nb0) {
-    local = g;
-    return 0;
+  int start = 0;
+#pragma unroll 1
+  for (int k = 0; k < kMaxRuns - 1; ++k) {
+    if (g < start + r.nb[k]) {
+      local = g - start;
+      return k;
+    }
+    start += r.nb[k];
   }
-  local = g - r.nb0;
-  return 1;
+  local = g - start;
+  return kMaxRuns - 1;
 }
 cudaError_t cnp_build_tc(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s);
-// dG: [nb[0] + nb[1]][b][b] fp32, receives the summed gradients (a run whose parts pointer is
+// dG: [total blocks][b][b] fp32, receives the summed gradients (a run whose parts pointer is
 // its own slice of dG with one split is read in place).
 cudaError_t dq_from_dg_tc(const BlockRuns& r, int64_t b, float* dG, void* ws, cudaStream_t s);
 
 size_t gemm_cnp_ws_bytes(int64_t nb, int64_t b);
 cudaError_t gemm_cnp_build(const float* q, int64_t nb, int64_t b, float* g, __nv_bfloat16* g_lp,
                            void* ws, cudaStream_t s);
-// both runs of a layer in one sequence (tensor cores), or one after the other (SIMT)
+// every run in one sequence (tensor cores), or one run after the other (SIMT)
 cudaError_t gemm_cnp_build_runs(const BlockRuns& r, int64_t b, void* ws, cudaStream_t s);
 size_t gemm_dq_ws_bytes(DT t, int64_t nb, int64_t b);
-// dq of the runs in r; dG: [nb[0] + nb[1]][b][b] fp32 scratch that receives summed gradients
+// dq of the runs in r; dG: [total blocks][b][b] fp32 scratch that receives summed gradients
 cudaError_t gemm_dq_from_dg_runs(DT t, const BlockRuns& r, int64_t b, float* dG, void* ws,
                                  cudaStream_t s);
 

@@ -64,6 +64,10 @@ cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Runs of b x b blocks one CNP / dq launch sequence handles (a layer's R and P blocks, or those
+// of up to eight layers).
+constexpr int kMaxRuns = 16;
 // element count rounded up to a multiple of 8 (16-byte aligned offsets for 2- and 4-byte types)
 __host__ __device__ inline int64_t pad8(int64_t x) { return (x + 7) & ~(int64_t)7; }
 

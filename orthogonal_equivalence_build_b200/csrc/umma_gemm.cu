@@ -291,9 +291,18 @@ __device__ __forceinline__ void st8_split(__nv_bfloat16* hi, __nv_bfloat16* lo, 
   *reinterpret_cast<uint4*>(hi) = pack8(h);
   *reinterpret_cast<uint4*>(lo) = pack8(l);
 }
+// Run of CNP output block g (kEpiCnpG) and the first block of that run: resolved once per tile.
+__device__ __forceinline__ int epi_run(const Epi& e, int g, int& first) {
+  int run = 0;
+  first = 0;
+#pragma unroll 1
+  while (run + 1 < e.nruns && g >= e.run_end[run]) first = e.run_end[run++];
+  return run;
+}
+
 __device__ __forceinline__ void epi_apply8(const Epi& e, int g, int i, int j, long long off,
                                            long long bb, const float (&acc)[8],
-                                           const float (&q)[8]) {
+                                           const float (&q)[8], int run, int first) {
   if (e.mode == kEpiCnpS) {
     float h[8];
 #pragma unroll
@@ -304,8 +313,7 @@ __device__ __forceinline__ void epi_apply8(const Epi& e, int g, int i, int j, lo
     float v[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) v[k] = (i == j + k ? 1.f : 0.f) + 2.f * q[k] + acc[k];
-    const int run = g < e.nb0 ? 0 : 1;
-    const long long loc = off - (run ? (long long)e.nb0 * bb : 0);
+    const long long loc = off - (long long)first * bb;
     if (e.g[run]) {
       float4* gp = reinterpret_cast<float4*>(e.g[run] + loc);
       gp[0] = make_float4(v[0], v[1], v[2], v[3]);
@@ -456,6 +464,8 @@ __device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols,
   const long long bb = (long long)e.b * e.b;
   const long long base = fused_base(e, g, row0, col0, lane);
   const int cg = lane & 3;
+  int first = 0;
+  const int run = e.mode == kEpiCnpG ? epi_run(e, g, first) : 0;
 #pragma unroll 1
   for (int cc = 0, half = 0; cc < ncols; cc += 32, half ^= 1) {
     uint32_t r[32];
@@ -485,7 +495,7 @@ __device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols,
           qq[2 * k + 1] = __high2float(h2) + __high2float(l2);
         }
         epi_apply8(e, g, row0 + rr, col0 + cc + 8 * cg, base + (long long)rr * e.b + cc, bb, a,
-                   qq);
+                   qq, run, first);
       }
     }
     if (cc + 32 < ncols) fused_q_load(e, base, cc + 32, nlive, lane, q);
@@ -496,7 +506,7 @@ __device__ __forceinline__ void epilogue_fused(uint32_t tmem_row0, int ncols,
 template <int BN, bool A_MN, bool B_MN, bool OUT_F32, int STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
 umma_gemm_kernel(const __grid_constant__ CUtensorMap tma_a, const __grid_constant__ CUtensorMap tma_b,
-                 const Params p) {
+                 const __grid_constant__ Params p) {
   constexpr int A_BYTES = BM * BK * 2;
   constexpr int B_BYTES = BN * BK * 2;
   constexpr uint32_t TMEM_COLS = 2 * BN;  // power of two: 128, 256 or 512
@@ -896,7 +906,8 @@ umma_gemm_pair_kernel(const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b,
                       const __grid_constant__ CUtensorMap tma_c,
                       const __grid_constant__ CUtensorMap tma_a2,
-                      const __grid_constant__ CUtensorMap tma_b2, const PairParams p) {
+                      const __grid_constant__ CUtensorMap tma_b2,
+                      const __grid_constant__ PairParams p) {
   using Cfg = PairCfg<B_I8, OUT_F32>;
   constexpr int EPI_W = Cfg::EPI_W;
   constexpr int STAGES = Cfg::STAGES;
@@ -1360,7 +1371,8 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
                       const __grid_constant__ CUtensorMap tma_b,
                       const __grid_constant__ CUtensorMap tma_c,
                       const __grid_constant__ CUtensorMap tma_a2,
-                      const __grid_constant__ CUtensorMap tma_b2, const PairParams p) {
+                      const __grid_constant__ CUtensorMap tma_b2,
+                      const __grid_constant__ PairParams p) {
   constexpr int STAGES = WideCfg::STAGES;
   constexpr int A_BYTES = WideCfg::A_BYTES;
   constexpr int B_BYTES = WideCfg::B_BYTES;

@@ -29,17 +29,19 @@ enum EpiMode : int {
   kEpiStore = 0,
   kEpiCnpS = 1,   // acc = S = Q Q: o0, o1 = hi / lo of S; o2, o3 = hi / lo of H = 2I + 2Q + S
   kEpiCnpG = 2,   // acc = S H:  G = I + 2Q + acc to g[run] (fp32) and g_lp[run] (bf16); block g
-                  // is block g of run 0 when g < nb0, else block g - nb0 of run 1
+                  // is block g - run_end[run - 1] of the run with run_end[run - 1] <= g <
+                  // run_end[run] (run_end[-1] = 0), for runs 0 .. nruns - 1
   kEpiDqS = 3,    // acc = S = Q Q: o0 = bf16(S), o1 = bf16(S - 2Q)
 };
 struct Epi {
   int mode = kEpiStore;
-  int b = 0, nb0 = 0;
+  int b = 0, nruns = 1;
   const __nv_bfloat16* qh = nullptr;
   const __nv_bfloat16* ql = nullptr;
   __nv_bfloat16* o[4] = {nullptr, nullptr, nullptr, nullptr};
-  float* g[2] = {nullptr, nullptr};
-  __nv_bfloat16* g_lp[2] = {nullptr, nullptr};
+  float* g[kMaxRuns] = {};
+  __nv_bfloat16* g_lp[kMaxRuns] = {};
+  int run_end[kMaxRuns] = {};
 };
 
 struct Gemm {

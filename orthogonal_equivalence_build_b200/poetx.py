@@ -57,6 +57,12 @@ def _load() -> ctypes.CDLL:
         "poetx_cnp_build_noalloc": (I32, [V, I64, I64, V, V, I32, V]),
         "poetx_layer_cnp_workspace_bytes": (SZ, [LP]),
         "poetx_layer_cnp_build": (I32, [LP, V, SZ, V]),
+        "poetx_layers_cnp_workspace_bytes": (SZ, [ctypes.POINTER(LP), I32]),
+        "poetx_layers_cnp_build": (I32, [ctypes.POINTER(LP), I32, V, SZ, V]),
+        "poetx_linear_bwd_dg": (I32, [LP, V, V, V, V, I64, V, V, V, SZ, V]),
+        "poetx_layers_dq_workspace_bytes": (SZ, [ctypes.POINTER(LP), I32]),
+        "poetx_layers_dq_from_dg": (I32, [ctypes.POINTER(LP), ctypes.POINTER(V),
+                                          ctypes.POINTER(V), ctypes.POINTER(V), I32, V, SZ, V]),
         "poetx_fwd_workspace_bytes": (SZ, [LP, I64]),
         "poetx_linear_fwd": (I32, [LP, V, I64, V, V, V, SZ, V]),
         "poetx_bwd_workspace_bytes": (SZ, [LP, I64]),
@@ -91,6 +97,8 @@ lib = _load()
 EXPORTED = (
     "poetx_cnp_workspace_bytes", "poetx_cnp_build", "poetx_cnp_build_noalloc",
     "poetx_layer_cnp_workspace_bytes", "poetx_layer_cnp_build",
+    "poetx_layers_cnp_workspace_bytes", "poetx_layers_cnp_build",
+    "poetx_linear_bwd_dg", "poetx_layers_dq_workspace_bytes", "poetx_layers_dq_from_dg",
     "poetx_fwd_workspace_bytes",
     "poetx_linear_fwd", "poetx_bwd_workspace_bytes", "poetx_linear_bwd",
     "poetx_linear_fwd_ex", "poetx_linear_bwd_ex",
@@ -216,6 +224,30 @@ def layer_cnp_build(layer: PoetxLinear, workspace: Optional[torch.Tensor] = None
                                      0 if ws is None else ws.numel(), _stream(stream)))
 
 
+def _layer_array(layers):
+    arr = (ctypes.POINTER(Layer) * len(layers))()
+    for i, layer in enumerate(layers):
+        arr[i] = ctypes.pointer(layer.desc)
+    return arr
+
+
+def layers_cnp_workspace_bytes(layers) -> int:
+    arr = _layer_array(layers)
+    return int(lib.poetx_layers_cnp_workspace_bytes(arr, len(layers)))
+
+
+def layers_cnp_build(layers, workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """CNP blocks of every layer in `layers` (PoetxLinear, same b and dtype) in one call
+    (poetx_layers_cnp_build)."""
+    if not layers:
+        return
+    arr = _layer_array(layers)
+    ws = _workspace(int(lib.poetx_layers_cnp_workspace_bytes(arr, len(layers))),
+                    layers[0].w0m.device, workspace)
+    _check(lib.poetx_layers_cnp_build(arr, len(layers), _ptr(ws), 0 if ws is None else ws.numel(),
+                                      _stream(stream)))
+
+
 def fwd_workspace_bytes(layer: PoetxLinear, T: int) -> int:
     return int(lib.poetx_fwd_workspace_bytes(ctypes.byref(layer.desc), T))
 
@@ -255,6 +287,37 @@ def linear_bwd(layer: PoetxLinear, x: torch.Tensor, dy: torch.Tensor, saved_b: t
     else:
         _check(lib.poetx_linear_bwd_ex(ctypes.byref(layer.desc), _ptr(x), _ptr(dy),
                                        _ptr(saved_b), _ptr(saved_a), *tail))
+
+
+def linear_bwd_dg(layer: PoetxLinear, x: Optional[torch.Tensor], dy: torch.Tensor,
+                  saved_b: Optional[torch.Tensor], dx: Optional[torch.Tensor],
+                  dG: torch.Tensor, workspace: Optional[torch.Tensor] = None, stream=None,
+                  saved_a: Optional[torch.Tensor] = None) -> None:
+    """The backward up to the per-block gradients: dG [m/b + n/b, b, b] fp32 (R blocks, then P
+    blocks); no dq (poetx_linear_bwd_dg)."""
+    T = dy.shape[0]
+    ws = _workspace(bwd_workspace_bytes(layer, T), dy.device, workspace)
+    _check(lib.poetx_linear_bwd_dg(ctypes.byref(layer.desc), _ptr(x), _ptr(dy), _ptr(saved_b),
+                                   _ptr(saved_a), T, _ptr(dx), _ptr(dG), _ptr(ws),
+                                   0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def layers_dq_workspace_bytes(layers) -> int:
+    return int(lib.poetx_layers_dq_workspace_bytes(_layer_array(layers), len(layers)))
+
+
+def layers_dq_from_dg(layers, dGs, dq_rs, dq_ps, workspace: Optional[torch.Tensor] = None,
+                      stream=None) -> None:
+    """dq of every layer from its dG in one launch sequence (poetx_layers_dq_from_dg)."""
+    if not layers:
+        return
+    n = len(layers)
+    arr = _layer_array(layers)
+    ptrs = lambda ts: (ctypes.c_void_p * n)(*[_ptr(t) for t in ts])
+    ws = _workspace(int(lib.poetx_layers_dq_workspace_bytes(arr, n)), layers[0].w0m.device,
+                    workspace)
+    _check(lib.poetx_layers_dq_from_dg(arr, ptrs(dGs), ptrs(dq_rs), ptrs(dq_ps), n, _ptr(ws),
+                                       0 if ws is None else ws.numel(), _stream(stream)))
 
 
 def merge_permutations(w0: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,

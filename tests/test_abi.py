@@ -195,3 +195,46 @@ def test_saved_a_entry_points_argument_checks():
     # x NULL with saved_a: passes the argument checks (then fails on the workspace size)
     assert bx(ctypes.byref(L), None, 0x200000, 0x300000, 0x500000, 128, None, None, None,
               0x400000, need - 1, None) == 8
+
+
+def test_layers_cnp_build_argument_checks():
+    """poetx_layers_cnp_build: nlayers = 0 is a no-op; a NULL array, a layer of another b or
+    dtype, or a layer without q are rejected before any launch."""
+    f = poetx.lib.poetx_layers_cnp_build
+    arr = (ctypes.POINTER(poetx.Layer) * 2)()
+    L0, L1 = _layer(), _layer(b=128)
+    arr[0], arr[1] = ctypes.pointer(L0), ctypes.pointer(L1)
+    assert f(arr, 0, None, 0, None) == 0
+    assert f(None, 2, None, 0, None) == 1
+    assert f(arr, -1, None, 0, None) == 1
+    assert f(arr, 2, 0x400000, 1 << 30, None) == 2              # b differs
+    L2 = _layer(dtype=poetx.F32, g_r_lp=None, g_p_lp=None)
+    arr[1] = ctypes.pointer(L2)
+    assert f(arr, 2, 0x400000, 1 << 30, None) == 4              # dtype differs
+    L3 = _layer(q_p=None)
+    arr[1] = ctypes.pointer(L3)
+    assert f(arr, 2, 0x400000, 1 << 30, None) == 1              # no q
+    arr[1] = ctypes.pointer(_layer(m=1024))
+    need = poetx.lib.poetx_layers_cnp_workspace_bytes(arr, 2)
+    assert need > poetx.lib.poetx_layer_cnp_workspace_bytes(ctypes.byref(L0))
+    assert f(arr, 2, 0x400000, need - 1, None) == 8
+
+
+def test_dg_backward_and_layers_dq_argument_checks():
+    L = _layer()
+    need = poetx.lib.poetx_bwd_workspace_bytes(ctypes.byref(L), 128)
+    f = poetx.lib.poetx_linear_bwd_dg
+    assert f(ctypes.byref(L), 0x100000, 0x200000, 0x300000, None, 128, None, None,
+             0x400000, need, None) == 1                       # dG NULL
+    assert f(ctypes.byref(L), 0x100000, 0x200000, 0x300000, None, 128, None, 0x500004,
+             0x400000, need, None) == 3                       # dG misaligned
+    g = poetx.lib.poetx_layers_dq_from_dg
+    arr = (ctypes.POINTER(poetx.Layer) * 1)(ctypes.pointer(L))
+    V1 = ctypes.c_void_p * 1
+    assert g(arr, V1(0x500000), V1(0x600000), V1(0x700000), 0, None, 0, None) == 0
+    assert g(arr, None, V1(0x600000), V1(0x700000), 1, None, 0, None) == 1
+    assert g(arr, V1(None), V1(0x600000), V1(0x700000), 1, None, 0, None) == 1
+    assert g(arr, V1(0x500008), V1(0x600000), V1(0x700000), 1, None, 0, None) == 3
+    need = poetx.lib.poetx_layers_dq_workspace_bytes(arr, 1)
+    assert need > 0
+    assert g(arr, V1(0x500000), V1(0x600000), V1(None), 1, 0x800000, need - 1, None) == 8

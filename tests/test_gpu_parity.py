@@ -282,6 +282,62 @@ def test_layer_cnp_build_matches_per_side_builds(key, m, n, b):
         assert torch.equal(lp_r, lay.g_r_lp) and torch.equal(lp_p, lay.g_p_lp)
 
 
+@pytest.mark.parametrize("key,shapes", [
+    ("llama8b_up_proj", [(1024, 3584), (2048, 1024), (512, 4096)]),
+    ("llama1p3b_attn", [(512, 768)] * 9),          # nine layers: two launch sequences
+    ("tiny_fp32", [(256, 512), (512, 256)]),
+])
+def test_layers_cnp_build_matches_per_layer_builds(key, shapes):
+    """One poetx_layers_cnp_build over a set of layers gives every layer's G blocks (fp32 and
+    bf16) bit for bit as one poetx_layer_cnp_build per layer."""
+    cases = [LayerCase(key, m=m, n=n, tokens=4, seed=1000 + i) for i, (m, n) in enumerate(shapes)]
+    ref = [(c.layer.g_r.clone(), c.layer.g_p.clone(),
+            None if c.layer.g_r_lp is None else c.layer.g_r_lp.clone(),
+            None if c.layer.g_p_lp is None else c.layer.g_p_lp.clone()) for c in cases]
+    for c in cases:
+        for t in (c.layer.g_r, c.layer.g_p, c.layer.g_r_lp, c.layer.g_p_lp):
+            if t is not None:
+                t.fill_(float("nan"))
+    poetx.layers_cnp_build([c.layer for c in cases])
+    torch.cuda.synchronize()
+    for c, (gr, gp, lr, lpp) in zip(cases, ref):
+        assert torch.equal(c.layer.g_r, gr) and torch.equal(c.layer.g_p, gp)
+        if lr is not None:
+            assert torch.equal(c.layer.g_r_lp, lr) and torch.equal(c.layer.g_p_lp, lpp)
+
+
+@pytest.mark.parametrize("key,shapes,T", [
+    ("llama8b_up_proj", [(1024, 3584), (2048, 1024), (512, 4096)], 700),
+    ("llama8b_up_proj", [(1024, 2048), (1024, 1024)], 2305),   # split token ranges
+    ("llama1p3b_attn", [(512, 768)] * 9, 333),                # nine layers: two sequences
+    ("tiny_fp32", [(256, 512), (512, 256)], 99),
+])
+def test_dg_backward_then_layers_dq_matches_per_layer_backward(key, shapes, T):
+    """poetx_linear_bwd_dg per layer (dX and dG) followed by one poetx_layers_dq_from_dg gives
+    the dX and dq of poetx_linear_bwd per layer (equal values), with the saved B and with B
+    rebuilt."""
+    cases = [LayerCase(key, m=m, n=n, tokens=T, seed=2000 + i) for i, (m, n) in enumerate(shapes)]
+    for rebuilt in (False, True):
+        refs, dGs, dxs = [], [], []
+        for c in cases:
+            y, bsave = c.forward()
+            saved = None if rebuilt else bsave
+            refs.append(c.backward(saved))
+            dx = torch.empty_like(c.x)
+            dG = torch.full((c.layer.m // c.b + c.layer.n // c.b, c.b, c.b), float("nan"),
+                            device="cuda")
+            poetx.linear_bwd_dg(c.layer, c.x, c.dy, saved, dx, dG)
+            dGs.append(dG)
+            dxs.append(dx)
+        dq_rs = [torch.empty_like(c.q_r) for c in cases]
+        dq_ps = [torch.empty_like(c.q_p) for c in cases]
+        poetx.layers_dq_from_dg([c.layer for c in cases], dGs, dq_rs, dq_ps)
+        torch.cuda.synchronize()
+        for (dx_ref, dqr_ref, dqp_ref), dx, dqr, dqp in zip(refs, dxs, dq_rs, dq_ps):
+            assert torch.equal(dx, dx_ref)
+            assert torch.equal(dqr, dqr_ref) and torch.equal(dqp, dqp_ref)
+
+
 @pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 700),
                                          ("tiny_fp32", 256, 512, 64, 99)])
 def test_one_sided_dq_matches_two_sided(key, m, n, b, T):
