@@ -143,7 +143,7 @@ def max_over_ranks(value: float, device=None, group=None) -> float:
 
 
 class ClockSampler:
-    """SM clock and clock-event reasons sampled every 20 ms through NVML (read-only queries)
+    """SM clock and clock-event reasons sampled every 5 ms through NVML (read-only queries)
     while the timed region runs."""
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -192,7 +192,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            self._stop.wait(0.02)
+            self._stop.wait(0.005)
 
     def stop(self):
         if self.t is None:
@@ -203,7 +203,7 @@ class ClockSampler:
             return None
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.smax,
                 "reasons": sorted(self.reasons), "samples": len(self.samples),
-                "source": "NVML, 20 ms period, timed region only"}
+                "source": "NVML, 5 ms period, timed region only"}
 
 
 # ----------------------------------------------------------------------------- oracle arm
@@ -673,7 +673,7 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama8b_up_proj", choices=list(W.WORKLOADS))

@@ -67,23 +67,27 @@ cudaError_t sum_partials(const float* part, float* out, int64_t count, int split
 }
 
 int grad_splits(int64_t nb, int64_t b, int64_t rows) {
-  // Split the contraction over tokens so the (group, tile, split) work units fill whole waves of
-  // the persistent grid (all units cost the same); each split keeps >= 512 token rows.
-  const int64_t tiles = nb * dg_ctas_per_block(b);
-  const int64_t waves_unit = sms();
+  // Split the contraction over tokens (each split keeps >= 512 token rows) where that shortens
+  // the launch: a time model over the split count s,
+  //   waves(s) x (64-row K blocks per split) x (one K block of one CTA's tile)
+  //   + the fp32 partial products' traffic (each split's b x b blocks written, then read back
+  //     by the sum; one range writes dG once),
+  // at the per-SM share of the bf16 peak and ~6 TB/s. More splits fill more of the last wave
+  // but every extra range costs 2 nb b^2 4 bytes of HBM traffic.
+  const int64_t ctas = nb * dg_ctas_per_block(b);
+  const int64_t n_sm = sms();
+  const double kb_us = (double)(b * b / dg_ctas_per_block(b)) * 64.0 * 2.0 / 11.0e6;
+  const double part_us = (double)nb * (double)(b * b) * 4.0 / 6.0e6;
   const int64_t max_s = std::max<int64_t>(1, std::min<int64_t>(16, rows / 512));
   int best = 1;
-  double best_eff = 0.0;
+  double best_t = 0.0;
   for (int64_t s = 1; s <= max_s; ++s) {
-    const int64_t units = tiles * s;
-    const int64_t waves = (units + waves_unit - 1) / waves_unit;
-    // efficiency of the last wave, discounted slightly per extra split (partial-sum traffic)
-    const double eff = (double)units / (double)(waves * waves_unit) - 0.05 * (double)(s - 1);
-    if (units < waves_unit) continue;  // below one wave: more splits always help
-    if (eff > best_eff + 1e-9) { best_eff = eff; best = (int)s; }
+    const int64_t waves = (ctas * s + n_sm - 1) / n_sm;
+    const int64_t kblocks = ((rows + s - 1) / s + 63) / 64;
+    const double t = (double)(waves * kblocks) * kb_us + (s == 1 ? 1.0 : 2.0 * (double)s) * part_us;
+    if (s == 1 || t < best_t * 0.98) { best_t = t; best = (int)s; }
   }
-  if (best_eff == 0.0) best = (int)std::min<int64_t>(max_s, (waves_unit + tiles - 1) / tiles);
-  return std::max(1, best);
+  return best;
 }
 
 cudaError_t gemm_blockwise(DT t, const void* A, const void* G, void* C, int64_t rows,

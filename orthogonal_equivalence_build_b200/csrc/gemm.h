@@ -24,7 +24,8 @@ cudaError_t gemm_dense_i8(const void* A, const int8_t* Wq, const float* scale, v
                           int64_t N, int64_t K, bool w_trans, void* deq_ws, cudaStream_t s);
 // dG_j = A_j^T B_j (contraction over the rows): A, B [rows, width], dG [width/b, b, b] fp32.
 // Tensor-core tiles: 256 x 512 CTA pairs for b % 512 == 0, 256 x 256 for b % 256 == 0.
-// bf16 operands split the contraction over `grad_splits` ranges of rows. With more than one
+// bf16 operands split the contraction over `grad_splits` ranges of rows (the count that a time
+// model of the launch plus its partial-sum traffic puts lowest). With more than one
 // range the fp32 partial products go to `partials` ([splits][width/b][b][b], block_grad_ws_bytes
 // bytes), dG is left untouched and *splits_used says how many ranges there are; the consumer
 // (gemm_dq_from_dg) adds them in a fixed order. With one range the result is written to dG.

@@ -393,8 +393,9 @@ def testing_gemm_bf16(a: torch.Tensor, a_mn: bool, b: torch.Tensor, b_mn: bool, 
                       K: int, c: torch.Tensor, splits: int = 1, variant: int = 0,
                       epi_wait_ns: int = 0, stream=None) -> None:
     """Kernel-level hook (include/poetx_testing.h): C = A B on the tcgen05 kernel
-    (variant 0: single CTA, 1: CTA pair); epi_wait_ns > 0 bounds the epilogue's accumulator
-    wait (a test of the timeout path)."""
+    (variant 0: single CTA, 1: CTA pair, 2 / 3: 256 x 512 pair tiles with / without the
+    collector buffer); epi_wait_ns > 0 bounds the epilogue's accumulator wait (a test of the
+    timeout path)."""
     _check(lib.poetx_testing_gemm_bf16(_ptr(a), a.shape[0], a.shape[1], int(a_mn), _ptr(b),
                                        b.shape[0], b.shape[1], int(b_mn), M, N, K, _ptr(c),
                                        int(c.dtype == torch.float32), c.shape[-1], splits,
