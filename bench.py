@@ -670,6 +670,76 @@ def run_ours(args):
     return 0
 
 
+def run_vs_cublas(args):
+    """The library's tensor-core kernels against cuBLAS (torch.matmul / torch.bmm) on the same
+    bf16 operands in the same process, at the workload's shapes: the block-diagonal product of
+    the P side (all n/b blocks of the T-token activation, stacked as one [n/b * T, b] x [b, b]
+    product, and as the strided batched form straight from the [T, n] activation) and the
+    forward W0' product [T, m] x [m, n]. L2 is flushed before every timed launch; medians of
+    --steps launches after --warmup. One JSON line; outputs are compared element by element."""
+    import torch
+    from orthogonal_equivalence_build_b200 import poetx
+    wl = W.WORKLOADS[args.workload]
+    m, n = wl.linears[0].m, wl.linears[0].n
+    b, T = wl.b, args.tokens or wl.tokens
+    nb = n // b
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def med_ms(fn):
+        for _ in range(args.warmup):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(c) for a, c in ev)
+
+    g = torch.Generator(device="cuda").manual_seed(7)
+    out = {"mode": "vs_cublas", "workload": args.workload, "T": T, "m": m, "n": n, "b": b,
+           "l2": "flushed before every launch", "steps": args.steps}
+    # block-diagonal product: bytes read + written, FLOPs
+    A = torch.randn(nb * T, b, device="cuda", generator=g).to(torch.bfloat16)
+    G = (torch.randn(b, b, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+    C, C2 = (torch.empty(nb * T, b, device="cuda", dtype=torch.bfloat16) for _ in range(2))
+    byt, fl = 2.0 * nb * T * b * 2, 2.0 * nb * T * b * b
+    rows = {}
+    ms = med_ms(lambda: poetx.testing_gemm_bf16(A, False, G, True, nb * T, b, b, C, variant=1))
+    rows["ours_block_stacked"] = ms
+    ms = med_ms(lambda: torch.matmul(A, G, out=C2))
+    rows["cublas_block_stacked"] = ms
+    same_block = bool(torch.equal(C, C2))
+    del A, C, C2
+    X = torch.randn(T, n, device="cuda", generator=g).to(torch.bfloat16)
+    Gb = (torch.randn(nb, b, b, device="cuda", generator=g) * 0.05).to(torch.bfloat16)
+    Cb = torch.empty(nb, T, b, device="cuda", dtype=torch.bfloat16)
+    Xv = X.view(T, nb, b).permute(1, 0, 2)
+    rows["cublas_block_bmm_strided"] = med_ms(lambda: torch.bmm(Xv, Gb, out=Cb))
+    del X, Gb, Cb
+    for k in list(rows):
+        ms = rows[k]
+        rows[k] = {"ms": ms, "TB/s": byt / ms / 1e9, "TFLOP/s": fl / ms / 1e9}
+    out["block_product"] = rows
+    out["block_product_outputs_equal"] = same_block
+    # forward W0' product
+    Ap = torch.randn(T, m, device="cuda", generator=g).to(torch.bfloat16)
+    W0 = (torch.randn(m, n, device="cuda", generator=g) * m ** -0.5).to(torch.bfloat16)
+    B1, B2 = (torch.empty(T, n, device="cuda", dtype=torch.bfloat16) for _ in range(2))
+    fl = 2.0 * T * m * n
+    rows = {"ours_w0": med_ms(lambda: poetx.testing_gemm_bf16(Ap, False, W0, True, T, n, m, B1,
+                                                             variant=2)),
+            "cublas_w0": med_ms(lambda: torch.matmul(Ap, W0, out=B2))}
+    out["w0_product"] = {k: {"ms": v, "TFLOP/s": fl / v / 1e9} for k, v in rows.items()}
+    out["w0_outputs_max_rel_diff"] = float((B1.float() - B2.float()).abs().max()
+                                           / B2.float().abs().max())
+    poetx.device_status()
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -687,7 +757,12 @@ def main(argv=None):
                     help="store W0' in 8 bits (int8 + column scales) and time that layer")
     ap.add_argument("--xq-staged", action="store_true",
                     help="with --xq: dequantise W0' into the workspace once per product")
+    ap.add_argument("--vs-cublas", action="store_true",
+                    help="time the block-diagonal and W0' products against cuBLAS on the same "
+                         "operands (one GPU) and print that comparison instead")
     args = ap.parse_args(argv)
+    if args.vs_cublas:
+        return run_vs_cublas(args)
     if args.xq_staged:
         args.xq = True
     if args.warmup < 3 and args.impl == "ours" and not os.environ.get("POETX_BENCH_ALLOW_SHORT"):
