@@ -311,7 +311,9 @@ def workload_config(wl, args, world):
                      else "cnp_build(R,P) + ") if wl.cnp_in_step else "")
            + ("linear_fwd + linear_bwd(dx, dq) per linear" if len(lins) == 1 else
               "linear_fwd + linear_bwd_dg(dx, dG) per linear + dq of all linears in one call")
-           + ", activations B [T, n] and A = X[:, perm_r] [T, m] kept from forward to backward"
+           + (", activation A = X[:, perm_r] [T, m] kept from forward to backward, B [T, n] "
+              "rebuilt in the backward" if getattr(args, "xmem", False) else
+              ", activations B [T, n] and A = X[:, perm_r] [T, m] kept from forward to backward")
            + (" + NCCL all-reduce of dq" if world > 1 else ""),
            "l2": (f"inputs larger than L2: X + dY = {in_bytes / 2**20:.0f} MiB per step"
                   if in_bytes > L2_BYTES else "L2 flushed (2x126 MiB write) between steps")}
@@ -322,6 +324,11 @@ def workload_config(wl, args, world):
             "int8 codes + fp32 column scales, dequantised to bf16 "
             + ("into the workspace once per W0' product (staged)" if args.xq_staged
                else "in the W0' GEMMs' shared-memory operand stages"))
+    if getattr(args, "xmem", False):
+        cfg["saved_b"] = ("none (POET-Xmem): the backward rebuilds B = A' W0' from the kept A; "
+                          "the roofline counts the forward work only")
+    if getattr(args, "fuse_w0p", False):
+        cfg["fused_w0_p"] = "forward W0' product and P-block product in one kernel"
     if wl.merge_every:
         cfg["merge_reinit"] = f"every {wl.merge_every} steps, amortised into ms_per_step"
     return cfg
@@ -400,7 +407,7 @@ def run_ours(args):
             w0m = wq
         L = poetx.PoetxLinear(w0m, pr, pp, torch.from_numpy(p["q_r"]).to(dev),
                               torch.from_numpy(p["q_p"]).to(dev), b, w0m_scale=scale,
-                              staged=args.xq_staged)
+                              staged=args.xq_staged, fused_w0_p=args.fuse_w0p)
         d = {"lin": lin, "layer": L,
              "x_host": torch.from_numpy(a["X"]).to(dt).pin_memory(),
              "dy_host": torch.from_numpy(a["dY"]).to(dt).pin_memory()}
@@ -408,8 +415,9 @@ def run_ours(args):
         d["x"] = d["x_host"].to(dev)
         d["dy"] = d["dy_host"].to(dev)
         d["y"] = torch.empty(T, lin.n, dtype=dt, device=dev)
-        d["bsave"] = torch.empty(T, lin.n, dtype=dt, device=dev)
-        # activations kept from the forward for the backward (POET-Xfast): B, and A = X[:, perm_r]
+        # activations kept from the forward for the backward: B (POET-Xfast; with --xmem it is
+        # not kept and the backward rebuilds it, POET-Xmem), and A = X[:, perm_r]
+        d["bsave"] = None if args.xmem else torch.empty(T, lin.n, dtype=dt, device=dev)
         d["asave"] = torch.empty(T, lin.m, dtype=dt, device=dev)
         if nlin > 1:   # per-block gradients, for one dq pass over every linear
             d["dG"] = torch.empty(lin.m // b + lin.n // b, b, b, device=dev)
@@ -482,7 +490,9 @@ def run_ours(args):
     torch.cuda.synchronize()
     # events only around the dominant kernel inside the timed region: an event between two
     # launches keeps the second from overlapping the first one's tail
+    # (with --xmem the backward's rebuild of B is a third W0' product, "umma_dense_W0")
     w0_names = (("umma_dense_W0_i8", "umma_dense_W0T_i8") if args.xq and not args.xq_staged
+                else ("umma_w0p_fused", "umma_dense_W0T", "umma_dense_W0") if args.fuse_w0p
                 else ("umma_dense_W0", "umma_dense_W0T"))
     poetx.trace_read()
     poetx.trace_select(w0_names)
@@ -539,7 +549,10 @@ def run_ours(args):
     peaks, peak_src = measured_peaks()
     roofline = None
     if w0_ms:
-        flops = sum(2.0 * 2 * T * d["lin"].m * d["lin"].n for d in layers) * args.steps
+        # (the fused forward kernel also does the P-block product: 2 T n b more)
+        flops = sum(2.0 * (3 if args.xmem else 2) * T * d["lin"].m * d["lin"].n
+                    + (2.0 * T * d["lin"].n * b if args.fuse_w0p else 0.0)
+                    for d in layers) * args.steps
         total_ms = sum(w0_ms)
         achieved = flops / (total_ms / 1e3) / 1e12
         # The W0' products are timed inside a sub-second region at the clock the bench samples,
@@ -549,13 +562,15 @@ def run_ours(args):
         peak = peaks["bf16_tflops"]
         roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": None,
-                    "kernel": f"{w0_names[0]} / {w0_names[1]} (B = A' W0', dA' = dB W0'^T)",
+                    "kernel": f"{w0_names[0]} / {w0_names[1]} (B = A' W0'"
+                              + (" with C = B Diag(G_P)" if args.fuse_w0p else "")
+                              + ", dA' = dB W0'^T)",
                     "peak_source": f"{peak_src} bf16_tflops (burst)",
                     "aside_frac_of_sustained_peak": (
                         achieved / peaks["bf16_tflops_sustained"]
                         if "bf16_tflops_sustained" in peaks else None),
                     "avg_launch_ms": total_ms / len(w0_ms), "launches": len(w0_ms)}
-        if nlin == 1:
+        if nlin == 1 and not args.fuse_w0p and not args.xmem:
             roofline["traffic"] = measured_traffic(w0_names, T)
     F = sum(layer_flops(T, d["lin"].m, d["lin"].n, b, wl.cnp_in_step) for d in layers)
     Bb = sum(layer_bytes(T, d["lin"].m, d["lin"].n, b, esz, 1 if args.xq else None)
@@ -757,6 +772,11 @@ def main(argv=None):
                     help="store W0' in 8 bits (int8 + column scales) and time that layer")
     ap.add_argument("--xq-staged", action="store_true",
                     help="with --xq: dequantise W0' into the workspace once per product")
+    ap.add_argument("--xmem", action="store_true",
+                    help="keep no B from the forward (POET-Xmem): the backward rebuilds it")
+    ap.add_argument("--fuse-w0p", action="store_true",
+                    help="set POETX_LAYER_FUSED_W0_P on every linear (the forward's W0' and "
+                         "P-block products in one kernel where it applies)")
     ap.add_argument("--vs-cublas", action="store_true",
                     help="time the block-diagonal and W0' products against cuBLAS on the same "
                          "operands (one GPU) and print that comparison instead")

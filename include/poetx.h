@@ -75,6 +75,15 @@ typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
  * bitwise the same; it needs 2*m*n more workspace bytes and is faster on this part, because
  * the in-kernel conversion is repeated for every row tile of tokens. */
 #define POETX_LAYER_W0M_STAGED 2
+/* poetx_layer.flags bit (may be combined with the others): the forward runs the W0' product and
+ * the P-block product as one kernel wherever that kernel covers the layer (bf16, bf16 W0',
+ * b = 512, T >= 256, m and n multiples of 512; other layers take the two launches). Each 256 x
+ * 512 tile of B = A' W0' spans one P block: it is finished on chip, multiplied by G_P^j there and
+ * only then stored, so B is not read back from HBM, and when saved_b is NULL (POET-Xmem) it is
+ * not written at all (back-to-back fusion, "POET-X" blog §第四斧 / §第五斧). Results are bitwise
+ * those of the two-launch forward. Off by default: on this part the fused kernel's phases
+ * between two tiles are not overlapped with MMAs and it measured slower at the 8B shapes. */
+#define POETX_LAYER_FUSED_W0_P 4
 
 /* One POET-X linear. Every pointer is a device pointer owned by the caller. */
 typedef struct {
@@ -82,7 +91,8 @@ typedef struct {
   int64_t n;       /* out-features: columns of W0 */
   int64_t b;       /* block size; must divide m and n */
   int32_t dtype;   /* poetx_dtype of w0m, activations, saved_b, gradients and g_*_lp */
-  int32_t flags;   /* 0, POETX_LAYER_W0M_I8, or POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED */
+  int32_t flags;   /* 0, POETX_LAYER_W0M_I8, or POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED;
+                      optionally | POETX_LAYER_FUSED_W0_P */
   void* w0m;       /* [m, n] merged weight W0' (see poetx_merge_permutations); int8 codes
                       when flags has POETX_LAYER_W0M_I8 */
   int32_t* perm_r; /* [m] permutation of R: each of 0..m-1 exactly once */

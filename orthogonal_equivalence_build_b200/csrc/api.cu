@@ -156,8 +156,9 @@ poetx_status check_layer(const poetx_layer* L, bool need_lp) {
   if (!L) return fail(POETX_ERR_INVALID_ARG, "layer is NULL");
   if (L->dtype != POETX_F32 && L->dtype != POETX_BF16)
     return fail(POETX_ERR_DTYPE, "unknown layer dtype %d", L->dtype);
-  if (L->flags != 0 && L->flags != POETX_LAYER_W0M_I8 &&
-      L->flags != (POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED))
+  const int32_t storage = L->flags & ~POETX_LAYER_FUSED_W0_P;
+  if (storage != 0 && storage != POETX_LAYER_W0M_I8 &&
+      storage != (POETX_LAYER_W0M_I8 | POETX_LAYER_W0M_STAGED))
     return fail(POETX_ERR_INVALID_ARG, "unknown layer flags %d", L->flags);
   if (L->flags & POETX_LAYER_W0M_I8) {
     if (L->dtype != POETX_BF16)
@@ -530,8 +531,17 @@ poetx_status linear_fwd_impl(const poetx_layer* L, const void* x, int64_t T, voi
   const void* Gp = L->dtype == POETX_BF16 ? L->g_p_lp : (const void*)L->g_p;
   CHECK_CUDA(gather_cols(x, A, T, m, nullptr, L->perm_r, e, s, "perm_fwd_gather_X"), "fwd gather");
   CHECK_CUDA(gemm_blockwise(t, A, Gr, w.A1, T, m, b, false, s), "fwd R blocks");
-  CHECK_CUDA(w0_product(L, w.A1, B, T, false, w.Wd, s), "fwd W0' GEMM");
-  CHECK_CUDA(gemm_blockwise(t, B, Gp, w.C, T, n, b, false, s), "fwd P blocks");
+  // B = A' W0' and C = B Diag(G_P): one kernel where the layer asks for it and it applies (B
+  // written only when the caller keeps it), else two launches
+  const bool fused = (L->flags & POETX_LAYER_FUSED_W0_P) && t == DT::BF16 && !w0m_i8(L) &&
+                     w0_p_fused_supported(w.A1, L->w0m, Gp, saved_b, w.C, T, m, n, b);
+  if (fused) {
+    CHECK_CUDA(gemm_w0_p_fused(w.A1, L->w0m, Gp, saved_b, w.C, T, m, n, b, s),
+               "fwd W0' GEMM + P blocks");
+  } else {
+    CHECK_CUDA(w0_product(L, w.A1, B, T, false, w.Wd, s), "fwd W0' GEMM");
+    CHECK_CUDA(gemm_blockwise(t, B, Gp, w.C, T, n, b, false, s), "fwd P blocks");
+  }
   CHECK_CUDA(scatter_cols(w.C, y, T, n, L->perm_p, e, w.inv, s, "perm_fwd_scatter_Y"), "fwd scatter");
   return POETX_OK;
 }

@@ -181,6 +181,17 @@ cudaError_t gemm_dense_i8(const void* A, const int8_t* Wq, const float* scale, v
   return gemm_dense(DT::BF16, A, W, C, M, N, K, w_trans, s);
 }
 
+bool w0_p_fused_supported(const void* A1, const void* W0, const void* Gp, const void* Bout,
+                          const void* Cout, int64_t T, int64_t m, int64_t n, int64_t b) {
+  return umma::w0p_fused_supported(A1, W0, Gp, Bout, Cout, T, m, n, b);
+}
+
+cudaError_t gemm_w0_p_fused(const void* A1, const void* W0, const void* Gp, void* Bout,
+                            void* Cout, int64_t T, int64_t m, int64_t n, int64_t b,
+                            cudaStream_t s) {
+  return umma::w0p_fused(A1, W0, Gp, Bout, Cout, T, m, n, b, s);
+}
+
 size_t block_grad_ws_bytes(DT t, int64_t width, int64_t b, int64_t rows) {
   if (t != DT::BF16) return 0;
   const int sp = umma::effective_splits(rows, grad_splits(width / b, b, rows));

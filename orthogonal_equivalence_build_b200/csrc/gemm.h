@@ -22,6 +22,13 @@ cudaError_t gemm_dense(DT t, const void* A, const void* W, void* C, int64_t M, i
 bool dense_i8_fused(int64_t M, int64_t N);
 cudaError_t gemm_dense_i8(const void* A, const int8_t* Wq, const float* scale, void* C, int64_t M,
                           int64_t N, int64_t K, bool w_trans, void* deq_ws, cudaStream_t s);
+// C = (A1 W0') Diag(G_P) in one tensor-core kernel (bf16, b = 512; see umma_gemm.h), B = A1 W0'
+// also written to Bout when it is not NULL. Not supported: cudaErrorNotSupported.
+bool w0_p_fused_supported(const void* A1, const void* W0, const void* Gp, const void* Bout,
+                          const void* Cout, int64_t T, int64_t m, int64_t n, int64_t b);
+cudaError_t gemm_w0_p_fused(const void* A1, const void* W0, const void* Gp, void* Bout,
+                            void* Cout, int64_t T, int64_t m, int64_t n, int64_t b,
+                            cudaStream_t s);
 // dG_j = A_j^T B_j (contraction over the rows): A, B [rows, width], dG [width/b, b, b] fp32.
 // Tensor-core tiles: 256 x 512 CTA pairs for b % 512 == 0, 256 x 256 for b % 256 == 0.
 // bf16 operands split the contraction over `grad_splits` ranges of rows (the count that a time

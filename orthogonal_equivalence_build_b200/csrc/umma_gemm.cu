@@ -1643,6 +1643,396 @@ umma_gemm_wide_kernel(const __grid_constant__ CUtensorMap tma_a,
   }
 }
 
+// ------------------------------------------------------------------ W0' -> P-block fused kernel
+// The forward's W0' product and P-block product in one launch, for b = 512 (back-to-back fusion
+// of "POET-X" blog §第四斧 / §第五斧's forward chain): the 256 x 512 pair tile of B = A' W0'
+// whose 512 columns are exactly P block j is finished in TMEM, written once as bf16 into shared
+// memory in the MMA operand layout (and, when the caller keeps B for the backward, to global
+// memory from there), and multiplied by G_P^j right away: C tile = B tile x G_P^j, into the same
+// TMEM columns, then stored. B never makes the HBM round trip between the two products.
+//   Per tile (mb, j) of a CTA pair:
+//     phase 1  B_acc = A'[256 rows] W0'[:, 512 j ..]: the 256 x 512 main loop (4-stage ring)
+//     phase 2  epilogue: B_acc -> bf16 B tile, 8 K-slots of 128 rows x 64 in each CTA's shared
+//              memory (the ring's first 128 KB, idle now), optionally stored to global B;
+//              columns 0-255 (slots 0-3) first, then 256-511
+//     phase 3  C_acc = B tile x G_P^j through four 16 KB G slots (the ring's last 64 KB), one
+//              256-column half of C after the other: C half 0 starts on B slots 0-3 as soon
+//              as B columns 0-255 are out of TMEM (while 256-511 drain), C half 1 writes the
+//              TMEM columns of B half 1; the tensor core reads the B tile of both CTAs
+//     phase 4  epilogue: C_acc -> bf16 C, half 0 while the MMAs of C half 1 run, half 1 while
+//              the next tile's main loop runs on accumulator half 0 (its stages held for half
+//              1 until that half is drained, as in the 256 x 512 kernel)
+//   The ring is busy with the B tile and the G slots from the end of phase 1 to the end of
+//   phase 3: the producer loads G after the main loop's last MMA and the next tile's stages
+//   after phase 3. What stays serial per tile is the drain of B half 0 and the refill of the
+//   ring's first stages.
+struct FusedCfg {
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = 128 * BK * 2;   // 16 KB
+  static constexpr int B_BYTES = 256 * BK * 2;   // 32 KB (N half 0 rows, then N half 1 rows)
+  static constexpr int RING = STAGES * (A_BYTES + B_BYTES);   // 192 KB
+  static constexpr int SLOTS = 8;                              // K slots of the B tile (b = 512)
+  static constexpr int SLOT_BYTES = 128 * BK * 2;              // 16 KB
+  static constexpr int GSLOTS = 4;                             // G slots of one C half's rows
+  static constexpr int G_BYTES = 128 * BK * 2;                 // 16 KB
+  static constexpr int G_OFF = SLOTS * SLOT_BYTES;             // 128 KB
+  static constexpr int EPI_W = 4;
+  static constexpr int THREADS = 64 + 32 * EPI_W;
+  static constexpr size_t SMEM = (size_t)RING + EPI_W * kEpiStageBytes + 1024 + 256;
+};
+static_assert(FusedCfg::G_OFF + FusedCfg::GSLOTS * FusedCfg::G_BYTES <= FusedCfg::RING,
+              "the B tile and the G slots overlay the ring");
+
+// A' [T][m] K-major, W0' [m][n] and the stacked G_P blocks [n][512] N-major; B and C [T][n] bf16.
+__global__ void __launch_bounds__(FusedCfg::THREADS, 1)
+umma_w0p_fused_kernel(const __grid_constant__ CUtensorMap tma_a,
+                      const __grid_constant__ CUtensorMap tma_w,
+                      const __grid_constant__ CUtensorMap tma_g,
+                      const __grid_constant__ CUtensorMap tma_bo,
+                      const __grid_constant__ CUtensorMap tma_co,
+                      const __grid_constant__ PairParams p, int save_b) {
+  constexpr int STAGES = FusedCfg::STAGES;
+  constexpr int A_BYTES = FusedCfg::A_BYTES;
+  constexpr int B_BYTES = FusedCfg::B_BYTES;
+  constexpr int SLOTS = FusedCfg::SLOTS;
+  constexpr int SLOT_BYTES = FusedCfg::SLOT_BYTES;
+  constexpr int GSLOTS = FusedCfg::GSLOTS;
+  constexpr int G_BYTES = FusedCfg::G_BYTES;
+  constexpr int EPI_W = FusedCfg::EPI_W;
+  constexpr uint32_t TMEM_COLS = 512;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sa = smem;                                 // ring: A stages
+  uint8_t* sb = smem + STAGES * A_BYTES;              //       B stages
+  uint8_t* btile = smem;                              // phases 2-3: B tile, SLOTS K slots
+  uint8_t* sg = smem + FusedCfg::G_OFF;               // phase 3: G slots
+  uint8_t* sepi = smem + FusedCfg::RING;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sepi + EPI_W * kEpiStageBytes);
+  uint64_t* full = bars;                       // [STAGES] leader
+  uint64_t* empty = full + STAGES;             // [STAGES] both (multicast commits)
+  uint64_t* gfull = empty + STAGES;            // [GSLOTS] leader
+  uint64_t* gempty = gfull + GSLOTS;           // [GSLOTS] both
+  uint64_t* tfull_b = gempty + GSLOTS;         // B_acc complete, both
+  uint64_t* btile_full = tfull_b + 1;          // [2] B half h out of TMEM and in the B tile,
+                                               //     leader (2 * EPI_W arrivals)
+  uint64_t* tfull_c = btile_full + 2;          // [2] C half h complete, both
+  uint64_t* tempty = tfull_c + 2;              // [2] C half h drained, leader (2 * EPI_W)
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const Ctl ctl{abort_flag, p.err};
+  const int cluster_id = blockIdx.x >> 1, num_clusters = gridDim.x >> 1;
+  const int nk = (p.K + BK - 1) / BK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(full + s), 1);
+      mbar_init(smem_u32(empty + s), 1);
+    }
+    for (int s = 0; s < GSLOTS; ++s) {
+      mbar_init(smem_u32(gfull + s), 1);
+      mbar_init(smem_u32(gempty + s), 1);
+    }
+    mbar_init(smem_u32(tfull_b), 1);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(smem_u32(btile_full + h), 2 * EPI_W);
+      mbar_init(smem_u32(tfull_c + h), 1);
+      mbar_init(smem_u32(tempty + h), 2 * EPI_W);
+    }
+    mbar_init(smem_u32(drain), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync_all();   // barriers of both CTAs initialised before any remote arrive
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  pdl_wait();
+  pdl_trigger();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int it = 0, git = 0, tcount = 0;
+      bool ok = true;
+      for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
+        const TileCoord tc = decode_pair_tile(p, tile);
+        const uint32_t tpar = (uint32_t)tcount & 1u;
+        const int am = tc.mb * 256 + (int)rank * 128;
+        // N half h of P block j: columns 512 j + 256 h + 128 rank .. + 127 of W0', and the same
+        // columns (within the block) of G_P^j, whose K rows start at 512 j
+        const int wn = tc.nb * 512 + (int)rank * 128, gk = tc.nb * 512;
+        // phase 1 (the previous tile's phase 3 has finished with the ring: the wait at the end
+        // of the loop body)
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          // the producers stop only when a wait runs out, never on the abort flag, so that
+          // both CTAs have issued the same loads (see the 256 x 256 pair kernel)
+          if (!wait_bounded(smem_u32(empty + s), ((uint32_t)(it / STAGES) & 1u) ^ 1u, ctl,
+                            kErrProducer, kWaitLimitNs, /*stop_on_abort=*/false)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = map_to_rank(smem_u32(full + s), 0);
+          if (leader) mbar_expect_tx(smem_u32(full + s), 2 * (A_BYTES + B_BYTES));
+          const int k = kb * BK;
+          tma_load_2d_pair(smem_u32(sa + s * A_BYTES), &tma_a, fb, k, am);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t dst = smem_u32(sb + s * B_BYTES + h * (128 * BK * 2));
+            tma_load_2d_pair(dst, &tma_w, fb, wn + 256 * h, k);
+            tma_load_2d_pair(dst + 64 * BK * 2, &tma_w, fb, wn + 256 * h + 64, k);
+          }
+        }
+        if (!ok) break;
+        // phase 3's G, C half 0's 256 columns then half 1's, K blocks in order: after the main
+        // loop's last MMA (the ring's last 64 KB is free then)
+        if (!wait_bounded(smem_u32(tfull_b), tpar, ctl, kErrProducer, kWaitLimitNs,
+                          /*stop_on_abort=*/false)) {
+          ok = false;
+          break;
+        }
+        for (int i = 0; i < 2 * SLOTS; ++i, ++git) {
+          const int h = i / SLOTS, kb = i % SLOTS, gs = git % GSLOTS;
+          if (!wait_bounded(smem_u32(gempty + gs), ((uint32_t)(git / GSLOTS) & 1u) ^ 1u, ctl,
+                            kErrProducer, kWaitLimitNs, /*stop_on_abort=*/false)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = map_to_rank(smem_u32(gfull + gs), 0);
+          if (leader) mbar_expect_tx(smem_u32(gfull + gs), 2 * G_BYTES);
+          const uint32_t dst = smem_u32(sg + gs * G_BYTES);
+          const int gx = 256 * h + 128 * (int)rank;
+          tma_load_2d_pair(dst, &tma_g, fb, gx, gk + kb * BK);
+          tma_load_2d_pair(dst + 64 * BK * 2, &tma_g, fb, gx + 64, gk + kb * BK);
+        }
+        if (!ok) break;
+        // the next tile's stages once phase 3's MMAs are done with the B tile and the G slots
+        if (!wait_bounded(smem_u32(tfull_c + 1), tpar, ctl, kErrProducer, kWaitLimitNs,
+                          /*stop_on_abort=*/false)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!ok && leader) {
+        // the leader's full barriers count both CTAs' bytes: let the armed loads land
+        for (int j = max(0, it - STAGES); j < it; ++j)
+          wait_bounded(smem_u32(full + j % STAGES), (uint32_t)(j / STAGES) & 1u, ctl, 0,
+                       kDrainLimitNs);
+        for (int j = max(0, git - GSLOTS); j < git; ++j)
+          wait_bounded(smem_u32(gfull + j % GSLOTS), (uint32_t)(j / GSLOTS) & 1u, ctl, 0,
+                       kDrainLimitNs);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (leader && lane == 0) {
+      constexpr uint32_t idesc = instr_desc_pair<false, true>();
+      int it = 0, git = 0, tcount = 0;
+      bool ok = true;
+      // the phase-1 MMAs of ring iteration j (K block i of the tile) for accumulator halves
+      // h0 .. h1 - 1
+      auto issue = [&](int j, int i, int h0, int h1) {
+        const int s = j % STAGES;
+        const uint32_t a0 = smem_u32(sa + s * A_BYTES), b0 = smem_u32(sb + s * B_BYTES);
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          const uint64_t ad = smem_desc(a0 + kk * 32, 16, 1024);
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          if (h0 == 0 && h1 == 2) {
+            umma_bf16_pair_coll<1>(tmem_base, ad, wide_b_desc<true>(b0, 0, kk), idesc, acc);
+            umma_bf16_pair_coll<2>(tmem_base + 256, ad, wide_b_desc<true>(b0, 1, kk), idesc, acc);
+          } else {
+            for (int h = h0; h < h1; ++h)
+              umma_bf16_pair(tmem_base + 256 * h, ad, wide_b_desc<true>(b0, h, kk), idesc, acc);
+          }
+        }
+      };
+      for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
+        const uint32_t tpar = (uint32_t)tcount & 1u;
+        // phase 1 on accumulator half 0 once the previous tile's C half 0 is drained; each
+        // stage held (its half-1 MMAs not issued) until C half 1 is drained too
+        if (!wait_bounded(smem_u32(tempty), tpar ^ 1u, ctl, kErrMma, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bool h1_free = false;
+        const int first = it;
+        int held = 0;
+        auto release_held = [&]() {
+          for (int i = 0; i < held; ++i) {
+            issue(first + i, i, 1, 2);
+            umma_commit_pair_both(smem_u32(empty + (first + i) % STAGES));
+          }
+          held = 0;
+        };
+        for (int i = 0; i < nk; ++i, ++it) {
+          const int s = it % STAGES;
+          if (!wait_bounded<false>(smem_u32(full + s), (uint32_t)(it / STAGES) & 1u, ctl, kErrMma,
+                                   kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (!h1_free && mbar_test_wait(smem_u32(tempty + 1), tpar ^ 1u)) {
+            h1_free = true;
+            tc_fence_after();
+            release_held();
+          }
+          if (h1_free) {
+            issue(it, i, 0, 2);
+            umma_commit_pair_both(smem_u32(empty + s));
+          } else {
+            issue(it, i, 0, 1);
+            if (++held == STAGES) {
+              if (!wait_bounded(smem_u32(tempty + 1), tpar ^ 1u, ctl, kErrMma, kWaitLimitNs)) {
+                ok = false;
+                break;
+              }
+              h1_free = true;
+              tc_fence_after();
+              release_held();
+            }
+          }
+        }
+        if (!ok) break;
+        if (!h1_free) {   // K shorter than the ring
+          if (!wait_bounded(smem_u32(tempty + 1), tpar ^ 1u, ctl, kErrMma, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          release_held();
+        }
+        umma_commit_pair_both(smem_u32(tfull_b));
+        // phase 3: C half h = B tile x G_P^j[:, 256 h ..], 16 G slots in order; C half 0
+        // needs B half 0 out of TMEM (its columns) and B slots 0-3, then slots 4-7 (B half 1
+        // written), which C half 1's columns need too. Acquire at cluster scope: the peer's
+        // epilogue wrote its half of the operand.
+        for (int i = 0; i < 2 * SLOTS; ++i, ++git) {
+          const int h = i / SLOTS, kb = i % SLOTS, gs = git % GSLOTS;
+          if (i == 0 || i == SLOTS / 2) {
+            if (!wait_bounded<true>(smem_u32(btile_full + (i ? 1 : 0)), tpar, ctl, kErrMma,
+                                    kWaitLimitNs)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          if (!wait_bounded<false>(smem_u32(gfull + gs), (uint32_t)(git / GSLOTS) & 1u, ctl,
+                                   kErrMma, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(btile + kb * SLOT_BYTES), b0 = smem_u32(sg + gs * G_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(tmem_base + 256 * h, smem_desc(a0 + kk * 32, 16, 1024),
+                           wide_b_desc<true>(b0, 0, kk), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair_both(smem_u32(gempty + gs));
+          if (kb == SLOTS - 1) umma_commit_pair_both(smem_u32(tfull_c + h));
+        }
+      }
+      umma_commit_pair_both(smem_u32(drain));
+      wait_bounded(smem_u32(drain), 0, ctl, ok ? kErrMma : 0, ok ? kWaitLimitNs : kDrainLimitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // TMEM lanes 32 * (warp % 4) .. + 31: rows quarter * 32 + lane of this CTA's 128
+    const int quarter = warp & 3;
+    const uint32_t leader_btile = map_to_rank(smem_u32(btile_full), 0);
+    const uint32_t leader_tempty = map_to_rank(smem_u32(tempty), 0);
+    int tcount = 0, chunk = 0;
+    bool ok = true;
+    for (int tile = cluster_id; ok && tile < p.total_tiles; tile += num_clusters, ++tcount) {
+      const TileCoord tc = decode_pair_tile(p, tile);
+      const uint32_t tpar = (uint32_t)tcount & 1u;
+      const int row0 = tc.mb * 256 + (int)rank * 128 + quarter * 32;
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16);
+      // phase 2: B_acc -> the B tile (slot c holds columns 64 c .. 64 c + 63, K-major, 128-byte
+      // rows with 16-byte unit v of row r at v ^ (r & 7)), and to global B when it is kept
+      if (!wait_bounded(smem_u32(tfull_b), tpar, ctl, kErrEpilogue, p.epi_wait_ns)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < SLOTS; ++c) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(trow + (uint32_t)(64 * c), r0);
+        tmem_ld32(trow + (uint32_t)(64 * c + 32), r1);
+        uint8_t* part = btile + c * SLOT_BYTES + quarter * 32 * 128;   // this warp's 32 rows
+        uint8_t* myrow = part + lane * 128;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+          const uint32_t* src = v < 4 ? &r0[8 * v] : &r1[8 * (v - 4)];
+          *reinterpret_cast<uint4*>(myrow + ((v ^ (lane & 7)) * 16)) = make_uint4(
+              pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1])),
+              pack_bf16x2(__uint_as_float(src[2]), __uint_as_float(src[3])),
+              pack_bf16x2(__uint_as_float(src[4]), __uint_as_float(src[5])),
+              pack_bf16x2(__uint_as_float(src[6]), __uint_as_float(src[7])));
+        }
+        // visible to the tensor core's reads and to the copy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (save_b && lane == 0) {
+          tma_store_2d(&tma_bo, smem_u32(part), tc.nb * 512 + 64 * c, row0);
+          bulk_commit();
+        }
+        if (c == SLOTS / 2 - 1 || c == SLOTS - 1) {
+          // B half (c == 3 ? 0 : 1) read out of TMEM and in the B tile; before the second
+          // arrive the B stores have finished reading the tile (the ring is refilled only
+          // after phase 3, which waits for that arrive)
+          tc_fence_before();
+          if (lane == 0) {
+            if (c == SLOTS - 1) bulk_wait_read<0>();
+            mbar_arrive_remote(leader_btile + (uint32_t)(c == SLOTS - 1 ? 8 : 0));
+          }
+          __syncwarp();
+        }
+      }
+      // phase 4: C half h -> C, each half handed back as soon as it is out of TMEM
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        if (!wait_bounded(smem_u32(tfull_c + h), tpar, ctl, kErrEpilogue, p.epi_wait_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        epilogue_tma_bf16(trow + (uint32_t)(256 * h), 256, sepi + (warp - 2) * kEpiStageBytes,
+                          &tma_co, tc.nb * 512 + 256 * h, row0, lane, chunk);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote_relaxed(leader_tempty + (uint32_t)(h * 8));
+      }
+    }
+    if (lane == 0) bulk_wait_all();   // every store written before the CTA leaves
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync_all();   // no remote arrive or copy may target a CTA that has left
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ------------------------------------------------------------------ host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -1917,6 +2307,61 @@ cudaError_t launch_wide_t(const Gemm& g, cudaStream_t s, const char* name) {
   return cudaGetLastError();
 }
 
+cudaError_t launch_w0p_fused(const void* A1, const void* W0, const void* Gp, void* Bout,
+                             void* Cout, int64_t T, int64_t m, int64_t n, cudaStream_t s) {
+  constexpr size_t smem = FusedCfg::SMEM;
+  CUtensorMap ta, tw, tg, tbo, tco;
+  if (!make_map(&ta, A1, T, m, m, 128) || !make_map(&tw, W0, m, n, n, BK) ||
+      !make_map(&tg, Gp, n, 512, 512, BK) || !make_map(&tco, Cout, T, n, n, 32))
+    return cudaErrorInvalidValue;
+  tbo = tco;
+  if (Bout && !make_map(&tbo, Bout, T, n, n, 32)) return cudaErrorInvalidValue;
+  PairParams p{};
+  p.M = (int)T; p.N = (int)n; p.K = (int)m; p.groups = 1; p.g2 = 1;
+  p.tiles_m = (int)((T + 255) / 256);
+  p.tiles_n = (int)(n / 512);   // one tile column per P block
+  p.splits = 1;
+  p.kblocks_per_split = (int)((m + BK - 1) / BK);
+  p.total_tiles = p.tiles_m * p.tiles_n;
+  p.narrow_from = p.total_tiles;
+  p.nseg = 1; p.kb_per_seg = p.kblocks_per_split;
+  p.C = Cout; p.ldc = n;
+  // the W0' product's forward raster: bands of 16 pair-rows sweep the P blocks
+  p.raster = 0;
+  p.band = 16;
+  p.err = device_error_word();
+  p.epi_wait_ns = kWaitLimitNs;
+  auto kern = umma_w0p_fused_kernel;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  set_pdl_attr(attr[1]);
+  cfg.blockDim = dim3(FusedCfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static int max_clusters = 0;
+  if (!max_clusters) {
+    cfg.gridDim = dim3(2 * 74, 1, 1);
+    if (cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg) != cudaSuccess ||
+        max_clusters <= 0)
+      max_clusters = sm_count() / 2;
+  }
+  cfg.numAttrs = 2;
+  const int clusters = std::min(p.total_tiles, max_clusters);
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  TraceScope t("umma_w0p_fused", s);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tw, tg, tbo, tco, p, Bout ? 1 : 0);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int BN>
 cudaError_t dispatch_majors(const Gemm& g, cudaStream_t s) {
 #define POETX_UM(AM, BMJ, F)                                                                   \
@@ -2078,6 +2523,22 @@ cudaError_t gemm_wide(const Gemm& g, cudaStream_t s) {
   POETX_UW(true, true, true, true)
 #undef POETX_UW
   return cudaErrorNotSupported;
+}
+
+bool w0p_fused_supported(const void* A1, const void* W0, const void* Gp, const void* Bout,
+                         const void* Cout, int64_t T, int64_t m, int64_t n, int64_t b) {
+  if (!encode_fn() || b != 512 || T < 256 || m < 512 || n < 512 || m % 512 || n % 512) return false;
+  const int64_t lim = (int64_t)1 << 31;
+  if (T >= lim || m >= lim || n >= lim) return false;
+  return ((reinterpret_cast<uintptr_t>(A1) | reinterpret_cast<uintptr_t>(W0) |
+           reinterpret_cast<uintptr_t>(Gp) | reinterpret_cast<uintptr_t>(Bout) |
+           reinterpret_cast<uintptr_t>(Cout)) & 15) == 0;
+}
+
+cudaError_t w0p_fused(const void* A1, const void* W0, const void* Gp, void* Bout, void* Cout,
+                      int64_t T, int64_t m, int64_t n, int64_t b, cudaStream_t s) {
+  if (!w0p_fused_supported(A1, W0, Gp, Bout, Cout, T, m, n, b)) return cudaErrorNotSupported;
+  return launch_w0p_fused(A1, W0, Gp, Bout, Cout, T, m, n, s);
 }
 
 cudaError_t gemm(const Gemm& g, cudaStream_t s) {

@@ -92,6 +92,14 @@ cudaError_t gemm_pair(const Gemm& g, cudaStream_t s);
 // tiles with one 512-column accumulator in two halves; needs N % 512 == 0 and M >= 256.
 bool wide_supported(const Gemm& g);
 cudaError_t gemm_wide(const Gemm& g, cudaStream_t s);
+// The forward's W0' product and P-block product in one launch (b = 512, bf16): C = (A1 W0')
+// Diag(G_P) with A1 [T][m], W0' [m][n], the stacked bf16 G_P blocks Gp [n][512] (block j in rows
+// 512 j ..), C [T][n]; Bout, when not NULL, also receives B = A1 W0' [T][n]. T >= 256, m and n
+// multiples of 512, 16-byte aligned pointers.
+bool w0p_fused_supported(const void* A1, const void* W0, const void* Gp, const void* Bout,
+                         const void* Cout, int64_t T, int64_t m, int64_t n, int64_t b);
+cudaError_t w0p_fused(const void* A1, const void* W0, const void* Gp, void* Bout, void* Cout,
+                      int64_t T, int64_t m, int64_t n, int64_t b, cudaStream_t s);
 
 // Number of K ranges the kernel actually uses for `splits` requested ranges over K
 // (ranges of whole 64-wide K blocks, none empty).

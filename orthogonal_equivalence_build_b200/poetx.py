@@ -41,6 +41,7 @@ class Layer(ctypes.Structure):
 
 LAYER_W0M_I8 = 1
 LAYER_W0M_STAGED = 2
+LAYER_FUSED_W0_P = 4
 
 
 def _load() -> ctypes.CDLL:
@@ -150,12 +151,14 @@ class PoetxLinear:
     w0m [m, n] (dtype), perm_r [m], perm_p [n] (int32), q_r [m/b, b(b-1)/2], q_p (fp32),
     g_r [m/b, b, b], g_p (fp32) and, for bf16 layers, g_r_lp / g_p_lp (bf16).
     An int8 w0m with its fp32 column scales w0m_scale [n] makes an 8-bit-weight layer
-    (POETX_LAYER_W0M_I8; activations and gradients bf16).
+    (POETX_LAYER_W0M_I8; activations and gradients bf16). fused_w0_p sets
+    POETX_LAYER_FUSED_W0_P (the forward's W0' and P-block products as one kernel).
     """
 
     def __init__(self, w0m: torch.Tensor, perm_r: torch.Tensor, perm_p: torch.Tensor,
                  q_r: torch.Tensor, q_p: torch.Tensor, b: int,
-                 w0m_scale: Optional[torch.Tensor] = None, staged: bool = False):
+                 w0m_scale: Optional[torch.Tensor] = None, staged: bool = False,
+                 fused_w0_p: bool = False):
         m, n = w0m.shape
         dev = w0m.device
         self.b = int(b)
@@ -171,7 +174,8 @@ class PoetxLinear:
         self.g_r_lp = torch.empty(m // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
         self.g_p_lp = torch.empty(n // b, b, b, dtype=torch.bfloat16, device=dev) if lp else None
         self.desc = Layer(m=m, n=n, b=self.b, dtype=BF16 if i8 else dtype_code(w0m.dtype),
-                          flags=(LAYER_W0M_I8 | (LAYER_W0M_STAGED if staged else 0)) if i8 else 0,
+                          flags=(((LAYER_W0M_I8 | (LAYER_W0M_STAGED if staged else 0)) if i8
+                                  else 0) | (LAYER_FUSED_W0_P if fused_w0_p else 0)),
                           w0m=_ptr(w0m), perm_r=_ptr(perm_r), perm_p=_ptr(perm_p),
                           q_r=_ptr(q_r), q_p=_ptr(q_p), g_r=_ptr(self.g_r), g_p=_ptr(self.g_p),
                           g_r_lp=_ptr(self.g_r_lp), g_p_lp=_ptr(self.g_p_lp),

@@ -57,7 +57,8 @@ def _fwd(L, x=0x100000, T=128, y=0x200000, ws=None, wsb=0):
     (dict(perm_r=0x20004), 3),                  # misaligned
     (dict(b=2048, m=4096, n=4096), 2),          # b too large
     (dict(flags=2), 1),                         # staged without the int8 flag
-    (dict(flags=4), 1),                         # unknown flag
+    (dict(flags=8), 1),                         # unknown flag
+    (dict(flags=6), 1),                         # staged without the int8 flag, fused
     (dict(flags=1, w0m_scale=0xA0000, dtype=poetx.F32), 4),   # int8 W0' needs a bf16 layer
     (dict(flags=1, w0m_scale=0xA0004), 3),      # misaligned scales
     (dict(flags=1, w0m_scale=0xA0000, m=520, n=1040, b=8), 2),  # int8 W0' rows of 16 bytes
@@ -76,6 +77,11 @@ def test_forward_argument_checks():
     assert need > 0
     assert _fwd(L, ws=0x400000, wsb=need - 1) == 8
     assert _fwd(L, ws=None, wsb=need) == 8
+    # POETX_LAYER_FUSED_W0_P alone or with the 8-bit bits is a valid layer (the call then
+    # stops at the missing workspace)
+    for flags, scale in ((4, None), (5, 0xA0000), (7, 0xA0000)):
+        Lf = _layer(flags=flags, w0m_scale=scale)
+        assert _fwd(Lf, ws=None, wsb=need) == 8
 
 
 def test_backward_argument_checks():

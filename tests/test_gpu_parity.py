@@ -170,6 +170,52 @@ def test_memory_saving_backward_matches_oracle(key, m, n, b, T, tol):
     _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), tol, xmem=True)
 
 
+# ------------------------------------------------------------------ W0' -> P-block fusion
+def _fused_twin(c: LayerCase):
+    """The same layer (same device tensors) with POETX_LAYER_FUSED_W0_P set."""
+    f = poetx.PoetxLinear(c.layer.w0m, c.perm_r, c.perm_p, c.q_r, c.q_p, c.b, fused_w0_p=True)
+    poetx.layer_cnp_build(f)
+    return f
+
+
+@pytest.mark.parametrize("m,n,T", [(1024, 2048, 1000), (512, 1536, 256), (2048, 1024, 300)])
+def test_fused_w0_p_forward_matches_oracle_and_two_launch_forward(m, n, T):
+    """The forward with the W0' product and the P-block product in one kernel: Y and the saved
+    B bit for bit those of the two-launch forward (same MMAs, same K order), Y within the bf16
+    bar of the oracle, and with saved_b = NULL (B never written) the same Y."""
+    c = LayerCase("llama8b_up_proj", m=m, n=n, b=512, tokens=T, seed=4000 + m + n + T)
+    y0, b0 = c.forward()
+    f = _fused_twin(c)
+    y1 = torch.full_like(y0, float("nan"))
+    b1 = torch.full_like(b0, float("nan"))
+    poetx.linear_fwd(f, c.x, y1, b1)
+    y2 = torch.full_like(y0, float("nan"))
+    poetx.linear_fwd(f, c.x, y2, None)
+    torch.cuda.synchronize()
+    poetx.device_status()
+    assert torch.equal(y1, y0) and torch.equal(b1, b0) and torch.equal(y2, y0)
+    h = c.host()
+    ref = O.linear_fwd(h["X"], h["W0m"], h["perm_r"], h["perm_p"], O.cnp(h["q_r"], c.b),
+                       O.cnp(h["q_p"], c.b))
+    assert rel_err(y1, ref["Y"]) <= TOL_BF16
+
+
+@pytest.mark.slow
+def test_fused_w0_p_forward_many_tiles_per_cluster_matches_two_launch_forward():
+    """16384 tokens x 8 P blocks: 512 tiles, several per CTA pair, so the ring, the B tile and
+    the G slots are handed from tile to tile; bit for bit the two-launch forward, and the
+    backward from the fused forward's saved B is the same too."""
+    c = LayerCase("llama8b_up_proj", m=1024, n=4096, b=512, tokens=16384, seed=4242)
+    y0, b0 = c.forward()
+    f = _fused_twin(c)
+    y1 = torch.full_like(y0, float("nan"))
+    b1 = torch.full_like(b0, float("nan"))
+    poetx.linear_fwd(f, c.x, y1, b1)
+    torch.cuda.synchronize()
+    poetx.device_status()
+    assert torch.equal(y1, y0) and torch.equal(b1, b0)
+
+
 # ------------------------------------------------------------------ merge-then-reinitialize
 @pytest.mark.parametrize("key,m,n,b,tol", [("tiny_fp32", None, None, None, TOL_F32),
                                            ("llama1p3b_attn", 512, 768, 128, TOL_BF16)])
