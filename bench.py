@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 import poetx_workloads as W  # noqa: E402
 
 METRIC = "POET-X linear fwd+bwd tokens/s at Llama-8B shapes; % of 1-B200 roofline"
+DEFAULT_WORKLOAD = "llama8b_up_proj"
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -678,11 +679,46 @@ def run_ours(args):
                                  f"{n_pass} steps after the timed region (which records events "
                                  "around the W0' GEMMs only)"),
         }
+        if (world == 1 and args.other_configs and args.workload == DEFAULT_WORKLOAD
+                and not (args.xq or args.xmem or args.fuse_w0p or args.tokens)):
+            line["other_configs"] = other_configs(args)
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     return 0
+
+
+OTHER_WORKLOADS = ("llama1p3b_attn", "llama8b_decoder", "llama13b_layers")
+
+
+def other_configs(args):
+    """The other bf16 workloads, each measured by this script in a process of its own after the
+    headline run (same GPU, default steps unless fewer are asked): a summary of each one's line
+    (its step time, tokens/s, step roofline fraction, W0' rate and clocks), so that one run of
+    the benchmark reports every configuration. A workload that fails is reported as such."""
+    import subprocess
+    out = {}
+    for key in OTHER_WORKLOADS:
+        cmd = [sys.executable, os.path.abspath(__file__), "--workload", key, "--no-cpu-baseline",
+               "--no-other-configs", "--steps", str(args.steps), "--warmup", str(args.warmup)]
+        try:
+            r = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
+            lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+            if r.returncode != 0 or not lines:
+                out[key] = {"error": f"exit {r.returncode}: " + (r.stderr.strip().splitlines()
+                                                                 or ["no output"])[-1][:200]}
+                continue
+            d = json.loads(lines[-1])
+            rl = d.get("roofline") or {}
+            out[key] = {"ms_per_step": d["ms_per_step"], "value": d["value"], "unit": d["unit"],
+                        "steps": d["steps"], "step_roofline_frac": d["step_roofline"]["frac"],
+                        "w0_tflops": rl.get("achieved"), "clocks": d.get("clocks"),
+                        "e2e": (d.get("e2e") or {}).get("value"),
+                        "linears": d["config"].get("linears")}
+        except Exception as ex:   # a timeout or an unparsable line: reported, not fatal
+            out[key] = {"error": f"{type(ex).__name__}: {ex}"[:200]}
+    return out
 
 
 def run_vs_cublas(args):
@@ -761,7 +797,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama8b_up_proj", choices=list(W.WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(W.WORKLOADS))
     ap.add_argument("--tokens", type=int, default=0, help="override tokens per GPU")
     ap.add_argument("--ref-tokens", type=int, default=256,
                     help="tokens in the oracle's bounded sample")
@@ -772,6 +808,9 @@ def main(argv=None):
                     help="store W0' in 8 bits (int8 + column scales) and time that layer")
     ap.add_argument("--xq-staged", action="store_true",
                     help="with --xq: dequantise W0' into the workspace once per product")
+    ap.add_argument("--no-other-configs", dest="other_configs", action="store_false",
+                    help="with the default workload on one GPU, do not also run the other bf16 "
+                         "workloads (each in a process of its own) for the other_configs key")
     ap.add_argument("--xmem", action="store_true",
                     help="keep no B from the forward (POET-Xmem): the backward rebuilds it")
     ap.add_argument("--fuse-w0p", action="store_true",
