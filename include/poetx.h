@@ -81,8 +81,9 @@ typedef enum { POETX_F32 = 0, POETX_BF16 = 1 } poetx_dtype;
  * 512 tile of B = A' W0' spans one P block: it is finished on chip, multiplied by G_P^j there and
  * only then stored, so B is not read back from HBM, and when saved_b is NULL (POET-Xmem) it is
  * not written at all (back-to-back fusion, "POET-X" blog §第四斧 / §第五斧). Results are bitwise
- * those of the two-launch forward. Off by default: on this part the fused kernel's phases
- * between two tiles are not overlapped with MMAs and it measured slower at the 8B shapes. */
+ * those of the two-launch forward. Off by default: on this part the drain of B into shared
+ * memory and the refill of the operand ring after the G_P product stall the tensor core once per
+ * tile, and the fused forward measured the same time as the two launches at the 8B shapes. */
 #define POETX_LAYER_FUSED_W0_P 4
 
 /* One POET-X linear. Every pointer is a device pointer owned by the caller. */
