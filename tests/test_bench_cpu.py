@@ -58,3 +58,19 @@ def test_cpu_baseline_reports_one_thread_blas_and_merge_extrapolation():
     ex = cb["extrapolated_with_merge"]
     assert ex["merge_reinit_s"] > 0 and "extrapolated" in ex["label"]
     assert 0 < ex["value"] < cb["value"]
+
+
+def test_other_configs_reports_a_failing_workload_without_failing():
+    """The default run's other_configs: each workload runs in a process of its own, and one that
+    fails (here an unknown workload name, rejected by the argument parser) is reported with its
+    exit status instead of ending the benchmark."""
+    sys.path.insert(0, ROOT)
+    import bench
+    saved = bench.OTHER_WORKLOADS
+    bench.OTHER_WORKLOADS = ("no_such_workload",)
+    try:
+        out = bench.other_configs(types.SimpleNamespace(steps=1, warmup=3))
+    finally:
+        bench.OTHER_WORKLOADS = saved
+    assert set(out) == {"no_such_workload"}
+    assert out["no_such_workload"]["error"].startswith("exit 2")
