@@ -200,6 +200,33 @@ def test_fused_w0_p_forward_matches_oracle_and_two_launch_forward(m, n, T):
     assert rel_err(y1, ref["Y"]) <= TOL_BF16
 
 
+def test_fused_w0_p_layer_full_steps_match_two_launch_layer():
+    """A whole step of the fused-forward layer, in both activation modes: with the saved A and B
+    (POET-Xfast) and with no B kept (POET-Xmem, B rebuilt by the backward), every output (Y, dX,
+    dq_r, dq_p) bit for bit that of the same layer without the flag."""
+    c = LayerCase("llama8b_up_proj", m=1024, n=2048, b=512, tokens=777, seed=4321)
+    f = _fused_twin(c)
+    T, m, n = c.T, c.layer.m, c.layer.n
+
+    def step(layer, keep_b):
+        y = torch.empty(T, n, dtype=c.dt, device="cuda")
+        a = torch.empty(T, m, dtype=c.dt, device="cuda")
+        bs = torch.empty(T, n, dtype=c.dt, device="cuda") if keep_b else None
+        poetx.linear_fwd(layer, c.x, y, bs, saved_a=a)
+        dx = torch.empty(T, m, dtype=c.dt, device="cuda")
+        dq_r, dq_p = torch.empty_like(c.q_r), torch.empty_like(c.q_p)
+        poetx.linear_bwd(layer, c.x, c.dy, bs, dx, dq_r, dq_p, saved_a=a)
+        return y, dx, dq_r, dq_p
+
+    for keep_b in (True, False):
+        ref = step(c.layer, keep_b)
+        got = step(f, keep_b)
+        torch.cuda.synchronize()
+        poetx.device_status()
+        for r, g in zip(ref, got):
+            assert torch.equal(r, g), keep_b
+
+
 @pytest.mark.slow
 def test_fused_w0_p_forward_many_tiles_per_cluster_matches_two_launch_forward():
     """16384 tokens x 8 P blocks: 512 tiles, several per CTA pair, so the ring, the B tile and
