@@ -153,6 +153,8 @@ def test_fp32_layer_shapes(m, n, b, T):
     ("llama8b_up_proj", 1024, 2048, 512, 1000),
     ("llama1p3b_attn", 768, 512, 256, 2049),
     ("llama8b_up_proj", 1024, 2048, 512, 2305),
+    ("llama8b_up_proj", 1024, 2048, 512, 1),     # b = 512 below one row tile: other kernels
+    ("llama8b_up_proj", 512, 1024, 512, 255),
 ])
 def test_bf16_layer_parity(key, m, n, b, T):
     _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), TOL_BF16)
