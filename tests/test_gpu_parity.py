@@ -165,6 +165,15 @@ def test_bf16_layer_parity(key, m, n, b, T):
     _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T), TOL_BF16)
 
 
+@pytest.mark.parametrize("key,m,n,b,T", [("llama8b_up_proj", 1024, 2048, 512, 600),
+                                         ("llama1p3b_attn", 1024, 512, 256, 333)])
+def test_bf16_layer_parity_with_grown_q(key, m, n, b, T):
+    """The layer with q four times the workloads' scale (as after many optimizer steps without
+    a merge): G further from the identity, larger Q^2..Q^4 terms in the forward and in every
+    product of the dq chain."""
+    _check_layer(LayerCase(key, m=m, n=n, b=b, tokens=T, q_scale=4.0), TOL_BF16)
+
+
 @pytest.mark.parametrize("key,m,n,b,T,tol", [
     ("llama8b_up_proj", 1024, 2048, 512, 2305, TOL_BF16),
     ("llama1p3b_attn", 1024, 1024, 256, 333, TOL_BF16),
