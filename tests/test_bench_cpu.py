@@ -34,12 +34,20 @@ def test_reference_line_has_the_contract_keys():
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
 
 
-def test_reference_config_is_the_gpu_arms_config():
+def test_reference_config_is_the_gpu_arms_config(capsys, monkeypatch):
+    """The reference arm prints the `config` object the GPU arm builds for the same workload
+    (one function builds both). The oracle step itself is stubbed here (its timing is not the
+    point; the first test runs it for real)."""
     sys.path.insert(0, ROOT)
     import bench
     import poetx_workloads as W
-    for key in ("llama8b_up_proj", "llama13b_layers"):
-        d = _run("--workload", key)
+    monkeypatch.setattr(bench, "oracle_step_sample", lambda wl, T, nlin=1: (1.0, None))
+    for key in ("llama8b_up_proj", "llama13b_layers", "llama8b_decoder", "llama1p3b_attn"):
+        capsys.readouterr()
+        assert bench.main(["--impl", "reference", "--workload", key, "--steps", "1",
+                           "--warmup", "0", "--ref-tokens", "8"]) == 0
+        lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+        d = json.loads(lines[-1])
         args = types.SimpleNamespace(tokens=None, all_linears=True, xq=False, xq_staged=False)
         assert d["config"] == bench.workload_config(W.WORKLOADS[key], args, 1), key
 
